@@ -1,0 +1,432 @@
+"""Benchmark of the gated delta rule chunked prefill on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--fwd-only]
+
+One step = one pass of the whole hot path over one batch of the synthetic
+workload: the chunked forward (prep + state propagation/output) followed by
+the chunked backward, all in libgdn.so's kernels. The default workload is the
+Qwen-style GDN prefill shape B=1, T=8192, Hq=16, Hv=32, K=V=128, bf16 q/k/v,
+fp32 gates and state. With N GPUs (torchrun) every rank runs its own copy of
+the workload (independent sequences: no collective on the data path) and the
+value is all ranks' tokens over the slowest rank's device time.
+
+Prints one JSON line (rank 0). `--impl reference` times the fp64 CPU oracle
+(the only reference this method has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN chunk-prefill fwd/bwd Mtokens/s and % of roofline (T=8192, Hv=32, K=V=128)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CHUNK = 64
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(w, tokens_per_seq=None):
+    """Algorithmic flops and bytes of one forward and one backward pass.
+
+    Bytes: inputs read once plus outputs written once. Flops: the dense
+    contractions of the 64-token chunked method, counting the q/k Gram
+    matrices once per qk head.
+      fwd per token: Hq*4CK + Hv*(2CK + 4CV + 6KV)
+      bwd per token: Hq*4CK + Hv*(14CK + 10CV + 18KV + 4C^2)
+    """
+    C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
+    ntok = w.B * w.T
+    N = w.varlen[0] if w.varlen else w.B
+    e = 2 if w.dtype == "bf16" else 4
+    f_fwd = ntok * (Hq * 4 * C * K + Hv * (2 * C * K + 4 * C * V + 6 * K * V))
+    f_bwd = ntok * (Hq * 4 * C * K + Hv * (14 * C * K + 10 * C * V + 18 * K * V + 4 * C * C))
+    qk = 2 * ntok * Hq * K * e
+    vv = ntok * Hv * V * e
+    gb = 2 * ntok * Hv * 4
+    st = N * Hv * K * V * 4
+    h0 = st if w.h0_std is not None else 0
+    b_fwd = qk + vv + gb + h0 + vv + st                       # q,k,v,g,beta,h0 -> o, final
+    # q,k,v,g,beta,h0,do,dht -> dq,dk,dv,dg,dbeta,dh0
+    b_bwd = (qk + vv + gb + h0 + vv + st) + (qk + vv + gb + st)
+    return dict(f_fwd=f_fwd, f_bwd=f_bwd, b_fwd=b_fwd, b_bwd=b_bwd, tokens=ntok)
+
+
+def kernel_bytes(name, w):
+    """Algorithmic bytes of one launch of a named kernel: the tensors that kernel
+    must read once and write once in this design."""
+    C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
+    ntok = w.B * w.T
+    N = w.varlen[0] if w.varlen else w.B
+    e = 2 if w.dtype == "bf16" else 4
+    nc = math.ceil(w.T / C) * w.B if not w.varlen else None
+    if nc is None:
+        nc = ntok // C + N  # upper bound for packed input
+    qk1 = ntok * Hq * K * e
+    v1 = ntok * Hv * V * e
+    gam = ntok * Hv * 4
+    ainv = nc * Hv * C * C * e
+    st = N * Hv * K * V * 4
+    h0 = st if w.h0_std is not None else 0
+    table = {
+        "prep_simt": qk1 + 2 * gam + gam + ainv,               # k, g, beta -> gamma, Ainv
+        "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
+    }
+    return table.get(name)
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gdn_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, w):
+    """fp64 CPU oracle timed on the host cores on a bounded sample of the workload."""
+    import oracle
+    from gated_deltanet_chunked_rule_b200.inputs import make_inputs, scaled
+    ws, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    sample_T = min(w.T, args.ref_tokens)
+    ws_ = scaled(w, T=sample_T, varlen=None)
+    x = make_inputs(scaled(ws_, grads=True))
+    cores = oracle.default_threads()
+    oracle.build()
+
+    def step():
+        oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], h0=x["h0"])
+        if not args.fwd_only:
+            oracle.bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["do"],
+                       dht=x["dht"], h0=x["h0"])
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t)
+    tok = ws_.B * ws_.T
+    ms = 1e3 * statistics.mean(times)
+    value = tok / (ms * 1e-3) / 1e6
+    sample = (f"first {sample_T} tokens of each of B={w.B} rows, all {w.Hv} heads; "
+              f"{'fwd' if args.fwd_only else 'fwd+bwd'} per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": sample_T, "Hq": w.Hq, "Hv": w.Hv,
+                   "K": w.K, "V": w.V, "step": "fwd" if args.fwd_only else "fwd+bwd"},
+        "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(args, w):
+    """The oracle, as it stands, on the GPU machine's host cores (bounded sample)."""
+    import oracle
+    from gated_deltanet_chunked_rule_b200.inputs import make_inputs, scaled
+    oracle.build()
+    sample_T = min(w.T, args.ref_tokens)
+    ws_ = scaled(w, T=sample_T, varlen=None, grads=True)
+    x = make_inputs(ws_)
+    t = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], h0=x["h0"])
+    if not args.fwd_only:
+        oracle.bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["do"], dht=x["dht"],
+                   h0=x["h0"])
+    dt = time.perf_counter() - t
+    tok = ws_.B * ws_.T
+    return {"value": tok / dt / 1e6, "unit": "Mtokens/s", "cores": oracle.default_threads(),
+            "kind": "oracle",
+            "sample": f"one {'fwd' if args.fwd_only else 'fwd+bwd'} pass over the first "
+                      f"{sample_T} tokens, all {w.Hv} heads ({dt:.2f} s wall)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen_prefill_t8192_hv32")
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, make_inputs, scaled
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import gated_deltanet_chunked_rule_b200 as gdn
+    from gated_deltanet_chunked_rule_b200 import _binding
+
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    gdn.lib()  # fail loudly if the extension is missing
+
+    wr = scaled(w, seed=w.seed + rank, grads=True)
+    xh = make_inputs(wr)
+    x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in xh.items()}
+    cu_host = xh["cu_seqlens"]
+    P = gdn.Problem(x["q"], x["v"], x["scale"], x["cu_seqlens"], cu_host)
+    ws_f = torch.empty(max(P.fwd_workspace_size(), 1), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(P.bwd_workspace_size(), 1), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(x["v"])
+
+    do_bwd = not args.fwd_only
+    if do_bwd:
+        try:
+            _, _, sv = gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                                      x["scale"], x["h0"], True, x["cu_seqlens"],
+                                                      cu_host, save_for_backward=True)
+            gdn.chunk_gated_delta_rule_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], sv, x["do"],
+                                           x["dht"], x["scale"], x["h0"], x["cu_seqlens"], cu_host)
+        except _binding.GdnError as e:
+            if e.code != _binding.GDN_ERR_UNSUPPORTED:
+                raise
+            do_bwd = False
+
+    def step(inp):
+        o_, fin_, sv_ = gdn.chunk_gated_delta_rule_fwd(
+            inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["scale"], inp["h0"], True,
+            inp["cu_seqlens"], cu_host, save_for_backward=do_bwd, workspace=ws_f, out=o)
+        if do_bwd:
+            grads = gdn.chunk_gated_delta_rule_bwd(
+                inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], sv_, inp["do"], inp["dht"],
+                inp["scale"], inp["h0"], inp["cu_seqlens"], cu_host, workspace=ws_b)
+            return o_, fin_, grads
+        return o_, fin_, None
+
+    # L2 flush buffer: 2x the L2 size, written between timed steps (outside the events).
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=dev)
+
+    def timed_steps(n, fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for a, b in ev:
+            flush.fill_(1.0)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        ms_list = timed_steps(args.steps, lambda: step(x))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = sum(ms_list)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    alg = algorithmic(w)
+    tokens = alg["tokens"]
+    ms_step = total_ms / args.steps
+    value = tokens * world * args.steps / (total_ms * 1e-3) / 1e6
+
+    # Per-kernel device times: a second pass of the same steps with the library's
+    # event timing on (events on the launch stream around every launch).
+    _binding.timing_enable(True)
+    timed_steps(args.steps, lambda: step(x))
+    rep = _binding.timing_report()
+    _binding.timing_enable(False)
+    launches_per_step = sum(v[0] for v in rep.values()) / args.steps
+    kern_total = sum(v[1] for v in rep.values())
+    kernels = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / v[0],
+                   "share": v[1] / kern_total if kern_total else None}
+               for k, v in rep.items()}
+    dom = max(rep, key=lambda k: rep[k][1])
+    pk, pk_kind = peaks()
+    dom_avg_s = rep[dom][1] / rep[dom][0] * 1e-3
+    dom_bytes = kernel_bytes(dom, w)
+    roofline = {"kernel": dom, "bound": "hbm", "unit": "GB/s",
+                "achieved": dom_bytes / dom_avg_s / 1e9 if dom_bytes else None,
+                "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)",
+                "traffic": None}
+    if roofline["achieved"]:
+        roofline["frac"] = roofline["achieved"] / roofline["peak"]
+
+    # Whole-chain roofline of the forward (and backward) against max(F/peak, B/peak).
+    fwd_ms = sum(v[1] for k, v in rep.items() if not k.startswith("bwd")) / args.steps
+    bwd_ms = sum(v[1] for k, v in rep.items() if k.startswith("bwd")) / args.steps
+
+    def chain(F, Bt, ms):
+        t_tc = F / (pk["bf16_tflops"] * 1e12)
+        t_hbm = Bt / (pk["hbm_gbs"] * 1e9)
+        return {"ms": ms, "Mtokens_s": tokens / (ms * 1e-3) / 1e6 if ms else None,
+                "tflops": F / (ms * 1e-3) / 1e12 if ms else None,
+                "gbs": Bt / (ms * 1e-3) / 1e9 if ms else None,
+                "bound_us": 1e6 * max(t_tc, t_hbm), "binding": "tensor" if t_tc > t_hbm else "hbm",
+                "frac": (1e3 * max(t_tc, t_hbm)) / ms if ms else None}
+
+    fwd_chain = chain(alg["f_fwd"], alg["b_fwd"], fwd_ms)
+    bwd_chain = chain(alg["f_bwd"], alg["b_bwd"], bwd_ms) if do_bwd else None
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the call, and D2H of its results, all inside the timing.
+    names_in = ["q", "k", "v", "g", "beta"] + (["h0"] if xh["h0"] is not None else []) + \
+        (["do", "dht"] if do_bwd else [])
+    host_in = {k: xh[k].pin_memory() for k in names_in}
+    dev_in = {k: torch.empty_like(x[k]) for k in names_in}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    host_out = {}
+
+    def e2e_step():
+        for k in names_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        inp = dict(x)
+        inp.update(dev_in)
+        o_, fin_, grads = step(inp)
+        outs = [o_, fin_] + (list(grads) if grads is not None else [])
+        for i, t in enumerate(outs):
+            if i not in host_out:
+                host_out[i] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            host_out[i].copy_(t, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = timed_steps(args.steps, e2e_step)
+    e2e_total = sum(e2e_ms)
+    if dist:
+        t = torch.tensor([e2e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e2e = {"value": tokens * world * args.steps / (e2e_total * 1e-3) / 1e6, "unit": "Mtokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    status = gdn.device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the bench")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args, w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hv": w.Hv, "K": w.K,
+                       "V": w.V, "chunk": CHUNK, "step": "fwd+bwd" if do_bwd else "fwd",
+                       "l2": "flushed between steps (2x L2 write, outside the events)",
+                       "parallelism": f"replicas x{world} (independent sequences per GPU)"},
+            "fwd": fwd_chain, "bwd": bwd_chain, "kernels": kernels, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

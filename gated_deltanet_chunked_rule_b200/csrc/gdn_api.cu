@@ -1,0 +1,374 @@
+// gdn_api.cu -- C ABI of the chunked gated delta rule library (see include/gdn.h).
+//
+// Host side only plans and launches: it validates the problem, lays the
+// caller's workspace out, builds (on the device, without a host sync) the
+// sequence table for packed variable-length input, and enqueues the kernels
+// on the caller's stream. It never allocates device memory.
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// Per-device status word: kernels record the first problem they meet here.
+__device__ unsigned g_status_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mutex;
+unsigned *g_status_ptr[kMaxDevices] = {};
+
+unsigned *status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mutex);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = (unsigned *)p;
+    }
+    return g_status_ptr[dev];
+}
+
+// ------------------------------------------------------------ kernel timing
+// While enabled, each launch is bracketed by two events on its stream.
+struct TimingRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {  // caller holds g_tmu
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+struct TimedLaunch {
+    const char *name;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    TimedLaunch(const char *n, cudaStream_t s) : name(n), st(s) {
+        std::lock_guard<std::mutex> lock(g_tmu);
+        if (!g_timing) return;
+        a = take_event();
+        if (a) cudaEventRecord(a, st);
+    }
+    ~TimedLaunch() {
+        if (!a) return;
+        std::lock_guard<std::mutex> lock(g_tmu);
+        cudaEvent_t b = take_event();
+        if (!b) return;
+        cudaEventRecord(b, st);
+        g_recs.push_back({name, a, b});
+    }
+};
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Validated problem summary computed on the host.
+struct Plan {
+    Dims d;
+    int dtype;
+    bool varlen;
+    size_t gamma_bytes, ainv_bytes, saved_bytes, seq_info_bytes;
+};
+
+int make_plan(const gdn_problem *p, Plan *out) {
+    if (!p) return GDN_ERR_INVALID_ARG;
+    if (p->dtype != GDN_DTYPE_F32 && p->dtype != GDN_DTYPE_BF16) return GDN_ERR_UNSUPPORTED;
+    if (p->B < 1 || p->T < 0 || p->Hq < 1 || p->Hv < 1 || p->K < 1 || p->V < 1)
+        return GDN_ERR_INVALID_ARG;
+    if (p->Hv % p->Hq) return GDN_ERR_INVALID_ARG;
+    if ((p->K != 64 && p->K != 128) || (p->V != 64 && p->V != 128)) return GDN_ERR_UNSUPPORTED;
+    if (!isfinite(p->scale)) return GDN_ERR_INVALID_ARG;
+    if (p->num_seqs < 0) return GDN_ERR_INVALID_ARG;
+    const long long ntok = (long long)p->B * p->T;
+    if (ntok > (1ll << 30)) return GDN_ERR_INVALID_ARG;  // token indices stay in int
+    Plan P;
+    memset(&P, 0, sizeof(P));
+    P.dtype = p->dtype;
+    P.varlen = p->num_seqs > 0;
+    Dims &d = P.d;
+    d.B = p->B; d.T = p->T; d.Hq = p->Hq; d.Hv = p->Hv; d.K = p->K; d.V = p->V;
+    d.T_total = (int)ntok;
+    d.scale = p->scale;
+    d.seq_info = nullptr;
+    if (P.varlen) {
+        if (p->B != 1 || !p->cu_seqlens || !p->cu_seqlens_host) return GDN_ERR_INVALID_ARG;
+        const int32_t *cu = p->cu_seqlens_host;
+        if (cu[0] != 0 || cu[p->num_seqs] != p->T) return GDN_ERR_INVALID_ARG;
+        long long nc = 0;
+        for (int n = 0; n < p->num_seqs; ++n) {
+            if (cu[n + 1] < cu[n]) return GDN_ERR_INVALID_ARG;
+            nc += (cu[n + 1] - cu[n] + kChunk - 1) / kChunk;
+        }
+        d.N = p->num_seqs;
+        d.NC = (int)nc;
+        P.seq_info_bytes = align_up(sizeof(int) * (3 * (size_t)d.N + 1));
+    } else {
+        d.N = p->B;
+        d.NC = p->B * ((p->T + kChunk - 1) / kChunk);
+    }
+    P.gamma_bytes = align_up(sizeof(float) * (size_t)d.T_total * d.Hv);
+    P.ainv_bytes = align_up((size_t)d.NC * d.Hv * kChunk * kChunk *
+                            (p->dtype == GDN_DTYPE_F32 ? sizeof(float) : sizeof(__nv_bfloat16)));
+    P.saved_bytes = P.gamma_bytes + P.ainv_bytes;
+    *out = P;
+    return GDN_OK;
+}
+
+size_t fwd_ws_bytes(const Plan &P) {
+    // sequence table + gamma/Ainv (used when the caller passes no `saved`)
+    return P.seq_info_bytes + P.saved_bytes;
+}
+
+size_t bwd_ws_bytes(const Plan &P) {
+    const Dims &d = P.d;
+    const size_t hc = align_up(sizeof(float) * (size_t)d.NC * d.Hv * d.K * d.V);
+    const size_t dl = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.V);
+    return P.seq_info_bytes + P.saved_bytes + 2 * hc + 2 * dl;
+}
+
+// Builds the sequence table from the device copy of cu_seqlens and checks it
+// against the host plan (total tokens, total chunks). On any disagreement it
+// writes an empty table (no sequence has tokens, so later kernels do nothing)
+// and records GDN_ERR_DEVICE_ARG in the status word.
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ cu, int N, int T_total,
+                                                    int NC_expected, int *__restrict__ info,
+                                                    unsigned *status) {
+    __shared__ int ok;
+    __shared__ int carry;
+    __shared__ int warp_sums[32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) {
+        ok = (cu[0] == 0 && cu[N] == T_total) ? 1 : 0;
+        carry = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + tid;
+        int nch = 0;
+        if (n < N) {
+            const int a = cu[n], b = cu[n + 1];
+            if (b < a || a < 0 || b > T_total) ok = 0;
+            const int len = b > a ? b - a : 0;
+            nch = (len + kChunk - 1) / kChunk;
+            info[n] = a;
+            info[N + n] = len;
+        }
+        // block-wide inclusive scan of nch
+        int x = nch;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int s = warp_sums[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += y;
+            }
+            warp_sums[lane] = s;
+        }
+        __syncthreads();
+        const int incl = x + (wid > 0 ? warp_sums[wid - 1] : 0);
+        if (n < N) info[2 * N + n] = carry + incl - nch;
+        __syncthreads();
+        if (tid == 1023) carry += incl;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        info[3 * N] = carry;
+        if (carry != NC_expected) ok = 0;
+    }
+    __syncthreads();
+    if (!ok) {
+        for (int e = tid; e < 3 * N + 1; e += 1024) info[e] = 0;
+        if (tid == 0) set_status(status, GDN_ERR_DEVICE_ARG);
+    }
+}
+
+bool use_simt(int dtype) {
+    if (dtype == GDN_DTYPE_F32) return true;
+    const char *e = getenv("GDN_IMPL");
+    return e && strcmp(e, "simt") == 0;
+}
+
+int launch_plan(const gdn_problem *p, Plan &P, char *ws, unsigned *status, cudaStream_t st) {
+    if (!P.varlen) return GDN_OK;
+    int *info = (int *)ws;
+    TimedLaunch t("plan", st);
+    plan_kernel<<<1, 1024, 0, st>>>(p->cu_seqlens, P.d.N, P.d.T_total, P.d.NC, info, status);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+    P.d.seq_info = info;
+    return GDN_OK;
+}
+
+}  // namespace
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+size_t gdn_fwd_workspace_size(const gdn_problem *p) {
+    Plan P;
+    return make_plan(p, &P) == GDN_OK ? fwd_ws_bytes(P) : 0;
+}
+
+size_t gdn_bwd_workspace_size(const gdn_problem *p) {
+    Plan P;
+    return make_plan(p, &P) == GDN_OK ? bwd_ws_bytes(P) : 0;
+}
+
+size_t gdn_saved_size(const gdn_problem *p) {
+    Plan P;
+    return make_plan(p, &P) == GDN_OK ? P.saved_bytes : 0;
+}
+
+int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, const float *h0, void *o,
+                  float *final_state, void *saved, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+    Plan P;
+    int rc = make_plan(p, &P);
+    if (rc != GDN_OK) return rc;
+    const bool has_tokens = P.d.T_total > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, final_state, saved};
+    for (const void *x : ptrs)
+        if (x && !aligned16(x)) return GDN_ERR_INVALID_ARG;
+    const size_t need = fwd_ws_bytes(P);
+    if (workspace_bytes < need || (need && !workspace) || ((uintptr_t)workspace & 255u))
+        return GDN_ERR_WORKSPACE;
+    if (saved && ((uintptr_t)saved & 255u)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned *status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    char *ws = (char *)workspace;
+    if ((rc = launch_plan(p, P, ws, status, st)) != GDN_OK) return rc;
+    char *sv = saved ? (char *)saved : ws + P.seq_info_bytes;
+
+    FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.d = P.d;
+    a.dtype = P.dtype;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0;
+    a.o = o; a.final_state = final_state;
+    a.gamma = (float *)sv;
+    a.ainv = sv + P.gamma_bytes;
+    a.status = status;
+    a.stream = st;
+    a.nseg = 1;
+    (void)use_simt;
+    {
+        TimedLaunch t("prep_simt", st);
+        if (launch_prep_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    {
+        TimedLaunch t("fwd_simt", st);
+        if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
+}
+
+int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, const float *h0, const void *saved,
+                  const void *d_o, const float *dht, void *dq, void *dk, void *dv, float *dg,
+                  float *dbeta, float *dh0, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+    Plan P;
+    int rc = make_plan(p, &P);
+    if (rc != GDN_OK) return rc;
+    (void)q; (void)k; (void)v; (void)g; (void)beta; (void)h0; (void)saved; (void)d_o;
+    (void)dht; (void)dq; (void)dk; (void)dv; (void)dg; (void)dbeta; (void)dh0;
+    (void)workspace; (void)workspace_bytes; (void)stream;
+    return GDN_ERR_UNSUPPORTED;
+}
+
+int gdn_get_device_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v)) != cudaSuccess) return GDN_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    return (int)v;
+}
+
+int gdn_timing_enable(int on) {
+    std::lock_guard<std::mutex> lock(g_tmu);
+    for (auto &r : g_recs) {
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_recs.clear();
+    g_timing = on != 0;
+    return GDN_OK;
+}
+
+int gdn_timing_report(char *buf, size_t buf_len) {
+    std::lock_guard<std::mutex> lock(g_tmu);
+    std::vector<std::pair<std::string, std::pair<int, double>>> agg;
+    for (auto &r : g_recs) {
+        if (cudaEventSynchronize(r.b) != cudaSuccess) return -GDN_ERR_CUDA;
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return -GDN_ERR_CUDA;
+        size_t i = 0;
+        while (i < agg.size() && agg[i].first != r.name) ++i;
+        if (i == agg.size()) agg.push_back({r.name, {0, 0.0}});
+        agg[i].second.first += 1;
+        agg[i].second.second += ms;
+    }
+    std::string out = "{";
+    for (size_t i = 0; i < agg.size(); ++i) {
+        char item[256];
+        snprintf(item, sizeof(item), "%s\"%s\": [%d, %.6f]", i ? ", " : "", agg[i].first.c_str(),
+                 agg[i].second.first, agg[i].second.second);
+        out += item;
+    }
+    out += "}";
+    if (buf && buf_len) {
+        const size_t n = out.size() < buf_len - 1 ? out.size() : buf_len - 1;
+        memcpy(buf, out.data(), n);
+        buf[n] = 0;
+    }
+    return (int)out.size();
+}
+
+const char *gdn_status_string(int s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_DEVICE_ARG: return "GDN_ERR_DEVICE_ARG";
+        default: return "GDN_ERR_UNKNOWN";
+    }
+}
+
+const char *gdn_version(void) { return "gdn-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule chunked-prefill library.
+ *
+ * The operation (per sequence n and value head h, qk head hq = h / (Hv/Hq)):
+ *
+ *   S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   o_t = scale * S_t q_t                      state S in R^{V x K}
+ *
+ * computed chunk-parallel (64-token chunks, WY form of the delta rule). The
+ * entry points follow the FlashQLA write-up's statement of the problem:
+ *   - gdn_chunk_fwd mirrors chunk_gated_delta_rule / chunk_gated_delta_rule_fwd
+ *     (page 1, "高级 API 示例" and "底层 API": q, k, v, g, beta, scale,
+ *     initial_state, output_final_state, cu_seqlens -> o, final_state, plus
+ *     the in-chunk cumulative gate "g" and the chunk matrix "A" it returns);
+ *   - gdn_chunk_bwd mirrors chunk_gated_delta_rule_bwd (page 1, "底层 API":
+ *     q, k, v, g, beta, A, do, dht, scale, initial_state, cu_seqlens ->
+ *     dq, dk, dv, db, dg, dh0);
+ *   - the automatic intra-GPU sequence split inside gdn_chunk_fwd is the
+ *     "gate-driven automatic intra-card context parallelism" of page 2
+ *     ("三大关键特性" table, first row), realised exactly (no truncation).
+ *
+ * Layouts (contiguous, row-major, device memory unless stated):
+ *   q, k        [B, T, Hq, K]   dtype (GDN_DTYPE_F32 or GDN_DTYPE_BF16)
+ *   v, o, do    [B, T, Hv, V]   dtype
+ *   g, beta     [B, T, Hv]      fp32. g is the per-token LOG decay (<= 0 in
+ *                               practice; any finite value is accepted),
+ *                               beta the delta-rule write strength.
+ *   h0, final_state, dht, dh0
+ *               [N, Hv, K, V]   fp32, h = S^T (row index over K, column over V).
+ *                               N = B, or num_seqs with cu_seqlens.
+ *   cu_seqlens  int32 [num_seqs + 1]: cu[0] = 0, non-decreasing, cu[N] = T,
+ *               B must be 1. Sequences are packed along T; each starts from
+ *               its own h0[n] and ends in its own final_state[n]. A
+ *               zero-length sequence gives final_state[n] = h0[n].
+ *   dq, dk      [B, T, Hq, K]   dtype; each sums the value heads of its group.
+ *   dv          [B, T, Hv, V]   dtype.
+ *   dg, dbeta   [B, T, Hv]      fp32; dg is w.r.t. the raw per-token g.
+ *
+ * Supported sizes: K, V in {64, 128}; Hv a multiple of Hq; T >= 0; B >= 1.
+ *
+ * Ownership and synchronisation: every pointer is caller-owned. The library
+ * never allocates, frees or synchronises (except gdn_get_device_status); it
+ * enqueues its kernels on the caller's stream and keeps no state between
+ * calls other than the device status word. Scratch memory comes from the
+ * caller's workspace (sizes from the *_workspace_size queries, 256-byte
+ * aligned pointer required). All pointers must be 16-byte aligned.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued;
+ * a rejected call enqueues nothing. Device-side problems (an inconsistent
+ * device copy of cu_seqlens, a bounded wait that expired) are recorded in a
+ * per-device status word read by gdn_get_device_status; the kernels then do
+ * no further work for that call and return, they never trap.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, Hv % Hq != 0, bad cu_seqlens, ... */
+    GDN_ERR_UNSUPPORTED = 2,  /* K or V not in {64,128}, unknown dtype                     */
+    GDN_ERR_WORKSPACE = 3,    /* workspace too small or misaligned                          */
+    GDN_ERR_CUDA = 4,         /* a CUDA launch or query failed                              */
+    GDN_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (status word)           */
+    GDN_ERR_DEVICE_ARG = 6    /* device copy of cu_seqlens disagrees with the host copy     */
+} gdn_status;
+
+typedef enum { GDN_DTYPE_F32 = 0, GDN_DTYPE_BF16 = 1 } gdn_dtype;
+
+typedef struct {
+    int B, T, Hq, Hv, K, V;
+    int num_seqs;                   /* 0: no packing (N = B); else B == 1 and cu_seqlens given */
+    const int32_t *cu_seqlens;      /* device, [num_seqs + 1], or NULL when num_seqs == 0       */
+    const int32_t *cu_seqlens_host; /* the same values in host memory (planning without a sync) */
+    int dtype;                      /* gdn_dtype of q, k, v, o, do, dq, dk, dv                  */
+    float scale;                    /* any finite value; 1/sqrt(K) is the usual choice          */
+} gdn_problem;
+
+/* Bytes of caller-provided scratch that gdn_chunk_fwd / gdn_chunk_bwd need
+ * for this problem (0 if the problem is invalid). */
+size_t gdn_fwd_workspace_size(const gdn_problem *p);
+size_t gdn_bwd_workspace_size(const gdn_problem *p);
+
+/* Bytes of the "saved" buffer: the in-chunk cumulative gate gamma (fp32
+ * [B*T, Hv]) followed by Ainv = (I + A)^-1 of every 64-token chunk
+ * ([num_chunks, Hv, 64, 64], fp32 for GDN_DTYPE_F32 problems, bf16 for
+ * GDN_DTYPE_BF16), i.e. the "g, A" that page 1's low-level forward returns
+ * and its backward takes back. */
+size_t gdn_saved_size(const gdn_problem *p);
+
+/* Forward. h0 may be NULL (zero initial state); final_state may be NULL (not
+ * written); saved may be NULL (not written). o must not be NULL. */
+int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, const float *h0, void *o,
+                  float *final_state, void *saved, void *workspace, size_t workspace_bytes,
+                  void *stream /* cudaStream_t */);
+
+/* Backward. h0 and dht may be NULL (zero); saved may be NULL (gamma and Ainv
+ * are then recomputed) or the buffer a gdn_chunk_fwd call with the same
+ * problem and inputs filled; dh0 may be NULL (not written). The other
+ * outputs must not be NULL. */
+int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                  const float *g, const float *beta, const float *h0, const void *saved,
+                  const void *d_o, const float *dht, void *dq, void *dk, void *dv, float *dg,
+                  float *dbeta, float *dh0, void *workspace, size_t workspace_bytes,
+                  void *stream /* cudaStream_t */);
+
+/* Synchronises `stream`, then returns and clears the current device's status
+ * word (GDN_OK if no kernel recorded a problem since the last call). */
+int gdn_get_device_status(void *stream /* cudaStream_t */);
+
+/* Kernel timing (tracing). While enabled (on != 0), every kernel launch the
+ * library makes is bracketed by a pair of CUDA events recorded on the launch
+ * stream. gdn_timing_report synchronises the device, then writes into buf a
+ * JSON object {"<kernel>": [launches, total_ms], ...} covering every launch
+ * since the last enable/reset, and returns the number of bytes needed
+ * (excluding the terminating NUL; the output is truncated if buf_len is too
+ * small), or minus a gdn_status code on failure. Enabling clears earlier records. The events come from a pool the
+ * library creates on first use; it holds no device memory. Timing changes
+ * nothing in the results; it adds a few microseconds per launch. */
+int gdn_timing_enable(int on);
+int gdn_timing_report(char *buf, size_t buf_len);
+
+/* Static, human-readable name of a status code. */
+const char *gdn_status_string(int status);
+
+/* Library build identifier (sm_100a kernels compiled in). */
+const char *gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,114 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/gdn.h declares, sizes workspaces, and rejects bad arguments before it
+touches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_chunked_rule_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_deltanet_chunked_rule_b200 import build
+    build.build()
+    return B.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = header_functions()
+    assert set(declared) == set(B.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in [(0, "GDN_OK"), (1, "GDN_ERR_INVALID_ARG"), (2, "GDN_ERR_UNSUPPORTED"),
+                       (3, "GDN_ERR_WORKSPACE"), (4, "GDN_ERR_CUDA"), (5, "GDN_ERR_TIMEOUT"),
+                       (6, "GDN_ERR_DEVICE_ARG")]:
+        assert B.status_string(code) == name
+    assert B.status_string(99) == "GDN_ERR_UNKNOWN"
+    assert b"sm_100a" in L.gdn_version()
+
+
+def prob(B_=1, T=256, Hq=2, Hv=4, K=128, V=128, ns=0, cu=None, dtype=1, scale=0.1):
+    arr = None
+    if cu is not None:
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+    p = B.gdn_problem(B_, T, Hq, Hv, K, V, ns, ctypes.cast(arr, ctypes.c_void_p) if arr else None,
+                      ctypes.cast(arr, ctypes.c_void_p) if arr else None, dtype, scale)
+    p._keep = arr
+    return p
+
+
+def test_workspace_sizes(L):
+    p = prob()
+    nc = 4  # 256 tokens -> 4 chunks
+    gamma = 256 * 4 * 4
+    ainv = nc * 4 * 64 * 64 * 2
+    assert L.gdn_saved_size(ctypes.byref(p)) == gamma + ainv
+    assert L.gdn_fwd_workspace_size(ctypes.byref(p)) >= gamma + ainv
+    assert L.gdn_bwd_workspace_size(ctypes.byref(p)) > L.gdn_fwd_workspace_size(ctypes.byref(p))
+    p32 = prob(dtype=0)
+    assert L.gdn_saved_size(ctypes.byref(p32)) == gamma + 2 * ainv
+    # ragged varlen: lengths 100, 0, 28, 128 -> 2 + 0 + 1 + 2 chunks
+    pv = prob(T=256, ns=4, cu=[0, 100, 100, 128, 256])
+    assert L.gdn_saved_size(ctypes.byref(pv)) == gamma + 5 * 4 * 64 * 64 * 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=3, Hv=4), B.GDN_ERR_INVALID_ARG),
+    (dict(K=96), B.GDN_ERR_UNSUPPORTED),
+    (dict(V=256), B.GDN_ERR_UNSUPPORTED),
+    (dict(dtype=7), B.GDN_ERR_UNSUPPORTED),
+    (dict(B_=0), B.GDN_ERR_INVALID_ARG),
+    (dict(T=-1), B.GDN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), B.GDN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), B.GDN_ERR_INVALID_ARG),
+    (dict(B_=2, ns=2, cu=[0, 100, 256]), B.GDN_ERR_INVALID_ARG),   # varlen needs B == 1
+    (dict(ns=2, cu=[0, 300, 256]), B.GDN_ERR_INVALID_ARG),         # decreasing
+    (dict(ns=2, cu=[0, 100, 200]), B.GDN_ERR_INVALID_ARG),         # cu[N] != T
+    (dict(ns=2, cu=[5, 100, 256]), B.GDN_ERR_INVALID_ARG),         # cu[0] != 0
+])
+def test_invalid_problems_rejected_before_any_launch(L, kw, code):
+    p = prob(**kw)
+    assert L.gdn_fwd_workspace_size(ctypes.byref(p)) == 0
+    assert L.gdn_bwd_workspace_size(ctypes.byref(p)) == 0
+    assert L.gdn_saved_size(ctypes.byref(p)) == 0
+    dummy = ctypes.c_void_p(1 << 20)
+    rc = L.gdn_chunk_fwd(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy, None, dummy, None,
+                         None, dummy, 1 << 40, None)
+    assert rc == code
+    rc = L.gdn_chunk_bwd(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy, None, None, dummy,
+                         None, dummy, dummy, dummy, dummy, dummy, None, dummy, 1 << 40, None)
+    assert rc == code
+    assert L.gdn_chunk_fwd(None, dummy, dummy, dummy, dummy, dummy, None, dummy, None, None,
+                           dummy, 0, None) == B.GDN_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    p = prob()
+    d = ctypes.c_void_p(1 << 20)
+    ws = L.gdn_fwd_workspace_size(ctypes.byref(p))
+    # o missing
+    assert L.gdn_chunk_fwd(ctypes.byref(p), d, d, d, d, d, None, None, None, None, d, ws,
+                           None) == B.GDN_ERR_INVALID_ARG
+    # misaligned q
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    assert L.gdn_chunk_fwd(ctypes.byref(p), bad, d, d, d, d, None, d, None, None, d, ws,
+                           None) == B.GDN_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert L.gdn_chunk_fwd(ctypes.byref(p), d, d, d, d, d, None, d, None, None, d, ws - 1,
+                           None) == B.GDN_ERR_WORKSPACE
+    assert L.gdn_chunk_fwd(ctypes.byref(p), d, d, d, d, d, None, d, None, None,
+                           ctypes.c_void_p((1 << 20) + 16), ws, None) == B.GDN_ERR_WORKSPACE

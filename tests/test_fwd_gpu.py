@@ -1,0 +1,128 @@
+"""Forward parity on the GPU: CUDA path (through the C ABI) vs the fp64 oracle,
+element by element on the same seeded inputs."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, Workload, make_inputs, scaled
+from parity_util import check_fwd, f64, gpu_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gated_deltanet_chunked_rule_b200 import build
+    build.build()
+
+
+def run(oracle_mod, w, label=None, **kw):
+    x = make_inputs(w)
+    o, fin, _ = gpu_fwd(x, **kw)
+    e = check_fwd(oracle_mod, x, o, fin, label or w.name)
+    print(f"[parity] {label or w.name}: o err {e[0]:.3e}  final err {e[1]:.3e}")
+    return x, o, fin
+
+
+def test_tiny_fp32_workload(oracle_mod):
+    run(oracle_mod, WORKLOADS["tiny_fp32"])
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("K,V", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_small_ragged_shapes(oracle_mod, dtype, K, V):
+    # several chunks plus a ragged tail (200 = 3*64 + 8), batch rows, GQA, nonzero h0
+    w = Workload(f"small_{dtype}_{K}x{V}", B=2, T=200, Hq=2, Hv=4, K=K, V=V, dtype=dtype,
+                 h0_std=0.02, seed=K + V)
+    run(oracle_mod, w)
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 129])
+def test_chunk_boundaries(oracle_mod, T):
+    w = Workload(f"edge_T{T}", B=1, T=T, Hq=1, Hv=2, K=128, V=128, h0_std=0.02, seed=T)
+    run(oracle_mod, w)
+
+
+def test_empty_batch_keeps_initial_state():
+    import gated_deltanet_chunked_rule_b200 as gdn
+    w = Workload("empty", B=2, T=0, Hq=1, Hv=2, K=64, V=64, h0_std=0.02)
+    x = to_dev(make_inputs(w))
+    o, fin, _ = gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                               x["scale"], initial_state=x["h0"])
+    torch.cuda.synchronize()
+    assert o.numel() == 0
+    torch.testing.assert_close(fin, x["h0"], rtol=0, atol=0)
+
+
+def test_varlen_with_empty_and_ragged_sequences(oracle_mod):
+    w = Workload("varlen_small", B=1, T=700, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, seed=3)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 0, 65, 130, 130, 192, 700], dtype=torch.int32)
+    x["h0"] = 0.02 * torch.randn((6, 4, 128, 128), generator=torch.Generator().manual_seed(1))
+    o, fin, _ = gpu_fwd(x)
+    check_fwd(oracle_mod, x, o, fin, "varlen_small")
+    # empty sequences: final state is the initial state, bit for bit
+    torch.testing.assert_close(fin[0].cpu(), x["h0"][0], rtol=0, atol=0)
+    torch.testing.assert_close(fin[3].cpu(), x["h0"][3], rtol=0, atol=0)
+
+
+def test_varlen_equals_separate_calls():
+    w = Workload("varlen_sep", B=1, T=400, Hq=1, Hv=2, K=128, V=128, h0_std=0.02, seed=4)
+    x = make_inputs(w)
+    cu = [0, 100, 250, 400]
+    x["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
+    x["h0"] = 0.02 * torch.randn((3, 2, 128, 128), generator=torch.Generator().manual_seed(2))
+    o, fin, _ = gpu_fwd(x)
+    for n in range(3):
+        a, b = cu[n], cu[n + 1]
+        xs = {k: v for k, v in x.items()}
+        for key in ("q", "k", "v", "g", "beta"):
+            xs[key] = x[key][:, a:b].contiguous()
+        xs["h0"] = x["h0"][n:n + 1].contiguous()
+        xs["cu_seqlens"] = None
+        on, fn, _ = gpu_fwd(xs)
+        torch.testing.assert_close(on, o[:, a:b], rtol=0, atol=0)
+        torch.testing.assert_close(fn, fin[n:n + 1], rtol=0, atol=0)
+
+
+def test_gqa_equals_repeated_heads():
+    w = Workload("gqa", B=1, T=300, Hq=2, Hv=6, K=128, V=128, h0_std=0.02, seed=5)
+    x = make_inputs(w)
+    o, fin, _ = gpu_fwd(x)
+    xr = dict(x)
+    xr["q"] = x["q"].repeat_interleave(3, dim=2).contiguous()
+    xr["k"] = x["k"].repeat_interleave(3, dim=2).contiguous()
+    o2, fin2, _ = gpu_fwd(xr)
+    torch.testing.assert_close(o, o2, rtol=0, atol=0)
+    torch.testing.assert_close(fin, fin2, rtol=0, atol=0)
+
+
+def test_deterministic_run_to_run():
+    w = Workload("det", B=1, T=1000, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, seed=6)
+    x = make_inputs(w)
+    a = gpu_fwd(x)
+    b = gpu_fwd(x)
+    torch.testing.assert_close(a[0], b[0], rtol=0, atol=0)
+    torch.testing.assert_close(a[1], b[1], rtol=0, atol=0)
+
+
+def test_device_cu_seqlens_mismatch_reports_status():
+    import gated_deltanet_chunked_rule_b200 as gdn
+    w = Workload("mismatch", B=1, T=128, Hq=1, Hv=1, K=64, V=64, seed=7)
+    x = to_dev(make_inputs(w))
+    host = torch.tensor([0, 64, 128], dtype=torch.int32)
+    dev = torch.tensor([0, 100, 128], dtype=torch.int32, device="cuda")  # 2+1 chunks != 1+1
+    gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"],
+                                   cu_seqlens=dev, cu_seqlens_host=host)
+    assert gdn.device_status() == 6  # GDN_ERR_DEVICE_ARG
+    assert gdn.device_status() == 0  # cleared by the read
+
+
+@pytest.mark.parametrize("name", ["qwen_prefill_t8192_hv32", "long_split_t65536_h8",
+                                  "varlen_16seq_32k_h32"])
+def test_full_size_workloads(oracle_mod, name):
+    run(oracle_mod, WORKLOADS[name])
