@@ -141,12 +141,32 @@ size_t fwd_ws_bytes(const Plan &P) {
     return P.seq_info_bytes + P.saved_bytes;
 }
 
-size_t bwd_ws_bytes(const Plan &P) {
+// Backward workspace: sequence table | gamma, Ainv (when no `saved`) | per-chunk
+// entry states h | per-chunk exit-state gradients dh' | Delta | dDelta |
+// per-value-head fp32 partials of dq and dk.
+struct BwdLayout {
+    size_t seq, saved, hc, dhc, delta, ddelta, dqp, dkp, total;
+};
+
+BwdLayout bwd_layout(const Plan &P) {
     const Dims &d = P.d;
+    BwdLayout L;
     const size_t hc = align_up(sizeof(float) * (size_t)d.NC * d.Hv * d.K * d.V);
     const size_t dl = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.V);
-    return P.seq_info_bytes + P.saved_bytes + 2 * hc + 2 * dl;
+    const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
+    L.seq = 0;
+    L.saved = L.seq + P.seq_info_bytes;
+    L.hc = L.saved + P.saved_bytes;
+    L.dhc = L.hc + hc;
+    L.delta = L.dhc + hc;
+    L.ddelta = L.delta + dl;
+    L.dqp = L.ddelta + dl;
+    L.dkp = L.dqp + qp;
+    L.total = L.dkp + qp;
+    return L;
 }
+
+size_t bwd_ws_bytes(const Plan &P) { return bwd_layout(P).total; }
 
 // Builds the sequence table from the device copy of cu_seqlens and checks it
 // against the host plan (total tokens, total chunks). On any disagreement it
@@ -301,10 +321,64 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     Plan P;
     int rc = make_plan(p, &P);
     if (rc != GDN_OK) return rc;
-    (void)q; (void)k; (void)v; (void)g; (void)beta; (void)h0; (void)saved; (void)d_o;
-    (void)dht; (void)dq; (void)dk; (void)dv; (void)dg; (void)dbeta; (void)dh0;
-    (void)workspace; (void)workspace_bytes; (void)stream;
-    return GDN_ERR_UNSUPPORTED;
+    const bool has_tokens = P.d.T_total > 0;
+    if (has_tokens && (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, h0, saved, d_o, dht, dq, dk, dv, dg, dbeta, dh0};
+    for (const void *x : ptrs)
+        if (x && !aligned16(x)) return GDN_ERR_INVALID_ARG;
+    const BwdLayout L = bwd_layout(P);
+    if (workspace_bytes < L.total || (L.total && !workspace) || ((uintptr_t)workspace & 255u))
+        return GDN_ERR_WORKSPACE;
+    if (saved && ((uintptr_t)saved & 255u)) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned *status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    char *ws = (char *)workspace;
+    if ((rc = launch_plan(p, P, ws, status, st)) != GDN_OK) return rc;
+
+    FwdArgs f;
+    memset(&f, 0, sizeof(f));
+    f.d = P.d;
+    f.dtype = P.dtype;
+    f.q = q; f.k = k; f.v = v; f.g = g; f.beta = beta; f.h0 = h0;
+    f.status = status;
+    f.stream = st;
+    f.nseg = 1;
+    char *sv = saved ? (char *)saved : ws + L.saved;
+    f.gamma = (float *)sv;
+    f.ainv = sv + P.gamma_bytes;
+    f.h_chunks = (float *)(ws + L.hc);
+    f.delta = (float *)(ws + L.delta);
+    if (!saved) {
+        TimedLaunch t("prep_simt", st);
+        if (launch_prep_simt(f) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    {
+        TimedLaunch t("bwd_recompute_simt", st);
+        if (launch_fwd_simt(f) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    BwdArgs b;
+    memset(&b, 0, sizeof(b));
+    b.d = P.d;
+    b.dtype = P.dtype;
+    b.q = q; b.k = k; b.v = v; b.d_o = d_o;
+    b.g = g; b.beta = beta; b.h0 = h0; b.dht = dht;
+    b.gamma = f.gamma;
+    b.ainv = f.ainv;
+    b.h_chunks = f.h_chunks;
+    b.delta = f.delta;
+    b.dh_chunks = (float *)(ws + L.dhc);
+    b.ddelta = (float *)(ws + L.ddelta);
+    b.dq = dq; b.dk = dk; b.dv = dv; b.dg = dg; b.dbeta = dbeta; b.dh0 = dh0;
+    b.status = status;
+    b.stream = st;
+    {
+        TimedLaunch t("bwd_simt", st);
+        if (launch_bwd_simt(b, (float *)(ws + L.dqp), (float *)(ws + L.dkp)) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    return GDN_OK;
 }
 
 int gdn_get_device_status(void *stream) {

@@ -131,6 +131,6 @@ struct BwdArgs {
 // Launchers (return a cudaError_t of the launch).
 cudaError_t launch_prep_simt(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
-cudaError_t launch_bwd_simt(const BwdArgs &a);
+cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part);
 
 }  // namespace gdn

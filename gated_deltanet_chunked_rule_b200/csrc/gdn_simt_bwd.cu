@@ -1,0 +1,521 @@
+// gdn_simt_bwd.cu -- CUDA-core (fp32) backward of the chunked gated delta rule.
+//
+// Per chunk (rows r, s; chunk-entry state h, exit state h', see gdn_internal.cuh),
+// given dO and dh' (the gradient w.r.t. h'), the adjoint of the forward steps is
+//
+//   dDelta = scale (M o QK^T)^T dO + Ktil dh'                      (C x V)
+//   dh     = scale Q^T diag(e^gamma) dO + e^{gamma_C} dh' - w^T dDelta   (K x V)
+//   dU     = Ainv^T dDelta                                          (C x V)
+//   dv     = diag(beta) dU
+//   dKb    = -dU h^T,   dA = -(dU Delta^T) restricted to s < r
+//
+// The last two lines use (I + A) Delta = diag(beta) V - diag(beta e^gamma) K h:
+// the adjoint of Ainv = (I + A)^-1 applied to dAinv = dDelta ((I + A) Delta)^T
+// collapses to -Ainv^T dDelta Delta^T, so no second product with Ainv is needed.
+// The remaining terms (q/k Gram masks, decay factors) follow by the chain rule;
+// dg is the in-chunk reverse cumulative sum of d(gamma).
+//
+// Kernels:
+//   bwd_dh_simt     one CTA per (sequence, value head, 32-column slice): walks
+//                   the chunks backwards carrying dh[:, slice], stores dh' of
+//                   every chunk and dDelta, ends with dh0.
+//   bwd_grad_simt   one CTA per (chunk, value head): all per-chunk gradients;
+//                   dq and dk go to per-value-head fp32 partials.
+//   bwd_final       sums the partials over each qk head's group of value heads
+//                   in a fixed order and casts dq, dk to the input dtype.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBV = 32;
+
+// ------------------------------------------------------------ reverse dh scan
+template <int K>
+constexpr size_t dh_smem_floats() {
+    return (size_t)K * kBV + 3 * (size_t)kChunk * (K + 1) + 2 * (size_t)kChunk * 65 +
+           2 * (size_t)kChunk * (kBV + 1) + 3 * kChunk;
+}
+
+template <typename Tin, typename TA, int K, int V>
+__global__ void __launch_bounds__(kThreads) bwd_dh_simt(
+    Dims d, const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ d_o,
+    const float *__restrict__ gamma, const float *__restrict__ beta, const TA *__restrict__ ainv,
+    const float *__restrict__ dht, float *__restrict__ dh_chunks, float *__restrict__ ddelta,
+    float *__restrict__ dh0) {
+    extern __shared__ float smem[];
+    float *dh = smem;                      // [K][kBV]
+    float *qs = dh + K * kBV;              // [64][K+1]
+    float *ks = qs + kChunk * (K + 1);
+    float *ws = ks + kChunk * (K + 1);
+    float *Ai = ws + kChunk * (K + 1);     // [64][65]
+    float *P = Ai + kChunk * 65;           // [64][65]
+    float *dos = P + kChunk * 65;          // [64][kBV+1]
+    float *dd = dos + kChunk * (kBV + 1);  // [64][kBV+1]  dDelta
+    float *gam = dd + kChunk * (kBV + 1);
+    float *bet = gam + kChunk;
+    float *egam = bet + kChunk;
+
+    const int n = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * kBV;
+    const int hq = h / (d.Hv / d.Hq);
+    const int tid = threadIdx.x;
+    const SeqRange sr = seq_range(d, n);
+    const int nchunks = (sr.len + kChunk - 1) / kChunk;
+
+    for (int e = tid; e < K * kBV; e += kThreads) {
+        const int j = e / kBV, cc = e % kBV;
+        dh[e] = dht ? dht[(((size_t)n * d.Hv + h) * K + j) * V + c0 + cc] : 0.f;
+    }
+    for (int ci = nchunks - 1; ci >= 0; --ci) {
+        const int cg = sr.chunk0 + ci;
+        const int t0 = sr.start + ci * kChunk;
+        const int len = min(kChunk, sr.len - ci * kChunk);
+        __syncthreads();
+        {
+            float *hc = dh_chunks + ((size_t)cg * d.Hv + h) * K * V;
+            for (int e = tid; e < K * kBV; e += kThreads)
+                hc[(size_t)(e / kBV) * V + c0 + (e % kBV)] = dh[e];
+        }
+        for (int e = tid; e < kChunk * K; e += kThreads) {
+            const int r = e / K, j = e % K;
+            const size_t off = ((size_t)(t0 + r) * d.Hq + hq) * K + j;
+            qs[r * (K + 1) + j] = r < len ? to_f32(q[off]) : 0.f;
+            ks[r * (K + 1) + j] = r < len ? to_f32(k[off]) : 0.f;
+        }
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            dos[r * (kBV + 1) + cc] =
+                r < len ? to_f32(d_o[((size_t)(t0 + r) * d.Hv + h) * V + c0 + cc]) : 0.f;
+        }
+        const TA *Ag = ainv + ((size_t)cg * d.Hv + h) * kChunk * kChunk;
+        for (int e = tid; e < kChunk * kChunk; e += kThreads)
+            Ai[(e / kChunk) * 65 + (e % kChunk)] = to_f32(Ag[e]);
+        if (tid < kChunk) {
+            gam[tid] = gamma[(size_t)(t0 + min(tid, len - 1)) * d.Hv + h];
+            bet[tid] = tid < len ? beta[(size_t)(t0 + tid) * d.Hv + h] : 0.f;
+        }
+        __syncthreads();
+        if (tid < kChunk) egam[tid] = expf(gam[tid]);
+        __syncthreads();
+        for (int e = tid; e < kChunk * K; e += kThreads) {
+            const int r = e / K, j = e % K;
+            float acc = 0.f;
+            for (int s = 0; s <= r; ++s) acc = fmaf(Ai[r * 65 + s] * bet[s] * egam[s], ks[s * (K + 1) + j], acc);
+            ws[r * (K + 1) + j] = acc;
+        }
+        for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+            const int r = e / kChunk, s = e % kChunk;
+            float acc = 0.f;
+            if (s <= r) {
+                for (int j = 0; j < K; ++j) acc = fmaf(qs[r * (K + 1) + j], ks[s * (K + 1) + j], acc);
+                acc *= expf(gam[r] - gam[s]);
+            }
+            P[r * 65 + s] = acc;
+        }
+        __syncthreads();
+        const float gl = gam[kChunk - 1];
+        // dDelta[s][c] = scale sum_{r>=s} P[r][s] dO[r][c] + e^{gl - gam_s} k_s . dh[:, c]
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int s = e / kBV, cc = e % kBV;
+            float acc = 0.f;
+            if (s < len) {
+                float a1 = 0.f;
+                for (int r = s; r < len; ++r) a1 = fmaf(P[r * 65 + s], dos[r * (kBV + 1) + cc], a1);
+                float a2 = 0.f;
+                for (int j = 0; j < K; ++j) a2 = fmaf(ks[s * (K + 1) + j], dh[j * kBV + cc], a2);
+                acc = d.scale * a1 + expf(gl - gam[s]) * a2;
+            }
+            dd[s * (kBV + 1) + cc] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int s = e / kBV, cc = e % kBV;
+            if (s < len) ddelta[((size_t)(t0 + s) * d.Hv + h) * V + c0 + cc] = dd[s * (kBV + 1) + cc];
+        }
+        // dh = scale Q^T diag(e^gamma) dO + e^{gl} dh - w^T dDelta
+        const float eC = expf(gl);
+        for (int e = tid; e < K * kBV; e += kThreads) {
+            const int j = e / kBV, cc = e % kBV;
+            float a1 = 0.f, a2 = 0.f;
+            for (int r = 0; r < len; ++r) {
+                a1 = fmaf(qs[r * (K + 1) + j] * egam[r], dos[r * (kBV + 1) + cc], a1);
+                a2 = fmaf(ws[r * (K + 1) + j], dd[r * (kBV + 1) + cc], a2);
+            }
+            dh[e] = d.scale * a1 + eC * dh[e] - a2;
+        }
+    }
+    __syncthreads();
+    if (dh0) {
+        for (int e = tid; e < K * kBV; e += kThreads) {
+            const int j = e / kBV, cc = e % kBV;
+            dh0[(((size_t)n * d.Hv + h) * K + j) * V + c0 + cc] = dh[e];
+        }
+    }
+}
+
+// ------------------------------------------------------------ per-chunk grads
+template <int K>
+constexpr size_t grad_smem_floats() {
+    return 3 * (size_t)kChunk * 65            // Ai, dMq, dA
+           + 2 * (size_t)kChunk * K           // Qacc, Kacc
+           + 2 * (size_t)K * kBV              // hs, dhs
+           + 6 * (size_t)kChunk * (kBV + 1)   // dO, Delta, dDelta, v, dU, tmp
+           + 8 * kChunk;                      // gam, bet, egam, dgam, dbet, t2, ...
+}
+
+template <typename Tin, typename TA, int K, int V>
+__global__ void __launch_bounds__(kThreads) bwd_grad_simt(
+    Dims d, const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+    const Tin *__restrict__ d_o, const float *__restrict__ gamma, const float *__restrict__ beta,
+    const TA *__restrict__ ainv, const float *__restrict__ h_chunks,
+    const float *__restrict__ dh_chunks, const float *__restrict__ delta,
+    const float *__restrict__ ddelta, float *__restrict__ dq_part, float *__restrict__ dk_part,
+    Tin *__restrict__ dv, float *__restrict__ dg, float *__restrict__ dbeta) {
+    extern __shared__ float smem[];
+    float *Ai = smem;                          // [64][65]
+    float *dMq = Ai + kChunk * 65;             // [64][65]  scale dO Delta^T (s <= r), later dP
+    float *dA = dMq + kChunk * 65;             // [64][65]  -dU Delta^T (s < r), later Y
+    float *Qacc = dA + kChunk * 65;            // [64][K]
+    float *Kacc = Qacc + kChunk * K;           // [64][K]
+    float *hs = Kacc + kChunk * K;             // [K][kBV]
+    float *dhs = hs + K * kBV;                 // [K][kBV]
+    float *dos = dhs + K * kBV;                // [64][kBV+1]
+    float *Ds = dos + kChunk * (kBV + 1);      // Delta slice
+    float *dDs = Ds + kChunk * (kBV + 1);      // dDelta slice
+    float *vs = dDs + kChunk * (kBV + 1);      // v slice
+    float *dU = vs + kChunk * (kBV + 1);       // dU slice
+    float *tmp = dU + kChunk * (kBV + 1);      // scratch slice
+    float *gam = tmp + kChunk * (kBV + 1);
+    float *bet = gam + kChunk;
+    float *egam = bet + kChunk;
+    float *dgam = egam + kChunk;               // d(gamma) per row
+    float *dbet = dgam + kChunk;
+    float *red = dbet + kChunk;                // [64] row reductions
+    float *dgC = red + kChunk;                 // [1] d(gamma_C)
+
+    const int c = blockIdx.x, h = blockIdx.y;
+    const int n = chunk_owner(d, c);
+    if (n < 0) return;
+    const SeqRange sr = seq_range(d, n);
+    const int ci = c - sr.chunk0;
+    const int t0 = sr.start + ci * kChunk;
+    const int len = min(kChunk, sr.len - ci * kChunk);
+    const int hq = h / (d.Hv / d.Hq);
+    const int tid = threadIdx.x;
+    const float sc = d.scale;
+
+    auto Qg = [&](int r, int j) -> float {
+        return r < len ? to_f32(q[((size_t)(t0 + r) * d.Hq + hq) * K + j]) : 0.f;
+    };
+    auto Kg = [&](int r, int j) -> float {
+        return r < len ? to_f32(k[((size_t)(t0 + r) * d.Hq + hq) * K + j]) : 0.f;
+    };
+
+    const TA *Ag = ainv + ((size_t)c * d.Hv + h) * kChunk * kChunk;
+    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+        const int r = e / kChunk, s = e % kChunk;
+        Ai[r * 65 + s] = to_f32(Ag[e]);
+        dMq[r * 65 + s] = 0.f;
+        dA[r * 65 + s] = 0.f;
+    }
+    for (int e = tid; e < kChunk * K; e += kThreads) {
+        Qacc[e] = 0.f;
+        Kacc[e] = 0.f;
+    }
+    if (tid < kChunk) {
+        gam[tid] = gamma[(size_t)(t0 + min(tid, len - 1)) * d.Hv + h];
+        bet[tid] = tid < len ? beta[(size_t)(t0 + tid) * d.Hv + h] : 0.f;
+        dgam[tid] = 0.f;
+        dbet[tid] = 0.f;
+    }
+    if (tid == 0) dgC[0] = 0.f;
+    __syncthreads();
+    if (tid < kChunk) egam[tid] = expf(gam[tid]);
+    __syncthreads();
+    const float gl = gam[kChunk - 1];
+    const float eC = expf(gl);
+    const float *hc = h_chunks + ((size_t)c * d.Hv + h) * K * V;
+    const float *dhc = dh_chunks + ((size_t)c * d.Hv + h) * K * V;
+
+    for (int c0 = 0; c0 < V; c0 += kBV) {
+        for (int e = tid; e < K * kBV; e += kThreads) {
+            const size_t off = (size_t)(e / kBV) * V + c0 + (e % kBV);
+            hs[e] = hc[off];
+            dhs[e] = dhc[off];
+        }
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            const size_t off = ((size_t)(t0 + r) * d.Hv + h) * V + c0 + cc;
+            const bool ok = r < len;
+            dos[r * (kBV + 1) + cc] = ok ? to_f32(d_o[off]) : 0.f;
+            Ds[r * (kBV + 1) + cc] = ok ? delta[off] : 0.f;
+            dDs[r * (kBV + 1) + cc] = ok ? ddelta[off] : 0.f;
+            vs[r * (kBV + 1) + cc] = ok ? to_f32(v[off]) : 0.f;
+        }
+        __syncthreads();
+        // dU = Ainv^T dDelta ; dv = beta dU
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            float acc = 0.f;
+            for (int s = r; s < kChunk; ++s) acc = fmaf(Ai[s * 65 + r], dDs[s * (kBV + 1) + cc], acc);
+            dU[r * (kBV + 1) + cc] = acc;
+            if (r < len) dv[((size_t)(t0 + r) * d.Hv + h) * V + c0 + cc] = from_f32<Tin>(bet[r] * acc);
+        }
+        __syncthreads();
+        // 64x64 accumulators
+        for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+            const int r = e / kChunk, s = e % kChunk;
+            if (s <= r) {
+                float a = 0.f, b = 0.f;
+                for (int cc = 0; cc < kBV; ++cc) {
+                    a = fmaf(dos[r * (kBV + 1) + cc], Ds[s * (kBV + 1) + cc], a);
+                    b = fmaf(dU[r * (kBV + 1) + cc], Ds[s * (kBV + 1) + cc], b);
+                }
+                dMq[r * 65 + s] += sc * a;
+                if (s < r) dA[r * 65 + s] -= b;
+            }
+        }
+        // 64xK accumulators: Qacc += scale e^gam_r (dO h^T); Kacc += -beta_r e^gam_r (dU h^T) + e^{gl-gam_r} (Delta dh'^T)
+        for (int e = tid; e < kChunk * K; e += kThreads) {
+            const int r = e / K, j = e % K;
+            float a = 0.f, b = 0.f, t = 0.f;
+            for (int cc = 0; cc < kBV; ++cc) {
+                const float hv = hs[j * kBV + cc];
+                a = fmaf(dos[r * (kBV + 1) + cc], hv, a);
+                b = fmaf(dU[r * (kBV + 1) + cc], hv, b);
+                t = fmaf(Ds[r * (kBV + 1) + cc], dhs[j * kBV + cc], t);
+            }
+            Qacc[e] += sc * egam[r] * a;
+            Kacc[e] += -bet[r] * egam[r] * b + expf(gl - gam[r]) * t;
+        }
+        // Row terms. tmp = Q h (slice): d(gamma_r) += scale e^gam_r <dO_r, (Qh)_r>
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            float a = 0.f;
+            for (int j = 0; j < K; ++j) a = fmaf(Qg(r, j), hs[j * kBV + cc], a);
+            tmp[r * (kBV + 1) + cc] = a;
+        }
+        __syncthreads();
+        if (tid < kChunk) {
+            const int r = tid;
+            float a = 0.f;
+            for (int cc = 0; cc < kBV; ++cc) a = fmaf(dos[r * (kBV + 1) + cc], tmp[r * (kBV + 1) + cc], a);
+            dgam[r] += sc * egam[r] * a;
+            // dbeta from u = Ainv diag(beta) V
+            float b = 0.f;
+            for (int cc = 0; cc < kBV; ++cc) b = fmaf(dU[r * (kBV + 1) + cc], vs[r * (kBV + 1) + cc], b);
+            dbet[r] += b;
+        }
+        __syncthreads();
+        // tmp = K h (slice): t1_r = <k_r, dKb_r> = -<dU_r, (Kh)_r>
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            float a = 0.f;
+            for (int j = 0; j < K; ++j) a = fmaf(Kg(r, j), hs[j * kBV + cc], a);
+            tmp[r * (kBV + 1) + cc] = a;
+        }
+        __syncthreads();
+        if (tid < kChunk) {
+            const int r = tid;
+            float a = 0.f;
+            for (int cc = 0; cc < kBV; ++cc) a = fmaf(dU[r * (kBV + 1) + cc], tmp[r * (kBV + 1) + cc], a);
+            const float t1 = -a;
+            dbet[r] += egam[r] * t1;
+            dgam[r] += bet[r] * egam[r] * t1;
+        }
+        __syncthreads();
+        // tmp = K dh' (slice): t2_s = <k_s, dKtil_s> = <Delta_s, (K dh')_s>
+        for (int e = tid; e < kChunk * kBV; e += kThreads) {
+            const int r = e / kBV, cc = e % kBV;
+            float a = 0.f;
+            for (int j = 0; j < K; ++j) a = fmaf(Kg(r, j), dhs[j * kBV + cc], a);
+            tmp[r * (kBV + 1) + cc] = a;
+        }
+        __syncthreads();
+        if (tid < kChunk) {
+            const int s = tid;
+            float a = 0.f;
+            for (int cc = 0; cc < kBV; ++cc) a = fmaf(Ds[s * (kBV + 1) + cc], tmp[s * (kBV + 1) + cc], a);
+            red[s] = expf(gl - gam[s]) * a;
+            dgam[s] -= red[s];
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float a = 0.f;
+            for (int s = 0; s < kChunk; ++s) a += red[s];
+            float b = 0.f;  // <dh', h> over this slice
+            for (int e = 0; e < K * kBV; ++e) b = fmaf(dhs[e], hs[e], b);
+            dgC[0] += a + eC * b;
+        }
+        __syncthreads();
+    }
+    // dP = dMq o M (gradient w.r.t. q_r.k_s); W = dA o M, so that with
+    // A_rs = beta_r M_rs (k_r.k_s): d beta_r += sum_s W_rs kk_rs and the gradient
+    // w.r.t. kk_rs is Y_rs = beta_r W_rs. The log-decay gradients of both masks are
+    // Z = dP o QK^T and Zr = Y o KK^T: row sums add to d(gamma_r), column sums
+    // subtract from d(gamma_s) (the diagonal cancels).
+    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+        const int r = e / kChunk, s = e % kChunk;
+        float P = 0.f, W = 0.f;
+        if (s <= r && r < len) {
+            const float m = expf(gam[r] - gam[s]);
+            P = dMq[r * 65 + s] * m;
+            if (s < r) W = dA[r * 65 + s] * m;
+        }
+        dMq[r * 65 + s] = P;
+        dA[r * 65 + s] = W;
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        const int r = tid;
+        float zrow = 0.f, dbrow = 0.f;
+        for (int s = 0; s < r; ++s) {
+            float qk = 0.f, kk = 0.f;
+            for (int j = 0; j < K; ++j) {
+                qk = fmaf(Qg(r, j), Kg(s, j), qk);
+                kk = fmaf(Kg(r, j), Kg(s, j), kk);
+            }
+            zrow = fmaf(dMq[r * 65 + s], qk, zrow);
+            zrow = fmaf(bet[r] * dA[r * 65 + s], kk, zrow);
+            dbrow = fmaf(dA[r * 65 + s], kk, dbrow);
+        }
+        float zcol = 0.f;
+        for (int rr = r + 1; rr < kChunk; ++rr) {
+            float qk = 0.f, kk = 0.f;
+            for (int j = 0; j < K; ++j) {
+                qk = fmaf(Qg(rr, j), Kg(r, j), qk);
+                kk = fmaf(Kg(rr, j), Kg(r, j), kk);
+            }
+            zcol = fmaf(dMq[rr * 65 + r], qk, zcol);
+            zcol = fmaf(bet[rr] * dA[rr * 65 + r], kk, zcol);
+        }
+        dgam[r] += zrow - zcol;
+        dbet[r] += dbrow;
+    }
+    __syncthreads();
+    // Y = beta_r W in place
+    for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+        const int r = e / kChunk, s = e % kChunk;
+        dA[r * 65 + s] *= bet[r];
+    }
+    __syncthreads();
+    // Qacc += dP K ; Kacc += dP^T Q + Y K + Y^T K
+    for (int e = tid; e < kChunk * K; e += kThreads) {
+        const int r = e / K, j = e % K;
+        float a = 0.f, b = 0.f;
+        for (int s = 0; s <= r; ++s) {
+            a = fmaf(dMq[r * 65 + s], Kg(s, j), a);
+            b = fmaf(dA[r * 65 + s], Kg(s, j), b);
+        }
+        for (int s = r; s < kChunk; ++s) {
+            b = fmaf(dMq[s * 65 + r], Qg(s, j), b);
+            b = fmaf(dA[s * 65 + r], Kg(s, j), b);
+        }
+        Qacc[e] += a;
+        Kacc[e] += b;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // d(gamma_C) lands on the last valid row; dg = in-chunk reverse cumsum of d(gamma).
+        dgam[len - 1] += dgC[0];
+        float run = 0.f;
+        for (int r = len - 1; r >= 0; --r) {
+            run += dgam[r];
+            dgam[r] = run;
+        }
+    }
+    __syncthreads();
+    if (tid < len) {
+        const size_t off = (size_t)(t0 + tid) * d.Hv + h;
+        dg[off] = dgam[tid];
+        dbeta[off] = dbet[tid];
+    }
+    for (int e = tid; e < kChunk * K; e += kThreads) {
+        const int r = e / K, j = e % K;
+        if (r < len) {
+            const size_t off = ((size_t)(t0 + r) * d.Hv + h) * K + j;
+            dq_part[off] = Qacc[e];
+            dk_part[off] = Kacc[e];
+        }
+    }
+}
+
+// dq[t, hq] = sum over the value heads of group hq (increasing order) of the partials.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) bwd_final(Dims d, const float *__restrict__ dq_part,
+                                                      const float *__restrict__ dk_part,
+                                                      Tin *__restrict__ dq, Tin *__restrict__ dk) {
+    const int G = d.Hv / d.Hq;
+    const size_t total = (size_t)d.T_total * d.Hq * d.K;
+    for (size_t e = (size_t)blockIdx.x * kThreads + threadIdx.x; e < total;
+         e += (size_t)gridDim.x * kThreads) {
+        const int j = (int)(e % d.K);
+        const size_t th = e / d.K;          // t * Hq + hq
+        const int hq = (int)(th % d.Hq);
+        const size_t t = th / d.Hq;
+        float a = 0.f, b = 0.f;
+        for (int g = 0; g < G; ++g) {
+            const size_t off = (t * d.Hv + (size_t)hq * G + g) * d.K + j;
+            a += dq_part[off];
+            b += dk_part[off];
+        }
+        dq[e] = from_f32<Tin>(a);
+        dk[e] = from_f32<Tin>(b);
+    }
+}
+
+template <typename Tin, typename TA, int K, int V>
+cudaError_t bwd_dispatch(const BwdArgs &a, float *dq_part, float *dk_part) {
+    cudaError_t e;
+    if (a.d.N > 0) {
+        const size_t smem = sizeof(float) * dh_smem_floats<K>();
+        auto kern = bwd_dh_simt<Tin, TA, K, V>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        kern<<<dim3(a.d.N, a.d.Hv, V / kBV), kThreads, smem, a.stream>>>(
+            a.d, (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.d_o, a.gamma, a.beta,
+            (const TA *)a.ainv, a.dht, a.dh_chunks, a.ddelta, a.dh0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (a.d.NC > 0) {
+        const size_t smem = sizeof(float) * grad_smem_floats<K>();
+        auto kern = bwd_grad_simt<Tin, TA, K, V>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        kern<<<dim3(a.d.NC, a.d.Hv), kThreads, smem, a.stream>>>(
+            a.d, (const Tin *)a.q, (const Tin *)a.k, (const Tin *)a.v, (const Tin *)a.d_o, a.gamma,
+            a.beta, (const TA *)a.ainv, a.h_chunks, a.dh_chunks, a.delta, a.ddelta, dq_part, dk_part,
+            (Tin *)a.dv, a.dg, a.dbeta);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (a.d.T_total > 0) {
+        const size_t total = (size_t)a.d.T_total * a.d.Hq * a.d.K;
+        const int blocks = (int)((total + kThreads - 1) / kThreads < 148 * 16 ? (total + kThreads - 1) / kThreads : 148 * 16);
+        bwd_final<Tin><<<blocks, kThreads, 0, a.stream>>>(a.d, dq_part, dk_part, (Tin *)a.dq, (Tin *)a.dk);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part) {
+    const int kv = (a.d.K == 64 ? 0 : 2) + (a.d.V == 64 ? 0 : 1);
+    if (a.dtype == GDN_DTYPE_F32) {
+        switch (kv) {
+            case 0: return bwd_dispatch<float, float, 64, 64>(a, dq_part, dk_part);
+            case 1: return bwd_dispatch<float, float, 64, 128>(a, dq_part, dk_part);
+            case 2: return bwd_dispatch<float, float, 128, 64>(a, dq_part, dk_part);
+            default: return bwd_dispatch<float, float, 128, 128>(a, dq_part, dk_part);
+        }
+    }
+    switch (kv) {
+        case 0: return bwd_dispatch<__nv_bfloat16, __nv_bfloat16, 64, 64>(a, dq_part, dk_part);
+        case 1: return bwd_dispatch<__nv_bfloat16, __nv_bfloat16, 64, 128>(a, dq_part, dk_part);
+        case 2: return bwd_dispatch<__nv_bfloat16, __nv_bfloat16, 128, 64>(a, dq_part, dk_part);
+        default: return bwd_dispatch<__nv_bfloat16, __nv_bfloat16, 128, 128>(a, dq_part, dk_part);
+    }
+}
+
+}  // namespace gdn

@@ -1,0 +1,113 @@
+"""Backward parity on the GPU: gradients from the CUDA path (through the C ABI)
+vs the fp64 oracle's hand-derived reverse mode, on the same seeded inputs.
+Gate: relative Frobenius error <= 1e-2 per gradient tensor; fp32 problems are
+also held to 1e-4 so that a small wrong term cannot hide under bf16 noise."""
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, Workload, make_inputs, scaled
+from parity_util import TOL_GRAD_REL, f64, gpu_fwd, rel_fro, to_dev
+
+pytestmark = pytest.mark.gpu
+NAMES = ("dq", "dk", "dv", "dbeta", "dg", "dh0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gated_deltanet_chunked_rule_b200 import build
+    build.build()
+
+
+def gpu_bwd(x, use_saved=True):
+    import gated_deltanet_chunked_rule_b200 as gdn
+    d = to_dev(x)
+    saved = None
+    if use_saved:
+        _, _, saved = gpu_fwd(x, save_for_backward=True)
+    out = gdn.chunk_gated_delta_rule_bwd(
+        d["q"], d["k"], d["v"], d["g"], d["beta"], saved, d["do"], d.get("dht"), d["scale"],
+        d.get("h0"), d.get("cu_seqlens"), x.get("cu_seqlens"))
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    return dict(zip(NAMES, out))
+
+
+def oracle_bwd(oracle, x):
+    cu = None if x.get("cu_seqlens") is None else x["cu_seqlens"].numpy()
+    return oracle.bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["do"],
+                      dht=x.get("dht"), h0=x.get("h0"), cu_seqlens=cu)
+
+
+def check(oracle, x, g, label, tol=TOL_GRAD_REL):
+    r = oracle_bwd(oracle, x)
+    errs = {n: rel_fro(f64(g[n]), r[n]) for n in NAMES}
+    print(f"[grad parity] {label}: " + "  ".join(f"{n} {e:.2e}" for n, e in errs.items()))
+    bad = {n: e for n, e in errs.items() if not e <= tol}
+    assert not bad, (label, bad)
+    return errs
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("K,V", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_small_ragged_shapes(oracle_mod, dtype, K, V):
+    w = Workload(f"bwd_{dtype}_{K}x{V}", B=2, T=200, Hq=2, Hv=4, K=K, V=V, dtype=dtype,
+                 h0_std=0.02, grads=True, seed=K + 2 * V)
+    x = make_inputs(w)
+    check(oracle_mod, x, gpu_bwd(x), w.name, tol=1e-4 if dtype == "fp32" else TOL_GRAD_REL)
+
+
+@pytest.mark.parametrize("T", [1, 64, 65])
+def test_chunk_boundaries(oracle_mod, T):
+    w = Workload(f"bwd_T{T}", B=1, T=T, Hq=1, Hv=1, K=64, V=64, dtype="fp32", h0_std=0.5,
+                 grads=True, dht_std=0.5, seed=T)
+    x = make_inputs(w)
+    check(oracle_mod, x, gpu_bwd(x), w.name, tol=1e-4)
+
+
+def test_varlen_with_empty_sequences(oracle_mod):
+    w = Workload("bwd_varlen", B=1, T=400, Hq=2, Hv=4, K=128, V=128, dtype="fp32", grads=True,
+                 seed=11)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 70, 70, 200, 400], dtype=torch.int32)
+    gen = torch.Generator().manual_seed(3)
+    x["h0"] = 0.1 * torch.randn((4, 4, 128, 128), generator=gen)
+    x["dht"] = 0.1 * torch.randn((4, 4, 128, 128), generator=gen)
+    g = gpu_bwd(x)
+    check(oracle_mod, x, g, "bwd_varlen", tol=1e-4)
+    # empty sequence: dh0 = dht exactly
+    torch.testing.assert_close(g["dh0"][1].cpu(), x["dht"][1], rtol=0, atol=0)
+
+
+def test_saved_equals_recompute():
+    w = Workload("bwd_saved", B=1, T=300, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, grads=True,
+                 seed=12)
+    x = make_inputs(w)
+    a = gpu_bwd(x, use_saved=True)
+    b = gpu_bwd(x, use_saved=False)
+    for n in NAMES:
+        torch.testing.assert_close(a[n], b[n], rtol=0, atol=0)
+
+
+def test_autograd_function(oracle_mod):
+    import gated_deltanet_chunked_rule_b200 as gdn
+    w = Workload("bwd_autograd", B=1, T=150, Hq=1, Hv=2, K=64, V=64, dtype="fp32",
+                 h0_std=0.1, grads=True, seed=13)
+    x = make_inputs(w)
+    d = to_dev(x)
+    leaves = {n: d[n].clone().requires_grad_(True) for n in ("q", "k", "v", "g", "beta", "h0")}
+    o, fin = gdn.chunk_gated_delta_rule(leaves["q"], leaves["k"], leaves["v"], leaves["g"],
+                                        leaves["beta"], d["scale"], leaves["h0"], True)
+    ((o * d["do"]).sum() + (fin * d["dht"]).sum()).backward()
+    g = dict(dq=leaves["q"].grad, dk=leaves["k"].grad, dv=leaves["v"].grad,
+             dbeta=leaves["beta"].grad, dg=leaves["g"].grad, dh0=leaves["h0"].grad)
+    check(oracle_mod, x, g, "bwd_autograd", tol=1e-4)
+
+
+@pytest.mark.parametrize("name", ["bwd_b2_t4096_h16", "qwen_prefill_t8192_hv32"])
+def test_full_size_workloads(oracle_mod, name):
+    w = scaled(WORKLOADS[name], grads=True)
+    x = make_inputs(w)
+    check(oracle_mod, x, gpu_bwd(x), name)
