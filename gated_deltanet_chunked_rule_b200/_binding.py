@@ -37,7 +37,11 @@ EXPORTS = (
     "gdn_version",
     "gdn_timing_enable",
     "gdn_timing_report",
+    "gdn_chunk_fwd_noalloc",
 )
+
+# Size of the static scratch array behind gdn_chunk_fwd_noalloc.
+GDN_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class gdn_problem(ctypes.Structure):
@@ -79,6 +83,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, vp, sz, vp]
             L.gdn_chunk_bwd.restype = i
+            L.gdn_chunk_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.gdn_chunk_fwd_noalloc.restype = i
             L.gdn_get_device_status.argtypes = [vp]
             L.gdn_get_device_status.restype = i
             L.gdn_status_string.argtypes = [i]

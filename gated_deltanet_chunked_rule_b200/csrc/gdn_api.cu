@@ -381,6 +381,47 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     return GDN_OK;
 }
 
+}  // extern "C"
+
+// ----------------------------------------------------- no-allocation forward
+// Static scratch for gdn_chunk_fwd_noalloc. In host code the array's name is
+// only a host-side stand-in; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+namespace gdn {
+namespace {
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+void *noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+}  // namespace gdn
+
+extern "C" {
+
+int gdn_chunk_fwd_noalloc(const gdn_problem *p, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, const float *h0, void *o,
+                          float *final_state, void *stream) {
+    Plan P;
+    int rc = make_plan(p, &P);
+    if (rc != GDN_OK) return rc;
+    if (fwd_ws_bytes(P) > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return GDN_ERR_CUDA;
+    return gdn_chunk_fwd(p, q, k, v, g, beta, h0, o, final_state, nullptr, scratch,
+                         GDN_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 int gdn_get_device_status(void *stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
     unsigned v = 0, zero = 0;

@@ -111,6 +111,34 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
                   float *dbeta, float *dh0, void *workspace, size_t workspace_bytes,
                   void *stream /* cudaStream_t */);
 
+/* Forward that allocates nothing and needs no workspace.
+ *
+ * For callers that cannot allocate device memory at all: a plugin hosted by
+ * an engine that owns every device allocation and hands out only inputs and
+ * outputs, or a latency-critical path that must not call cudaMalloc/cudaFree
+ * (either can synchronise the whole device). It runs the same forward as
+ * gdn_chunk_fwd with saved = NULL, but its scratch is a fixed static device
+ * array of GDN_NOALLOC_SCRATCH_BYTES (16 MiB) inside this library, which every
+ * GPU that loads the library holds until the process exits. It calls no
+ * cudaMalloc, cudaFree or other allocating routine. The caller still passes
+ * inputs and outputs, as for gdn_chunk_fwd.
+ *   - A problem whose forward scratch (gdn_fwd_workspace_size) is larger than
+ *     GDN_NOALLOC_SCRATCH_BYTES is rejected with GDN_ERR_WORKSPACE before
+ *     anything is enqueued.
+ *   - The first call on each device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads on the
+ *     same device) race on it and corrupt each other's results, so serialise
+ *     them. Nothing in it has to start at zero: each call writes every byte it
+ *     reads before reading it.
+ * The FlashQLA pages have no counterpart to this entry point. */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int gdn_chunk_fwd_noalloc(const gdn_problem *p, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, const float *h0, void *o,
+                          float *final_state, void *stream /* cudaStream_t */);
+
 /* Synchronises `stream`, then returns and clears the current device's status
  * word (GDN_OK if no kernel recorded a problem since the last call). */
 int gdn_get_device_status(void *stream /* cudaStream_t */);
