@@ -89,7 +89,9 @@ def kernel_bytes(name, w):
     h0 = st if w.h0_std is not None else 0
     table = {
         "prep_simt": qk1 + 2 * gam + gam + ainv,               # k, g, beta -> gamma, Ainv
+        "prep_tc": qk1 + 2 * gam + gam + ainv,
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
+        "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
     }
     return table.get(name)
 

@@ -235,6 +235,16 @@ bool use_simt(int dtype) {
     return e && strcmp(e, "simt") == 0;
 }
 
+// Chunk prep: tensor-core Gram + blocked inverse for bf16 K=128, CUDA cores otherwise.
+int launch_prep(const FwdArgs &a) {
+    if (!use_simt(a.dtype) && prep_tc_supported(a)) {
+        TimedLaunch t("prep_tc", a.stream);
+        return launch_prep_tc(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    }
+    TimedLaunch t("prep_simt", a.stream);
+    return launch_prep_simt(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 int launch_plan(const gdn_problem *p, Plan &P, char *ws, unsigned *status, cudaStream_t st) {
     if (!P.varlen) return GDN_OK;
     int *info = (int *)ws;
@@ -301,12 +311,11 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.status = status;
     a.stream = st;
     a.nseg = 1;
-    (void)use_simt;
-    {
-        TimedLaunch t("prep_simt", st);
-        if (launch_prep_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
-    }
-    {
+    if ((rc = launch_prep(a)) != GDN_OK) return rc;
+    if (!use_simt(P.dtype) && tc_fwd_supported(a)) {
+        TimedLaunch t("fwd_tc", st);
+        if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
+    } else {
         TimedLaunch t("fwd_simt", st);
         if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
     }
@@ -350,10 +359,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     f.ainv = sv + P.gamma_bytes;
     f.h_chunks = (float *)(ws + L.hc);
     f.delta = (float *)(ws + L.delta);
-    if (!saved) {
-        TimedLaunch t("prep_simt", st);
-        if (launch_prep_simt(f) != cudaSuccess) return GDN_ERR_CUDA;
-    }
+    if (!saved && (rc = launch_prep(f)) != GDN_OK) return rc;
     {
         TimedLaunch t("bwd_recompute_simt", st);
         if (launch_fwd_simt(f) != cudaSuccess) return GDN_ERR_CUDA;

@@ -132,5 +132,9 @@ struct BwdArgs {
 cudaError_t launch_prep_simt(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
 cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part);
+bool tc_fwd_supported(const FwdArgs &a);
+bool prep_tc_supported(const FwdArgs &a);
+cudaError_t launch_prep_tc(const FwdArgs &a);
+cudaError_t launch_fwd_tc(const FwdArgs &a);
 
 }  // namespace gdn
