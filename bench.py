@@ -92,6 +92,7 @@ def kernel_bytes(name, w):
         "prep_tc": qk1 + 2 * gam + gam + ainv,
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
         "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
+        "fwd_hybrid": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
     }
     return table.get(name)
 

@@ -313,8 +313,14 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.nseg = 1;
     if ((rc = launch_prep(a)) != GDN_OK) return rc;
     if (!use_simt(P.dtype) && tc_fwd_supported(a)) {
-        TimedLaunch t("fwd_tc", st);
-        if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
+        const char *which = getenv("GDN_FWD");
+        if (which && strcmp(which, "v1") == 0) {
+            TimedLaunch t("fwd_tc", st);
+            if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
+        } else {
+            TimedLaunch t("fwd_hybrid", st);
+            if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
+        }
     } else {
         TimedLaunch t("fwd_simt", st);
         if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;

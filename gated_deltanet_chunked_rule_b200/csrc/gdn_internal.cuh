@@ -136,5 +136,6 @@ bool tc_fwd_supported(const FwdArgs &a);
 bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
+cudaError_t launch_fwd2(const FwdArgs &a);
 
 }  // namespace gdn

@@ -128,17 +128,19 @@ def test_full_size_workloads(oracle_mod, name):
     run(oracle_mod, WORKLOADS[name])
 
 
-def test_tensor_core_and_cuda_core_paths_agree(oracle_mod, monkeypatch):
-    # K = V = 128 bf16 runs on the tcgen05 kernel by default; GDN_IMPL=simt forces
-    # the fp32 CUDA-core kernel. Both must meet the oracle tolerance, and agree.
+@pytest.mark.parametrize("env", [("GDN_IMPL", "simt"), ("GDN_FWD", "v1")])
+def test_tensor_core_and_cuda_core_paths_agree(oracle_mod, monkeypatch, env):
+    # K = V = 128 bf16 runs on the hybrid (mma.sync chain + tcgen05) kernel by
+    # default; GDN_FWD=v1 selects the all-tcgen05 kernel and GDN_IMPL=simt the
+    # fp32 CUDA-core one. Each must meet the oracle tolerance, and they agree.
     w = Workload("paths", B=1, T=777, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, seed=8)
     x = make_inputs(w)
     o_tc, f_tc, _ = gpu_fwd(x)
-    monkeypatch.setenv("GDN_IMPL", "simt")
+    monkeypatch.setenv(*env)
     o_si, f_si, _ = gpu_fwd(x)
-    monkeypatch.delenv("GDN_IMPL")
+    monkeypatch.delenv(env[0])
     e_tc = check_fwd(oracle_mod, x, o_tc, f_tc, "tc")
     e_si = check_fwd(oracle_mod, x, o_si, f_si, "simt")
-    print(f"[paths] tc o {e_tc[0]:.3e} final {e_tc[1]:.3e} | simt o {e_si[0]:.3e} final {e_si[1]:.3e}")
+    print(f"[paths] default o {e_tc[0]:.3e} final {e_tc[1]:.3e} | {env} o {e_si[0]:.3e} final {e_si[1]:.3e}")
     from parity_util import rel_fro
     assert rel_fro(f64(o_tc), f64(o_si)) <= 5e-3
