@@ -90,6 +90,7 @@ struct Plan {
     int dtype;
     bool varlen;
     size_t gamma_bytes, ainv_bytes, saved_bytes, seq_info_bytes;
+    size_t wy_bytes;  // scaled inverses for the tensor-core forward (bf16, K = V = 128)
 };
 
 int make_plan(const gdn_problem *p, Plan *out) {
@@ -132,13 +133,16 @@ int make_plan(const gdn_problem *p, Plan *out) {
     P.ainv_bytes = align_up((size_t)d.NC * d.Hv * kChunk * kChunk *
                             (p->dtype == GDN_DTYPE_F32 ? sizeof(float) : sizeof(__nv_bfloat16)));
     P.saved_bytes = P.gamma_bytes + P.ainv_bytes;
+    P.wy_bytes = (p->dtype == GDN_DTYPE_BF16 && p->K == 128 && p->V == 128)
+                     ? align_up((size_t)d.NC * d.Hv * 2 * kChunk * kChunk * sizeof(__nv_bfloat16))
+                     : 0;
     *out = P;
     return GDN_OK;
 }
 
 size_t fwd_ws_bytes(const Plan &P) {
-    // sequence table + gamma/Ainv (used when the caller passes no `saved`)
-    return P.seq_info_bytes + P.saved_bytes;
+    // sequence table | gamma, Ainv (used when the caller passes no `saved`) | scaled inverses
+    return P.seq_info_bytes + P.saved_bytes + P.wy_bytes;
 }
 
 // Backward workspace: sequence table | gamma, Ainv (when no `saved`) | per-chunk
@@ -311,16 +315,21 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.status = status;
     a.stream = st;
     a.nseg = 1;
+    const char *which = getenv("GDN_FWD");
+    const bool tc = !use_simt(P.dtype) && tc_fwd_supported(a);
+    const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.wy_bytes > 0;
+    if (hybrid) {
+        // the hybrid forward reads the scaled inverses; Ainv itself only when saved
+        a.wy = ws + P.seq_info_bytes + P.saved_bytes;
+        if (!saved) a.ainv = nullptr;
+    }
     if ((rc = launch_prep(a)) != GDN_OK) return rc;
-    if (!use_simt(P.dtype) && tc_fwd_supported(a)) {
-        const char *which = getenv("GDN_FWD");
-        if (which && strcmp(which, "v1") == 0) {
-            TimedLaunch t("fwd_tc", st);
-            if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
-        } else {
-            TimedLaunch t("fwd_hybrid", st);
-            if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
-        }
+    if (hybrid) {
+        TimedLaunch t("fwd_hybrid", st);
+        if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
+    } else if (tc) {
+        TimedLaunch t("fwd_tc", st);
+        if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
     } else {
         TimedLaunch t("fwd_simt", st);
         if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;

@@ -102,7 +102,9 @@ struct FwdArgs {
     void *o;
     float *final_state;
     float *gamma;    // [T_total, Hv] fp32
-    void *ainv;      // [NC, Hv, 64, 64], fp32 (F32 problems) or bf16 (BF16 problems)
+    void *ainv;      // [NC, Hv, 64, 64], fp32 (F32 problems) or bf16 (BF16 problems); may be null
+                     // for the tensor-core forward when nothing is saved
+    void *wy;        // [NC, Hv, 2, 64, 64] bf16: Ainv diag(beta), Ainv diag(beta e^gamma) (tensor-core forward)
     unsigned *status;
     cudaStream_t stream;
     // Per-chunk entry states and Delta for the backward's recompute (nullable).

@@ -7,6 +7,7 @@
 //   gamma = in-chunk cumulative sum of g (per value head)
 //   A_rs  = beta_r exp(gamma_r - gamma_s) G_rs   for s < r
 //   Ainv  = (I + A)^-1                   (fp32, then stored as bf16)
+//   and, for the tensor-core forward, Ainv diag(beta) and Ainv diag(beta e^gamma)
 //
 // The unit lower-triangular inverse is taken block-wise on 16 x 16 blocks:
 // the four diagonal blocks by forward substitution (one thread per column),
@@ -69,7 +70,8 @@ __global__ void __launch_bounds__(kThreads) prep_tc_kernel(Dims d, const __nv_bf
                                                            const float *__restrict__ g,
                                                            const float *__restrict__ beta,
                                                            float *__restrict__ gamma_out,
-                                                           __nv_bfloat16 *__restrict__ ainv_out) {
+                                                           __nv_bfloat16 *__restrict__ ainv_out,
+                                                           __nv_bfloat16 *__restrict__ wy_out) {
     extern __shared__ uint8_t smem_raw[];
     PrepSmem &S = *reinterpret_cast<PrepSmem *>(smem_raw);
     const int c = blockIdx.x, hq = blockIdx.y;
@@ -224,14 +226,35 @@ __global__ void __launch_bounds__(kThreads) prep_tc_kernel(Dims d, const __nv_bf
             }
             __syncthreads();
         }
-        // ---- Ainv -> bf16 (16-byte stores)
-        __nv_bfloat16 *out = ainv_out + ((size_t)c * d.Hv + h) * kChunk * kChunk;
-        for (int e = tid; e < 64 * 8; e += kThreads) {
-            const int r = e >> 3, q = e & 7;
-            __align__(16) __nv_bfloat162 v[4];
+        // ---- Ainv -> bf16 (16-byte stores); optionally the two scaled inverses
+        //      Ainv diag(beta) and Ainv diag(beta e^gamma) that the forward multiplies
+        //      with V and K (so it needs no elementwise pass of its own)
+        if (ainv_out) {
+            __nv_bfloat16 *out = ainv_out + ((size_t)c * d.Hv + h) * kChunk * kChunk;
+            for (int e = tid; e < 64 * 8; e += kThreads) {
+                const int r = e >> 3, q = e & 7;
+                __align__(16) __nv_bfloat162 v[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) v[p] = __floats2bfloat162_rn(S.X[r][q * 8 + 2 * p], S.X[r][q * 8 + 2 * p + 1]);
-            *reinterpret_cast<uint4 *>(out + r * 64 + q * 8) = *reinterpret_cast<uint4 *>(v);
+                for (int pp = 0; pp < 4; ++pp) v[pp] = __floats2bfloat162_rn(S.X[r][q * 8 + 2 * pp], S.X[r][q * 8 + 2 * pp + 1]);
+                *reinterpret_cast<uint4 *>(out + r * 64 + q * 8) = *reinterpret_cast<uint4 *>(v);
+            }
+        }
+        if (wy_out) {
+            __nv_bfloat16 *ou = wy_out + ((size_t)c * d.Hv + h) * 2 * kChunk * kChunk;
+            __nv_bfloat16 *ow = ou + kChunk * kChunk;
+            for (int e = tid; e < 64 * 8; e += kThreads) {
+                const int r = e >> 3, q = e & 7;
+                __align__(16) __nv_bfloat162 vu[4], vw[4];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const int s0 = q * 8 + 2 * pp;
+                    const float a0 = S.X[r][s0] * S.bet[s0], a1 = S.X[r][s0 + 1] * S.bet[s0 + 1];
+                    vu[pp] = __floats2bfloat162_rn(a0, a1);
+                    vw[pp] = __floats2bfloat162_rn(a0 * __expf(S.gam[s0]), a1 * __expf(S.gam[s0 + 1]));
+                }
+                *reinterpret_cast<uint4 *>(ou + r * 64 + q * 8) = *reinterpret_cast<uint4 *>(vu);
+                *reinterpret_cast<uint4 *>(ow + r * 64 + q * 8) = *reinterpret_cast<uint4 *>(vw);
+            }
         }
         __syncthreads();
     }
@@ -248,7 +271,7 @@ cudaError_t launch_prep_tc(const FwdArgs &a) {
     if (e != cudaSuccess) return e;
     dim3 grid(a.d.NC, a.d.Hq);
     prep_tc_kernel<<<grid, kThreads, smem, a.stream>>>(a.d, (const __nv_bfloat16 *)a.k, a.g, a.beta, a.gamma,
-                                                       (__nv_bfloat16 *)a.ainv);
+                                                       (__nv_bfloat16 *)a.ainv, (__nv_bfloat16 *)a.wy);
     return cudaGetLastError();
 }
 

@@ -155,6 +155,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // t/4 + 8 of the 16, columns 8 i + 2 (t % 4) + {0, 1} for i < X, in the order
 // v[4i] = (row t/4, col 8i+2(t%4)), v[4i+1] = (row t/4, +1),
 // v[4i+2] = (row t/4 + 8, col 8i+2(t%4)), v[4i+3] = (row t/4 + 8, +1).
+__device__ __forceinline__ void tmem_ld16x256_x2(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
