@@ -71,28 +71,46 @@ def algorithmic(w, tokens_per_seq=None):
     return dict(f_fwd=f_fwd, f_bwd=f_bwd, b_fwd=b_fwd, b_bwd=b_bwd, tokens=ntok)
 
 
-def kernel_bytes(name, w):
+def kernel_bytes(name, w, saved=False):
     """Algorithmic bytes of one launch of a named kernel: the tensors that kernel
-    must read once and write once in this design."""
+    must read once and write once in this design (intermediates between the
+    kernels of the chain included, since each kernel has to move them).
+
+    Per token and value head at K = V = 128, bf16 (e = 2), G = Hv / Hq:
+      prep_tc          k/G*K*e + 3*4 (g, beta, gamma) + 2*C*e (scaled inverses) [+ C*e Ainv when saved]
+      fwd_hybrid       2K*e/G (q, k) + 2V*e (v, o) + 4 (gamma) + 2*C*e (scaled inverses)
+      bwd_recompute    K*e/G (k) + V*e (v) + 4 + 2*C*e + K*V*e/C (entry states) + V*e (Delta)
+      bwd_dh           2K*e/G (q, k) + V*e (dO) + C*e (Aw) + 4 + K*V*e/C (dh') + V*e (dDelta)
+      bwd_grad         2K*e/G + 2V*e (v, dO) + 8 (gamma, beta) + C*e (Ainv) + 2K*V*e/C (h, dh')
+                       + 2V*e (Delta, dDelta) + 2K*4 (dq, dk partials) + V*e (dv) + 8 (dg, dbeta)
+      bwd_final        2K*4 (partials) + 2K*e/G (dq, dk)
+    plus the per-sequence states (h0, final, dht, dh0: K*V*4 each) where a kernel touches them.
+    """
     C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
     ntok = w.B * w.T
     N = w.varlen[0] if w.varlen else w.B
     e = 2 if w.dtype == "bf16" else 4
-    nc = math.ceil(w.T / C) * w.B if not w.varlen else None
-    if nc is None:
-        nc = ntok // C + N  # upper bound for packed input
+    nc = math.ceil(w.T / C) * w.B if not w.varlen else ntok // C + N  # upper bound for packed input
     qk1 = ntok * Hq * K * e
     v1 = ntok * Hv * V * e
     gam = ntok * Hv * 4
     ainv = nc * Hv * C * C * e
     st = N * Hv * K * V * 4
     h0 = st if w.h0_std is not None else 0
+    hc = nc * Hv * K * V * 2
+    d16 = ntok * Hv * V * 2
+    part = ntok * Hv * K * 4
     table = {
         "prep_simt": qk1 + 2 * gam + gam + ainv,               # k, g, beta -> gamma, Ainv
-        "prep_tc": qk1 + 2 * gam + gam + ainv,
+        "prep_tc": qk1 + 2 * gam + gam + 2 * ainv + (ainv if saved else 0),
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
         "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
-        "fwd_hybrid": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
+        "fwd_hybrid": 2 * qk1 + v1 + gam + 2 * ainv + h0 + v1 + st,
+        "bwd_prep_tc": qk1 + 2 * gam + gam + 2 * ainv + (0 if saved else ainv),
+        "bwd_recompute": qk1 + v1 + gam + 2 * ainv + h0 + hc + d16,
+        "bwd_dh": 2 * qk1 + v1 + ainv + gam + st + hc + d16 + st,
+        "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + 2 * d16 + 2 * part + v1 + 2 * gam,
+        "bwd_final": 2 * part + 2 * qk1,
     }
     return table.get(name)
 
@@ -343,7 +361,7 @@ def main():
     dom = max(rep, key=lambda k: rep[k][1])
     pk, pk_kind = peaks()
     dom_avg_s = rep[dom][1] / rep[dom][0] * 1e-3
-    dom_bytes = kernel_bytes(dom, w)
+    dom_bytes = kernel_bytes(dom, w, saved=do_bwd)
     roofline = {"kernel": dom, "bound": "hbm", "unit": "GB/s",
                 "achieved": dom_bytes / dom_avg_s / 1e9 if dom_bytes else None,
                 "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)",

@@ -170,7 +170,44 @@ BwdLayout bwd_layout(const Plan &P) {
     return L;
 }
 
-size_t bwd_ws_bytes(const Plan &P) { return bwd_layout(P).total; }
+// Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv
+// (when no `saved`) | gamma (prep output when `saved` is given) | scaled inverses |
+// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta |
+// fp32 dq, dk partials per value head.
+struct TcBwdLayout {
+    size_t seq, saved, gam2, wy, hc, dhc, delta, ddelta, dqp, dkp, total;
+};
+
+TcBwdLayout tc_bwd_layout(const Plan &P) {
+    const Dims &d = P.d;
+    TcBwdLayout L;
+    const size_t hc = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
+    const size_t dl = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
+    const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
+    L.seq = 0;
+    L.saved = L.seq + P.seq_info_bytes;
+    L.gam2 = L.saved + P.saved_bytes;
+    L.wy = L.gam2 + P.gamma_bytes;
+    L.hc = L.wy + P.wy_bytes;
+    L.dhc = L.hc + hc;
+    L.delta = L.dhc + hc;
+    L.ddelta = L.delta + dl;
+    L.dqp = L.ddelta + dl;
+    L.dkp = L.dqp + qp;
+    L.total = L.dkp + qp;
+    return L;
+}
+
+bool tc_bwd_path(const Plan &P) {
+    return !(P.dtype == GDN_DTYPE_F32 || (getenv("GDN_IMPL") && strcmp(getenv("GDN_IMPL"), "simt") == 0)) &&
+           tc_bwd_supported(P.d, P.dtype) && P.wy_bytes > 0;
+}
+
+// Either backward path fits in the size reported to callers.
+size_t bwd_ws_bytes(const Plan &P) {
+    const size_t a = bwd_layout(P).total, b = P.wy_bytes > 0 ? tc_bwd_layout(P).total : 0;
+    return a > b ? a : b;
+}
 
 // Builds the sequence table from the device copy of cu_seqlens and checks it
 // against the host plan (total tokens, total chunks). On any disagreement it
@@ -240,12 +277,12 @@ bool use_simt(int dtype) {
 }
 
 // Chunk prep: tensor-core Gram + blocked inverse for bf16 K=128, CUDA cores otherwise.
-int launch_prep(const FwdArgs &a) {
+int launch_prep(const FwdArgs &a, const char *tc_name = "prep_tc", const char *simt_name = "prep_simt") {
     if (!use_simt(a.dtype) && prep_tc_supported(a)) {
-        TimedLaunch t("prep_tc", a.stream);
+        TimedLaunch t(tc_name, a.stream);
         return launch_prep_tc(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
     }
-    TimedLaunch t("prep_simt", a.stream);
+    TimedLaunch t(simt_name, a.stream);
     return launch_prep_simt(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -352,7 +389,8 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     for (const void *x : ptrs)
         if (x && !aligned16(x)) return GDN_ERR_INVALID_ARG;
     const BwdLayout L = bwd_layout(P);
-    if (workspace_bytes < L.total || (L.total && !workspace) || ((uintptr_t)workspace & 255u))
+    const size_t need = bwd_ws_bytes(P);
+    if (workspace_bytes < need || (need && !workspace) || ((uintptr_t)workspace & 255u))
         return GDN_ERR_WORKSPACE;
     if (saved && ((uintptr_t)saved & 255u)) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
@@ -360,6 +398,67 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     if (!status) return GDN_ERR_CUDA;
     char *ws = (char *)workspace;
     if ((rc = launch_plan(p, P, ws, status, st)) != GDN_OK) return rc;
+
+    if (tc_bwd_path(P)) {
+        // tensor-core path: prep (gamma, Ainv when not saved, scaled inverses) ->
+        // recompute of h, Delta (bf16) -> reverse dh scan -> per-chunk gradients -> GQA sum
+        const TcBwdLayout T = tc_bwd_layout(P);
+        FwdArgs f;
+        memset(&f, 0, sizeof(f));
+        f.d = P.d;
+        f.dtype = P.dtype;
+        f.q = q; f.k = k; f.v = v; f.g = g; f.beta = beta; f.h0 = h0;
+        f.status = status;
+        f.stream = st;
+        f.nseg = 1;
+        f.wy = ws + T.wy;
+        const void *ainv;
+        if (saved) {
+            f.gamma = (float *)(ws + T.gam2);
+            f.ainv = nullptr;
+            ainv = (const char *)saved + P.gamma_bytes;
+        } else {
+            f.gamma = (float *)(ws + T.saved);
+            f.ainv = ws + T.saved + P.gamma_bytes;
+            ainv = f.ainv;
+        }
+        if ((rc = launch_prep(f, "bwd_prep_tc", "bwd_prep_simt")) != GDN_OK) return rc;
+        f.o = nullptr;
+        f.final_state = nullptr;
+        f.h_chunks16 = ws + T.hc;
+        f.delta16 = ws + T.delta;
+        {
+            TimedLaunch t("bwd_recompute", st);
+            if (launch_fwd2(f) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        BwdArgs b;
+        memset(&b, 0, sizeof(b));
+        b.d = P.d;
+        b.dtype = P.dtype;
+        b.q = q; b.k = k; b.v = v; b.d_o = d_o;
+        b.g = g; b.beta = beta; b.h0 = h0; b.dht = dht;
+        b.gamma = f.gamma;
+        b.ainv = ainv;
+        b.dq = dq; b.dk = dk; b.dv = dv; b.dg = dg; b.dbeta = dbeta; b.dh0 = dh0;
+        b.status = status;
+        b.stream = st;
+        {
+            TimedLaunch t("bwd_dh", st);
+            if (launch_bwd_dh_tc(b, f.wy, ws + T.dhc, ws + T.ddelta) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        {
+            TimedLaunch t("bwd_grad", st);
+            if (launch_bwd_grad_tc(b, ws + T.hc, ws + T.dhc, ws + T.delta, ws + T.ddelta, (float *)(ws + T.dqp),
+                                   (float *)(ws + T.dkp)) != cudaSuccess)
+                return GDN_ERR_CUDA;
+        }
+        {
+            TimedLaunch t("bwd_final", st);
+            if (launch_bwd_final(b, (const float *)(ws + T.dqp), (const float *)(ws + T.dkp)) != cudaSuccess)
+                return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
 
     FwdArgs f;
     memset(&f, 0, sizeof(f));
@@ -374,7 +473,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
     f.ainv = sv + P.gamma_bytes;
     f.h_chunks = (float *)(ws + L.hc);
     f.delta = (float *)(ws + L.delta);
-    if (!saved && (rc = launch_prep(f)) != GDN_OK) return rc;
+    if (!saved && (rc = launch_prep(f, "bwd_prep_tc", "bwd_prep_simt")) != GDN_OK) return rc;
     {
         TimedLaunch t("bwd_recompute_simt", st);
         if (launch_fwd_simt(f) != cudaSuccess) return GDN_ERR_CUDA;

@@ -44,12 +44,14 @@
 #include <cstddef>
 
 #include "gdn_internal.cuh"
+#include "gdn_warp.cuh"
 #include "sm100_ptx.cuh"
 
 namespace gdn {
 namespace {
 
 using namespace sm100;
+using namespace warp;
 
 constexpr int kThreads = 576;  // 8 chain + 8 aux + 2 TMA/MMA warps
 constexpr int kRole = 256;     // threads per CUDA-core role
@@ -93,105 +95,19 @@ struct Small {
 static_assert(sizeof(Small) <= 2560, "small area");
 static_assert(kSmall % 16 == 0 && offsetof(Small, gates) % 16 == 0, "small area alignment");
 
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait (2 s of wall-clock time); false if it expired or the CTA is aborting.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    const uint32_t a = smem_u32(bar);
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if ((i & 1023u) == 0) {
-            if (*abort_flag) return false;
-            const uint64_t t = globaltimer();
-            if (i == 0) t0 = t;
-            else if (t - t0 > 2000000000ull) return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void publish(uint32_t *ctr, uint32_t v) {
-    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(ctr)), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *ctr) {
-    uint32_t v;
-    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(ctr)) : "memory");
-    return v;
-}
-
-// Waits (bounded, 2 s) until *ctr >= need; false if it expired or the CTA is aborting.
-__device__ __forceinline__ bool wait_ge(const uint32_t *ctr, uint32_t need, volatile int *abort_flag) {
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        if (ld_acquire(ctr) >= need) return true;
-        if ((i & 255u) == 0) {
-            if (*abort_flag) return false;
-            const uint64_t t = globaltimer();
-            if (i == 0) t0 = t;
-            else if (t - t0 > 2000000000ull) return false;
-        }
-    }
-}
-
-// Named barrier over one role (kRole threads) that also ANDs a predicate across it.
+template <int N = kRole>
 __device__ __forceinline__ bool role_sync_and(int id, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "n"(kRole)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// Per-access shared-memory stores and fragment loads carry no "memory" clobber
-// so the compiler may overlap them; ordering across roles comes from the
-// barrier, fence and release/acquire statements, which do clobber memory.
-__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t a) {
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(a));
-}
-__device__ __forceinline__ void st_shared_v2f(uint32_t addr, float a, float b) {
-    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void hmma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    return warp::role_sync_and<N>(id, pred);
 }
 
 struct Fwd2Params {
     Dims d;
     const float *gamma;   // [T_total, Hv]
     const float *h0;      // [N, Hv, K, V] or null
-    __nv_bfloat16 *o;     // [T_total, Hv, V]
+    __nv_bfloat16 *o;     // [T_total, Hv, V], or null: no output products (the backward's recompute)
     float *final_state;   // [N, Hv, K, V] or null
+    __nv_bfloat16 *h_chunks;  // [NC, Hv, K, V] entry state of every chunk (bf16, as the products read it) or null
+    __nv_bfloat16 *delta;     // [T_total, Hv, V] Delta (bf16) or null
     unsigned *status;
 };
 
@@ -292,6 +208,19 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             // gate scalars of chunk j (its slot is refilled only after this chunk's -w is consumed)
             const Gates &G = sm->gates[j % 3];
             const float gl = G.gam[63];
+            if (prm.h_chunks) {  // entry state of chunk j, rounded as the products read it
+                __nv_bfloat16 *hc = prm.h_chunks + ((size_t)(sr.chunk0 + j) * d.Hv + h) * K * V + c0;
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int dim = 32 * p + 16 * mt + g + half * 8;
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+                            *reinterpret_cast<uint32_t *>(hc + (size_t)dim * V + 8 * (cb + nt) + 2 * c4) =
+                                pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
+                    }
+            }
             const float gtok[2] = {G.gam[16 * p + g], G.gam[16 * p + g + 8]};
             // ---- Delta = u + (-w) h : tokens 16p..16p+15, columns of n-tiles cb, cb+1
             float acc[2][4];
@@ -339,6 +268,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         const float x0 = live ? acc[nt][2 * half] : 0.f, x1 = live ? acc[nt][2 * half + 1] : 0.f;
                         st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(x0, x1));
                         st_shared_b32(dt + (cb + nt) * 1024 + off, pack_bf16(sc * x0, sc * x1));
+                        if (prm.delta && live)
+                            *reinterpret_cast<uint32_t *>(prm.delta + ((size_t)(sr.start + j * kChunk + tok) * d.Hv + h) * V +
+                                                          c0 + 8 * (cb + nt) + 2 * c4) = pack_bf16(x0, x1);
                     }
                 }
             }
@@ -415,8 +347,10 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int ag = lane >> 2, ac = lane & 3;
         const int ar0 = ap * 16 + ag, ar1 = ar0 + 8;  // rows of M=64 results this thread holds
         bool ok = true;
+        const bool want_o = prm.o != nullptr;
         auto output = [&](int jo) -> bool {  // o of chunk jo from DQ, DP (16 columns per warp)
             if (!wait_ge(&ctr[kODone], jo + 1, abort_flag)) return false;
+            if (!want_o) return true;
             tc_fence_after();
             const Gates &G = sm->gates[jo % 3];
             const int len = min(kChunk, sr.len - jo * kChunk);
@@ -505,7 +439,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             // ---- P = causal decay mask o S -> SW128 tile for DP, once DP of chunk j-1 is done with it
             ok = role_sync_and(2, j < 1 || wait_ge(&ctr[kODone], j, abort_flag));
             if (!ok) break;
-            {
+            if (want_o) {
                 const Gates &G = sm->gates[j % 3];
                 float v[16];
                 tmem_ld16x256_x4(tmem + lane_base + abuf + kColS + 32 * ah, v);  // key columns 32 ah .. +31
@@ -569,7 +503,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     mma_bf16(tb + kColU, smem_desc(st + kAu + ks * 32, 16, 1024, kSw128),
                              smem_desc(st + kVt + ks * 1024, 4096, 512, kSw64), id_U, ks > 0);
                 }
-                for (int ks = 0; ks < 8; ++ks) {
+                for (int ks = 0; ks < 8 && prm.o; ++ks) {
                     const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
                     mma_bf16(tb + kColS, smem_desc(st + kQ + off, 16, 1024, kSw128),
                              smem_desc(st + kK + off, 16, 1024, kSw128), id_S, ks > 0);
@@ -593,6 +527,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 ok = wait_ge(&ctr[kH], j + 1, abort_flag) && wait_ge(&ctr[kDelta], j + 1, abort_flag) &&
                      wait_ge(&ctr[kPReady], j + 1, abort_flag) && wait_ge(&ctr[kTmemO], j, abort_flag);
                 if (!ok) break;
+                if (!prm.o) {  // recompute for the backward: no output products
+                    publish(&ctr[kODone], j + 1);
+                } else {
                 tc_fence_after();
                 const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j % 3) * 4096;
                 for (int ks = 0; ks < 8; ++ks) {
@@ -608,6 +545,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (!ok) break;
                 tc_fence_before();
                 publish(&ctr[kODone], j + 1);
+                }
                 // refill the stage of chunk j with chunk j + 3 once the chain is done with its k tile
                 if (issued < nch) {
                     ok = wait_ge(&ctr[kStage], j + 1, abort_flag);
@@ -642,26 +580,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
               const cuuint32_t *box, CUtensorMapSwizzle sw) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return warp::make_bf16_map(m, base, rank, dims, strides, box, sw);
 }
 
 }  // namespace
@@ -691,6 +612,8 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     p.h0 = a.h0;
     p.o = (__nv_bfloat16 *)a.o;
     p.final_state = a.final_state;
+    p.h_chunks = (__nv_bfloat16 *)a.h_chunks16;
+    p.delta = (__nv_bfloat16 *)a.delta16;
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(fwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -110,6 +110,8 @@ struct FwdArgs {
     // Per-chunk entry states and Delta for the backward's recompute (nullable).
     float *h_chunks;  // [NC, Hv, K, V]
     float *delta;     // [T_total, Hv, V]
+    // The same for the tensor-core backward, in bf16 (nullable).
+    void *h_chunks16, *delta16;
     int nseg;         // sequence-split segments per sequence (1 = no split)
     float *seg_ws;    // split-path scratch
 };
@@ -139,5 +141,12 @@ bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_fwd2(const FwdArgs &a);
+// Tensor-core backward (bf16, K = V = 128): reverse dh scan, per-chunk gradients,
+// and the GQA reduction of the dq / dk partials.
+bool tc_bwd_supported(const Dims &d, int dtype);
+cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *wy, void *dh_chunks16, void *ddelta16);
+cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const void *dh_chunks16,
+                               const void *delta16, const void *ddelta16, float *dq_part, float *dk_part);
+cudaError_t launch_bwd_final(const BwdArgs &a, const float *dq_part, const float *dk_part);
 
 }  // namespace gdn

@@ -500,6 +500,18 @@ cudaError_t bwd_dispatch(const BwdArgs &a, float *dq_part, float *dk_part) {
 
 }  // namespace
 
+cudaError_t launch_bwd_final(const BwdArgs &a, const float *dq_part, const float *dk_part) {
+    const size_t total = (size_t)a.d.T_total * a.d.Hq * a.d.K;
+    if (total == 0) return cudaSuccess;
+    const int blocks = (int)((total + kThreads - 1) / kThreads < 148 * 16 ? (total + kThreads - 1) / kThreads : 148 * 16);
+    if (a.dtype == GDN_DTYPE_F32)
+        bwd_final<float><<<blocks, kThreads, 0, a.stream>>>(a.d, dq_part, dk_part, (float *)a.dq, (float *)a.dk);
+    else
+        bwd_final<__nv_bfloat16><<<blocks, kThreads, 0, a.stream>>>(a.d, dq_part, dk_part, (__nv_bfloat16 *)a.dq,
+                                                                    (__nv_bfloat16 *)a.dk);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part) {
     const int kv = (a.d.K == 64 ? 0 : 2) + (a.d.V == 64 ? 0 : 1);
     if (a.dtype == GDN_DTYPE_F32) {

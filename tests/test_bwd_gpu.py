@@ -111,3 +111,41 @@ def test_full_size_workloads(oracle_mod, name):
     w = scaled(WORKLOADS[name], grads=True)
     x = make_inputs(w)
     check(oracle_mod, x, gpu_bwd(x), name)
+
+
+def test_varlen_bf16_tensor_core_path(oracle_mod):
+    # bf16 K = V = 128 runs the tensor-core backward: ragged and empty sequences,
+    # per-sequence h0 and dht
+    w = Workload("bwd_varlen_bf16", B=1, T=520, Hq=2, Hv=4, K=128, V=128, grads=True, seed=14)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 0, 130, 137, 137, 520], dtype=torch.int32)
+    gen = torch.Generator().manual_seed(5)
+    x["h0"] = 0.02 * torch.randn((5, 4, 128, 128), generator=gen)
+    x["dht"] = 0.01 * torch.randn((5, 4, 128, 128), generator=gen)
+    g = gpu_bwd(x)
+    check(oracle_mod, x, g, "bwd_varlen_bf16")
+    for n in (0, 3):  # empty sequences: dh0 = dht exactly
+        torch.testing.assert_close(g["dh0"][n].cpu(), x["dht"][n], rtol=0, atol=0)
+
+
+def test_tensor_core_and_cuda_core_backward_agree(oracle_mod, monkeypatch):
+    w = Workload("bwd_paths", B=1, T=333, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, grads=True,
+                 seed=15)
+    x = make_inputs(w)
+    a = gpu_bwd(x)
+    monkeypatch.setenv("GDN_IMPL", "simt")
+    b = gpu_bwd(x)
+    monkeypatch.delenv("GDN_IMPL")
+    ea = check(oracle_mod, x, a, "bwd tensor-core")
+    eb = check(oracle_mod, x, b, "bwd cuda-core")
+    for n in NAMES:
+        assert rel_fro(f64(a[n]), f64(b[n])) <= TOL_GRAD_REL, n
+
+
+def test_backward_deterministic():
+    w = Workload("bwd_det", B=1, T=700, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, grads=True, seed=16)
+    x = make_inputs(w)
+    a = gpu_bwd(x)
+    b = gpu_bwd(x)
+    for n in NAMES:
+        torch.testing.assert_close(a[n], b[n], rtol=0, atol=0)
