@@ -132,17 +132,19 @@ int make_plan(const gdn_problem *p, Plan *out) {
     P.gamma_bytes = align_up(sizeof(float) * (size_t)d.T_total * d.Hv);
     P.ainv_bytes = align_up((size_t)d.NC * d.Hv * kChunk * kChunk *
                             (p->dtype == GDN_DTYPE_F32 ? sizeof(float) : sizeof(__nv_bfloat16)));
-    P.saved_bytes = P.gamma_bytes + P.ainv_bytes;
     P.wy_bytes = (p->dtype == GDN_DTYPE_BF16 && p->K == 128 && p->V == 128)
                      ? align_up((size_t)d.NC * d.Hv * 2 * kChunk * kChunk * sizeof(__nv_bfloat16))
                      : 0;
+    // saved = gamma | Ainv | (bf16 K = V = 128) the scaled inverses, so that a
+    // backward given `saved` needs no chunk prep of its own
+    P.saved_bytes = P.gamma_bytes + P.ainv_bytes + P.wy_bytes;
     *out = P;
     return GDN_OK;
 }
 
 size_t fwd_ws_bytes(const Plan &P) {
-    // sequence table | gamma, Ainv (used when the caller passes no `saved`) | scaled inverses
-    return P.seq_info_bytes + P.saved_bytes + P.wy_bytes;
+    // sequence table | gamma, Ainv, scaled inverses (used when the caller passes no `saved`)
+    return P.seq_info_bytes + P.saved_bytes;
 }
 
 // Backward workspace: sequence table | gamma, Ainv (when no `saved`) | per-chunk
@@ -170,12 +172,12 @@ BwdLayout bwd_layout(const Plan &P) {
     return L;
 }
 
-// Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv
-// (when no `saved`) | gamma (prep output when `saved` is given) | scaled inverses |
+// Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv,
+// scaled inverses (when no `saved`) |
 // bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta |
 // fp32 dq, dk partials per value head.
 struct TcBwdLayout {
-    size_t seq, saved, gam2, wy, hc, dhc, delta, ddelta, dqp, dkp, total;
+    size_t seq, saved, hc, dhc, delta, ddelta, dqp, dkp, total;
 };
 
 TcBwdLayout tc_bwd_layout(const Plan &P) {
@@ -186,9 +188,7 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
-    L.gam2 = L.saved + P.saved_bytes;
-    L.wy = L.gam2 + P.gamma_bytes;
-    L.hc = L.wy + P.wy_bytes;
+    L.hc = L.saved + P.saved_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dl;
@@ -349,17 +349,14 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.o = o; a.final_state = final_state;
     a.gamma = (float *)sv;
     a.ainv = sv + P.gamma_bytes;
+    a.wy = P.wy_bytes ? sv + P.gamma_bytes + P.ainv_bytes : nullptr;
     a.status = status;
     a.stream = st;
     a.nseg = 1;
     const char *which = getenv("GDN_FWD");
     const bool tc = !use_simt(P.dtype) && tc_fwd_supported(a);
     const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.wy_bytes > 0;
-    if (hybrid) {
-        // the hybrid forward reads the scaled inverses; Ainv itself only when saved
-        a.wy = ws + P.seq_info_bytes + P.saved_bytes;
-        if (!saved) a.ainv = nullptr;
-    }
+    if (hybrid && !saved) a.ainv = nullptr;  // the hybrid forward reads only the scaled inverses
     if ((rc = launch_prep(a)) != GDN_OK) return rc;
     if (hybrid) {
         TimedLaunch t("fwd_hybrid", st);
@@ -411,18 +408,13 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         f.status = status;
         f.stream = st;
         f.nseg = 1;
-        f.wy = ws + T.wy;
-        const void *ainv;
-        if (saved) {
-            f.gamma = (float *)(ws + T.gam2);
-            f.ainv = nullptr;
-            ainv = (const char *)saved + P.gamma_bytes;
-        } else {
-            f.gamma = (float *)(ws + T.saved);
-            f.ainv = ws + T.saved + P.gamma_bytes;
-            ainv = f.ainv;
-        }
-        if ((rc = launch_prep(f, "bwd_prep_tc", "bwd_prep_simt")) != GDN_OK) return rc;
+        // gamma | Ainv | scaled inverses: from the forward's `saved`, else made here
+        char *sv = saved ? (char *)saved : ws + T.saved;
+        f.gamma = (float *)sv;
+        f.ainv = sv + P.gamma_bytes;
+        f.wy = sv + P.gamma_bytes + P.ainv_bytes;
+        const void *ainv = f.ainv;
+        if (!saved && (rc = launch_prep(f, "bwd_prep_tc", "bwd_prep_simt")) != GDN_OK) return rc;
         f.o = nullptr;
         f.final_state = nullptr;
         f.h_chunks16 = ws + T.hc;

@@ -81,7 +81,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_older() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // rows [0, rows) of a bf16 matrix with `cols` columns, global row stride `ld` elements;
 // rows >= valid are zero-filled.
@@ -137,17 +139,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
     const Tile tD{sb + kSD, 256}, tdD{sb + kSdD, 256}, th{sb + kSh, 256}, tdh{sb + kSdh, 256};
     const Tile tA{sb + kSA, 128}, tT1{sb + kST1, 128}, tdG{sb + kSdG, 128};
 
-    // ---- loads (cp.async; rows past the chunk's end are zero)
+    // ---- loads (cp.async; rows past the chunk's end are zero). Two groups: the
+    //      chunk tiles for phases A-C, then the two states, which land while A-C run.
     const size_t hbase = ((size_t)cg * d.Hv + h) * K * V;
     load_tile(tQ, prm.q + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
     load_tile(tK, prm.k + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
-    load_tile(tV, prm.v + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
     load_tile(tdO, prm.d_o + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
     load_tile(tD, prm.delta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
     load_tile(tdD, prm.ddelta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    load_tile(tA, prm.ainv + ((size_t)cg * d.Hv + h) * C * C, C, C, C, C, tid);
+    load_tile(tV, prm.v + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    cp_async_commit();
     load_tile(th, prm.h_chunks + hbase, V, K, V, K, tid);
     load_tile(tdh, prm.dh_chunks + hbase, V, K, V, K, tid);
-    load_tile(tA, prm.ainv + ((size_t)cg * d.Hv + h) * C * C, C, C, C, C, tid);
+    cp_async_commit();
     if (tid < C) {
         const int r = tid, rr = min(r, len - 1);
         const float gm = prm.gamma[(size_t)(t0 + rr) * d.Hv + h];
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
         vec.egam[r] = __expf(gm);
         vec.bet[r] = r < len ? prm.beta[(size_t)(t0 + r) * d.Hv + h] : 0.f;
     }
-    cp_async_wait_all();
+    cp_async_wait_older();
     __syncthreads();
 
     const float gC = vec.gam[63];  // gamma at the chunk's last token (padded rows repeat it)
@@ -247,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
             st_shared_b32(toff(tdG, r1, s), pack_bf16(dgv[2], dgv[3]));
         }
     }
-    __syncthreads();  // dG visible
+    cp_async_wait_all();  // the two states
+    __syncthreads();      // dG and the states visible
 
     // ---- phase D: dq = scale diag(e^gamma) dO h^T + T1 K  (16 x 64 per warp)
     {

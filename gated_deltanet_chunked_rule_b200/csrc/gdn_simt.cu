@@ -30,7 +30,8 @@ __global__ void __launch_bounds__(kThreads) prep_simt(Dims d, const Tin *__restr
                                                       const float *__restrict__ g,
                                                       const float *__restrict__ beta,
                                                       float *__restrict__ gamma_out,
-                                                      TA *__restrict__ ainv_out) {
+                                                      TA *__restrict__ ainv_out,
+                                                      __nv_bfloat16 *__restrict__ wy_out) {
     extern __shared__ float smem[];
     float *ks = smem;                        // [64][K+1]
     float *A = ks + kChunk * (K + 1);        // [64][65]
@@ -94,6 +95,15 @@ __global__ void __launch_bounds__(kThreads) prep_simt(Dims d, const Tin *__restr
     TA *out = ainv_out + ((size_t)c * d.Hv + h) * kChunk * kChunk;
     for (int e = tid; e < kChunk * kChunk; e += kThreads)
         store_a(out + e, X[(e / kChunk) * 65 + (e % kChunk)]);
+    if (wy_out) {  // Ainv diag(beta), Ainv diag(beta e^gamma) for the tensor-core kernels
+        __nv_bfloat16 *ou = wy_out + ((size_t)c * d.Hv + h) * 2 * kChunk * kChunk, *ow = ou + kChunk * kChunk;
+        for (int e = tid; e < kChunk * kChunk; e += kThreads) {
+            const int r = e / kChunk, s = e % kChunk;
+            const float a = X[r * 65 + s] * bet[s];
+            ou[e] = __float2bfloat16_rn(a);
+            ow[e] = __float2bfloat16_rn(a * expf(gam[s]));
+        }
+    }
 }
 
 // ---------------------------------------------------------------- forward
@@ -252,7 +262,8 @@ cudaError_t prep_dispatch(const FwdArgs &a) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.d.NC, a.d.Hv);
-    kern<<<grid, kThreads, smem, a.stream>>>(a.d, (const Tin *)a.k, a.g, a.beta, a.gamma, (TA *)a.ainv);
+    kern<<<grid, kThreads, smem, a.stream>>>(a.d, (const Tin *)a.k, a.g, a.beta, a.gamma, (TA *)a.ainv,
+                                             (__nv_bfloat16 *)a.wy);
     return cudaGetLastError();
 }
 

@@ -91,7 +91,11 @@ size_t gdn_bwd_workspace_size(const gdn_problem *p);
  * [B*T, Hv]) followed by Ainv = (I + A)^-1 of every 64-token chunk
  * ([num_chunks, Hv, 64, 64], fp32 for GDN_DTYPE_F32 problems, bf16 for
  * GDN_DTYPE_BF16), i.e. the "g, A" that page 1's low-level forward returns
- * and its backward takes back. */
+ * and its backward takes back ("底层 API" section of the FlashQLA write-up).
+ * For bf16 problems with K = V = 128 the buffer continues with the two
+ * scaled inverses Ainv diag(beta) and Ainv diag(beta e^gamma) (bf16,
+ * [num_chunks, Hv, 2, 64, 64]) that the tensor-core kernels consume, so a
+ * backward given `saved` runs no chunk prep. Each 256-byte aligned. */
 size_t gdn_saved_size(const gdn_problem *p);
 
 /* Forward. h0 may be NULL (zero initial state); final_state may be NULL (not
