@@ -9,6 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -91,7 +92,42 @@ struct Plan {
     bool varlen;
     size_t gamma_bytes, ainv_bytes, saved_bytes, seq_info_bytes;
     size_t wy_bytes;  // scaled inverses for the tensor-core forward (bf16, K = V = 128)
+    int max_chunks;   // chunks of the longest sequence
+    int nseg;         // forward sequence split: segments per sequence (1 = none)
+    size_t seg_bytes; // split scratch: c, P, start states of every segment
 };
+
+// Forward sequence split (the pages' gate-driven intra-card context
+// parallelism). With u = N * Hv * V/32 chain units and the longest sequence
+// of C chunks, an unsplit forward takes ceil(u / SMs) waves of C chunk steps;
+// split into S segments it takes ceil(2 u S / SMs) waves of the segment pass
+// (state and operator columns) plus ceil(u S / SMs) waves of the output pass,
+// each ceil(C / S) steps long, plus S small composition steps. S minimises
+// that estimate (segments of at least 8 chunks); GDN_NSEG overrides it.
+int choose_nseg(const Plan &P) {
+    const Dims &d = P.d;
+    if (P.wy_bytes == 0 || P.max_chunks < 2) return 1;
+    if (const char *e = getenv("GDN_NSEG")) {
+        const int v = atoi(e);
+        return v < 1 ? 1 : (v > P.max_chunks ? P.max_chunks : v);
+    }
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    }
+    const long long units = (long long)d.N * d.Hv * (d.V / 32);
+    auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
+    const double step_compose = 1.5;  // one composition step, in chunk steps
+    double best = (double)waves(units) * P.max_chunks;
+    int best_s = 1;
+    for (int S = 2; S <= 64 && S * 8 <= P.max_chunks; ++S) {
+        const long long per = (P.max_chunks + S - 1) / S;
+        const double cost = (double)(waves(2 * units * S) + waves(units * S)) * per + step_compose * S;
+        if (cost < 0.9 * best) best = cost, best_s = S;
+    }
+    return best_s;
+}
 
 int make_plan(const gdn_problem *p, Plan *out) {
     if (!p) return GDN_ERR_INVALID_ARG;
@@ -138,13 +174,22 @@ int make_plan(const gdn_problem *p, Plan *out) {
     // saved = gamma | Ainv | (bf16 K = V = 128) the scaled inverses, so that a
     // backward given `saved` needs no chunk prep of its own
     P.saved_bytes = P.gamma_bytes + P.ainv_bytes + P.wy_bytes;
+    if (P.varlen) {
+        for (int n = 0; n < p->num_seqs; ++n)
+            P.max_chunks = std::max(P.max_chunks, (p->cu_seqlens_host[n + 1] - p->cu_seqlens_host[n] + kChunk - 1) / kChunk);
+    } else {
+        P.max_chunks = (p->T + kChunk - 1) / kChunk;
+    }
+    P.nseg = choose_nseg(P);
+    P.seg_bytes = P.nseg > 1 ? align_up(sizeof(float) * (size_t)d.N * P.nseg * d.Hv * d.K * (2 * d.V + d.K)) : 0;
     *out = P;
     return GDN_OK;
 }
 
 size_t fwd_ws_bytes(const Plan &P) {
     // sequence table | gamma, Ainv, scaled inverses (used when the caller passes no `saved`)
-    return P.seq_info_bytes + P.saved_bytes;
+    // | sequence-split scratch
+    return P.seq_info_bytes + P.saved_bytes + P.seg_bytes;
 }
 
 // Backward workspace: sequence table | gamma, Ainv (when no `saved`) | per-chunk
@@ -358,7 +403,30 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.wy_bytes > 0;
     if (hybrid && !saved) a.ainv = nullptr;  // the hybrid forward reads only the scaled inverses
     if ((rc = launch_prep(a)) != GDN_OK) return rc;
-    if (hybrid) {
+    if (hybrid && P.nseg > 1) {
+        // sequence split: segment pass (c, P) -> composition of start states -> output pass
+        float *seg = (float *)(ws + P.seq_info_bytes + P.saved_bytes);
+        const size_t per = (size_t)P.d.N * P.nseg * P.d.Hv * P.d.K;
+        a.nseg = P.nseg;
+        a.seg_c = seg;
+        a.seg_P = seg + per * P.d.V;
+        a.seg_h0 = seg + per * (P.d.V + P.d.K);
+        FwdArgs s1 = a;
+        s1.o = nullptr;
+        s1.final_state = nullptr;
+        s1.fwd_mode = 1;
+        {
+            TimedLaunch t("fwd_split_seg", st);
+            if (launch_fwd2(s1) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        {
+            TimedLaunch t("fwd_split_compose", st);
+            if (launch_split_compose(a) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        a.fwd_mode = 2;
+        TimedLaunch t("fwd_hybrid", st);
+        if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
+    } else if (hybrid) {
         TimedLaunch t("fwd_hybrid", st);
         if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
     } else if (tc) {

@@ -100,6 +100,13 @@ __device__ __forceinline__ bool role_sync_and(int id, bool pred) {
     return warp::role_sync_and<N>(id, pred);
 }
 
+// kWhole: one CTA column per sequence, from h0.
+// kSegPass: per segment, the chain on [c | P] with c from zero (V columns, u as
+//   input) and P from the identity (K more columns, whose v tile is read out of
+//   range and so is zero): the segment maps a start state h to P h + c.
+// kSegOut: per segment, the chain and the output from the composed start state.
+enum Fwd2Mode { kWhole = 0, kSegPass = 1, kSegOut = 2 };
+
 struct Fwd2Params {
     Dims d;
     const float *gamma;   // [T_total, Hv]
@@ -108,6 +115,13 @@ struct Fwd2Params {
     float *final_state;   // [N, Hv, K, V] or null
     __nv_bfloat16 *h_chunks;  // [NC, Hv, K, V] entry state of every chunk (bf16, as the products read it) or null
     __nv_bfloat16 *delta;     // [T_total, Hv, V] Delta (bf16) or null
+    // Sequence split: blockIdx.x = sequence * nseg + segment; a segment is a
+    // contiguous run of ceil(chunks / nseg) chunks of its sequence.
+    int nseg;
+    int mode;             // kWhole, kSegPass or kSegOut
+    const float *seg_h0;  // kSegOut: [N * nseg, Hv, K, V] start state of every segment
+    float *seg_c;         // kSegPass: [N * nseg, Hv, K, V] end state from a zero start
+    float *seg_P;         // kSegPass: [N * nseg, Hv, K, K] transition operator of the segment
     unsigned *status;
 };
 
@@ -122,12 +136,22 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t sb = smem_u32(smem);
 
     const Dims &d = prm.d;
-    const int n = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * kBV;
+    const int nseg = prm.nseg;
+    const int n = blockIdx.x / nseg, sseg = blockIdx.x % nseg, h = blockIdx.y, c0 = blockIdx.z * kBV;
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const SeqRange sr = seq_range(d, n);
-    const int nch = (sr.len + kChunk - 1) / kChunk;
     constexpr int K = 128, V = 128;
+    // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
+    const SeqRange seq = seq_range(d, n);
+    const int nch_seq = (seq.len + kChunk - 1) / kChunk;
+    const int per_seg = (nch_seq + nseg - 1) / nseg;
+    const int j0 = min(sseg * per_seg, nch_seq), j1 = min(j0 + per_seg, nch_seq);
+    SeqRange sr;
+    sr.start = seq.start + j0 * kChunk;
+    sr.chunk0 = seq.chunk0 + j0;
+    sr.len = j1 > j0 ? min(seq.len - j0 * kChunk, (j1 - j0) * kChunk) : 0;
+    const int nch = j1 - j0;
+    const size_t seg_idx = (size_t)n * nseg + sseg;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm->full[s], 1);
@@ -171,7 +195,10 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int g = lane >> 2, c4 = lane & 3;
         float hf[2][2][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8(cb+nt)+2c4(+1)
         {
-            const float *src = prm.h0 ? prm.h0 + ((size_t)n * d.Hv + h) * K * V : nullptr;
+            const float *src = prm.mode == kWhole ? (prm.h0 ? prm.h0 + ((size_t)n * d.Hv + h) * K * V : nullptr)
+                               : prm.mode == kSegOut ? prm.seg_h0 + (seg_idx * d.Hv + h) * K * V
+                                                     : nullptr;
+            const bool ident = prm.mode == kSegPass && c0 >= V;  // operator columns start as I
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -180,7 +207,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int q = 0; q < 4; ++q) {
                         const int dim = 32 * p + 16 * mt + g + ((q >> 1) << 3);
                         const int col = 8 * (cb + nt) + 2 * c4 + (q & 1);
-                        hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : 0.f;
+                        hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : (ident && dim == c0 - V + col ? 1.f : 0.f);
                     }
         }
         auto write_hb = [&](int buf) {
@@ -326,18 +353,29 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (!ok) {
             if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
             *abort_flag = 1;
-        } else if (prm.final_state) {
-            float *dst = prm.final_state + ((size_t)n * d.Hv + h) * K * V + c0;
+        } else {
+            // end state: the sequence's final state (from the CTA holding its last chunk),
+            // or the segment's c / P columns
+            float *dst = nullptr;
+            int ld = V;
+            if (prm.mode == kSegPass) {
+                if (c0 < V) dst = prm.seg_c + (seg_idx * d.Hv + h) * K * V + c0;
+                else dst = prm.seg_P + (seg_idx * d.Hv + h) * K * K + (c0 - V), ld = K;
+            } else if (prm.final_state && j1 == nch_seq && (j0 < j1 || sseg == 0)) {
+                dst = prm.final_state + ((size_t)n * d.Hv + h) * K * V + c0;
+            }
+            if (dst) {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int dim = 32 * p + 16 * mt + g + half * 8;
-                        *reinterpret_cast<float2 *>(dst + (size_t)dim * V + 8 * (cb + nt) + 2 * c4) =
-                            make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
-                    }
+                        for (int half = 0; half < 2; ++half) {
+                            const int dim = 32 * p + 16 * mt + g + half * 8;
+                            *reinterpret_cast<float2 *>(dst + (size_t)dim * ld + 8 * (cb + nt) + 2 * c4) =
+                                make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
+                        }
+            }
         }
     } else if (warp < 16) {
         // ============================================================= aux
@@ -614,10 +652,19 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     p.final_state = a.final_state;
     p.h_chunks = (__nv_bfloat16 *)a.h_chunks16;
     p.delta = (__nv_bfloat16 *)a.delta16;
+    p.nseg = a.nseg > 0 ? a.nseg : 1;
+    p.mode = a.fwd_mode;
+    p.seg_h0 = a.seg_h0;
+    p.seg_c = a.seg_c;
+    p.seg_P = a.seg_P;
+    if (p.mode != kWhole && (p.nseg < 1 || (p.mode == kSegOut && !p.seg_h0) ||
+                             (p.mode == kSegPass && (!p.seg_c || !p.seg_P || p.o))))
+        return cudaErrorInvalidValue;
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(fwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(d.N, d.Hv, d.V / kBV);
+    // the segment pass also carries the K operator columns
+    dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
     fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, mw, p);
     return cudaGetLastError();
 }

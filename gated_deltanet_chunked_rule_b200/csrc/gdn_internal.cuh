@@ -113,7 +113,9 @@ struct FwdArgs {
     // The same for the tensor-core backward, in bf16 (nullable).
     void *h_chunks16, *delta16;
     int nseg;         // sequence-split segments per sequence (1 = no split)
-    float *seg_ws;    // split-path scratch
+    int fwd_mode;     // 0: whole sequences; 1: segment pass (c, P); 2: segment output pass
+    const float *seg_h0;     // [N * nseg, Hv, K, V] composed start state of every segment
+    float *seg_c, *seg_P;    // [N * nseg, Hv, K, V] / [.., K, K] segment end state from zero, operator
 };
 
 struct BwdArgs {
@@ -141,6 +143,8 @@ bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_fwd2(const FwdArgs &a);
+// Sequence split: start state of every segment from h0 and the segments' (c, P).
+cudaError_t launch_split_compose(const FwdArgs &a);
 // Tensor-core backward (bf16, K = V = 128): reverse dh scan, per-chunk gradients,
 // and the GQA reduction of the dq / dk partials.
 bool tc_bwd_supported(const Dims &d, int dtype);

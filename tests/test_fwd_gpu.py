@@ -144,3 +144,38 @@ def test_tensor_core_and_cuda_core_paths_agree(oracle_mod, monkeypatch, env):
     print(f"[paths] default o {e_tc[0]:.3e} final {e_tc[1]:.3e} | {env} o {e_si[0]:.3e} final {e_si[1]:.3e}")
     from parity_util import rel_fro
     assert rel_fro(f64(o_tc), f64(o_si)) <= 5e-3
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 7])
+def test_sequence_split_matches_oracle_and_unsplit(oracle_mod, monkeypatch, nseg):
+    # Intra-GPU sequence split: segments run in parallel, their start states are
+    # composed through each segment's K x K transition operator. Packed batch with
+    # an empty sequence, one shorter than the segment count (empty segments) and
+    # a ragged tail; per-sequence h0.
+    w = Workload("split", B=1, T=1500, Hq=2, Hv=4, K=128, V=128, seed=21)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 0, 100, 1037, 1500], dtype=torch.int32)
+    x["h0"] = 0.02 * torch.randn((4, 4, 128, 128), generator=torch.Generator().manual_seed(9))
+    monkeypatch.setenv("GDN_NSEG", "1")
+    o1, f1, _ = gpu_fwd(x)
+    monkeypatch.setenv("GDN_NSEG", str(nseg))
+    o2, f2, _ = gpu_fwd(x)
+    monkeypatch.delenv("GDN_NSEG")
+    e = check_fwd(oracle_mod, x, o2, f2, f"split{nseg}")
+    print(f"[split nseg={nseg}] o err {e[0]:.3e} final err {e[1]:.3e}")
+    from parity_util import rel_fro
+    assert rel_fro(f64(o2), f64(o1)) <= 5e-3 and rel_fro(f64(f2), f64(f1)) <= 5e-3
+    torch.testing.assert_close(f2[0].cpu(), x["h0"][0], rtol=0, atol=0)  # empty sequence
+
+
+def test_sequence_split_with_fast_decay_and_slow_decay(oracle_mod, monkeypatch):
+    # the composition is exact whatever the gates do: nearly-undecayed states
+    # (g close to 0) carry h0 across every segment boundary
+    w = Workload("split_slow", B=1, T=1024, Hq=1, Hv=2, K=128, V=128, h0_std=0.05, seed=22)
+    x = make_inputs(w)
+    x["g"] = x["g"] * 0.01
+    monkeypatch.setenv("GDN_NSEG", "4")
+    o, f, _ = gpu_fwd(x)
+    monkeypatch.delenv("GDN_NSEG")
+    e = check_fwd(oracle_mod, x, o, f, "split_slow")
+    print(f"[split slow decay] o err {e[0]:.3e} final err {e[1]:.3e}")
