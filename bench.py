@@ -77,10 +77,11 @@ def kernel_bytes(name, w, saved=False):
     kernels of the chain included, since each kernel has to move them).
 
     Per token and value head at K = V = 128, bf16 (e = 2), G = Hv / Hq:
-      prep_tc          k/G*K*e + 3*4 (g, beta, gamma) + 2*C*e (scaled inverses) [+ C*e Ainv when saved]
-      fwd_hybrid       2K*e/G (q, k) + 2V*e (v, o) + 4 (gamma) + 2*C*e (scaled inverses)
-      bwd_recompute    K*e/G (k) + V*e (v) + 4 + 2*C*e + K*V*e/C (entry states) + V*e (Delta)
-      bwd_dh           2K*e/G (q, k) + V*e (dO) + C*e (Aw) + 4 + K*V*e/C (dh') + V*e (dDelta)
+      prep3            2K*e/G (q, k) + V*e (v) + 3*4 (g, beta, gamma) + K*2 (w) + V*4 (u) + C*2 (P)
+                       [+ C*e Ainv when saved]
+      fwd_hybrid       2K*e/G (q, k) + K*2 (w) + V*4 (u) + C*2 (P) + 4 (gamma) + V*e (o)
+      bwd_recompute    K*e/G (k) + K*2 + V*4 + 4 + K*V*e/C (entry states) + V*e (Delta)
+      bwd_dh           2K*e/G (q, k) + K*2 (w) + C*2 (P) + V*e (dO) + 4 + K*V*e/C (dh') + V*e (dDelta)
       bwd_grad         2K*e/G + 2V*e (v, dO) + 8 (gamma, beta) + C*e (Ainv) + 2K*V*e/C (h, dh')
                        + 2V*e (Delta, dDelta) + 2K*4 (dq, dk partials) + V*e (dv) + 8 (dg, dbeta)
       bwd_final        2K*4 (partials) + 2K*e/G (dq, dk)
@@ -100,15 +101,20 @@ def kernel_bytes(name, w, saved=False):
     hc = nc * Hv * K * V * 2
     d16 = ntok * Hv * V * 2
     part = ntok * Hv * K * 4
+    wb = ntok * Hv * K * 2      # w (bf16)
+    ub = ntok * Hv * V * 4      # u (fp32)
+    pb = nc * Hv * C * C * 2    # P (bf16)
+    prep3 = 2 * qk1 + v1 + 2 * gam + gam + wb + ub + pb
     table = {
         "prep_simt": qk1 + 2 * gam + gam + ainv,               # k, g, beta -> gamma, Ainv
-        "prep_tc": qk1 + 2 * gam + gam + 2 * ainv + (ainv if saved else 0),
+        "prep_tc": qk1 + 2 * gam + gam + ainv,
+        "prep3": prep3 + (ainv if saved else 0),                # q,k,v,g,beta -> gamma,w,u,P[,Ainv]
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
         "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
-        "fwd_hybrid": 2 * qk1 + v1 + gam + 2 * ainv + h0 + v1 + st,
-        "bwd_prep_tc": qk1 + 2 * gam + gam + 2 * ainv + (0 if saved else ainv),
-        "bwd_recompute": qk1 + v1 + gam + 2 * ainv + h0 + hc + d16,
-        "bwd_dh": 2 * qk1 + v1 + ainv + gam + st + hc + d16 + st,
+        "fwd_hybrid": 2 * qk1 + wb + ub + pb + gam + h0 + v1 + st,  # q,k,w,u,P,gamma,h0 -> o,final
+        "bwd_prep3": prep3 + (0 if saved else ainv),
+        "bwd_recompute": qk1 + wb + ub + gam + h0 + hc + d16,
+        "bwd_dh": 2 * qk1 + wb + pb + v1 + gam + st + hc + d16 + st,
         "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + 2 * d16 + 2 * part + v1 + 2 * gam,
         "bwd_final": 2 * part + 2 * qk1,
     }

@@ -91,7 +91,8 @@ struct Plan {
     int dtype;
     bool varlen;
     size_t gamma_bytes, ainv_bytes, saved_bytes, seq_info_bytes;
-    size_t wy_bytes;  // scaled inverses for the tensor-core forward (bf16, K = V = 128)
+    bool tc_ok;       // bf16 with K = V = 128: the tensor-core path
+    size_t w_bytes, u_bytes, p_bytes;  // its chunk-prep outputs w (bf16), u (fp32), P (bf16)
     int max_chunks;   // chunks of the longest sequence
     int nseg;         // forward sequence split: segments per sequence (1 = none)
     size_t seg_bytes; // split scratch: c, P, start states of every segment
@@ -106,7 +107,7 @@ struct Plan {
 // that estimate (segments of at least 8 chunks); GDN_NSEG overrides it.
 int choose_nseg(const Plan &P) {
     const Dims &d = P.d;
-    if (P.wy_bytes == 0 || P.max_chunks < 2) return 1;
+    if (!P.tc_ok || P.max_chunks < 2) return 1;
     if (const char *e = getenv("GDN_NSEG")) {
         const int v = atoi(e);
         return v < 1 ? 1 : (v > P.max_chunks ? P.max_chunks : v);
@@ -168,12 +169,15 @@ int make_plan(const gdn_problem *p, Plan *out) {
     P.gamma_bytes = align_up(sizeof(float) * (size_t)d.T_total * d.Hv);
     P.ainv_bytes = align_up((size_t)d.NC * d.Hv * kChunk * kChunk *
                             (p->dtype == GDN_DTYPE_F32 ? sizeof(float) : sizeof(__nv_bfloat16)));
-    P.wy_bytes = (p->dtype == GDN_DTYPE_BF16 && p->K == 128 && p->V == 128)
-                     ? align_up((size_t)d.NC * d.Hv * 2 * kChunk * kChunk * sizeof(__nv_bfloat16))
-                     : 0;
-    // saved = gamma | Ainv | (bf16 K = V = 128) the scaled inverses, so that a
-    // backward given `saved` needs no chunk prep of its own
-    P.saved_bytes = P.gamma_bytes + P.ainv_bytes + P.wy_bytes;
+    P.tc_ok = p->dtype == GDN_DTYPE_BF16 && p->K == 128 && p->V == 128;
+    if (P.tc_ok) {
+        P.w_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.K);
+        P.u_bytes = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.V);
+        P.p_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * kChunk * kChunk);
+    }
+    // saved = gamma | Ainv | (bf16 K = V = 128) w, u, P, so that a backward
+    // given `saved` needs no chunk prep of its own
+    P.saved_bytes = P.gamma_bytes + P.ainv_bytes + P.w_bytes + P.u_bytes + P.p_bytes;
     if (P.varlen) {
         for (int n = 0; n < p->num_seqs; ++n)
             P.max_chunks = std::max(P.max_chunks, (p->cu_seqlens_host[n + 1] - p->cu_seqlens_host[n] + kChunk - 1) / kChunk);
@@ -245,12 +249,24 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
 
 bool tc_bwd_path(const Plan &P) {
     return !(P.dtype == GDN_DTYPE_F32 || (getenv("GDN_IMPL") && strcmp(getenv("GDN_IMPL"), "simt") == 0)) &&
-           tc_bwd_supported(P.d, P.dtype) && P.wy_bytes > 0;
+           tc_bwd_supported(P.d, P.dtype) && P.tc_ok;
+}
+
+// Pointers into a saved buffer (or the workspace's copy of one): gamma | Ainv | w | u | P.
+void set_saved_ptrs(FwdArgs &a, char *sv, const Plan &P) {
+    a.gamma = (float *)sv;
+    a.ainv = sv + P.gamma_bytes;
+    if (P.tc_ok) {
+        char *x = sv + P.gamma_bytes + P.ainv_bytes;
+        a.w16 = x;
+        a.u32 = (float *)(x + P.w_bytes);
+        a.p16 = x + P.w_bytes + P.u_bytes;
+    }
 }
 
 // Either backward path fits in the size reported to callers.
 size_t bwd_ws_bytes(const Plan &P) {
-    const size_t a = bwd_layout(P).total, b = P.wy_bytes > 0 ? tc_bwd_layout(P).total : 0;
+    const size_t a = bwd_layout(P).total, b = P.tc_ok ? tc_bwd_layout(P).total : 0;
     return a > b ? a : b;
 }
 
@@ -392,17 +408,24 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.dtype = P.dtype;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0;
     a.o = o; a.final_state = final_state;
-    a.gamma = (float *)sv;
-    a.ainv = sv + P.gamma_bytes;
-    a.wy = P.wy_bytes ? sv + P.gamma_bytes + P.ainv_bytes : nullptr;
+    set_saved_ptrs(a, sv, P);
     a.status = status;
     a.stream = st;
     a.nseg = 1;
     const char *which = getenv("GDN_FWD");
     const bool tc = !use_simt(P.dtype) && tc_fwd_supported(a);
-    const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.wy_bytes > 0;
-    if (hybrid && !saved) a.ainv = nullptr;  // the hybrid forward reads only the scaled inverses
-    if ((rc = launch_prep(a)) != GDN_OK) return rc;
+    const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.tc_ok;
+    if (hybrid) {
+        if (!saved) a.ainv = nullptr;  // the hybrid forward reads w, u, P; Ainv only for `saved`
+        TimedLaunch t("prep3", st);
+        if (launch_prep3(a) != cudaSuccess) return GDN_ERR_CUDA;
+    } else {
+        if ((rc = launch_prep(a)) != GDN_OK) return rc;
+        if (saved && P.tc_ok) {  // keep `saved` complete for a tensor-core backward
+            TimedLaunch t("prep3", st);
+            if (launch_prep3(a) != cudaSuccess) return GDN_ERR_CUDA;
+        }
+    }
     if (hybrid && P.nseg > 1) {
         // sequence split: segment pass (c, P) -> composition of start states -> output pass
         float *seg = (float *)(ws + P.seq_info_bytes + P.saved_bytes);
@@ -476,13 +499,14 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         f.status = status;
         f.stream = st;
         f.nseg = 1;
-        // gamma | Ainv | scaled inverses: from the forward's `saved`, else made here
+        // gamma | Ainv | w | u | P: from the forward's `saved`, else made here
         char *sv = saved ? (char *)saved : ws + T.saved;
-        f.gamma = (float *)sv;
-        f.ainv = sv + P.gamma_bytes;
-        f.wy = sv + P.gamma_bytes + P.ainv_bytes;
+        set_saved_ptrs(f, sv, P);
         const void *ainv = f.ainv;
-        if (!saved && (rc = launch_prep(f, "bwd_prep_tc", "bwd_prep_simt")) != GDN_OK) return rc;
+        if (!saved) {
+            TimedLaunch t("bwd_prep3", st);
+            if (launch_prep3(f) != cudaSuccess) return GDN_ERR_CUDA;
+        }
         f.o = nullptr;
         f.final_state = nullptr;
         f.h_chunks16 = ws + T.hc;
@@ -504,7 +528,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         b.stream = st;
         {
             TimedLaunch t("bwd_dh", st);
-            if (launch_bwd_dh_tc(b, f.wy, ws + T.dhc, ws + T.ddelta) != cudaSuccess) return GDN_ERR_CUDA;
+            if (launch_bwd_dh_tc(b, f.w16, f.p16, ws + T.dhc, ws + T.ddelta) != cudaSuccess) return GDN_ERR_CUDA;
         }
         {
             TimedLaunch t("bwd_grad", st);

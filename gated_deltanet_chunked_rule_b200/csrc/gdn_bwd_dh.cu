@@ -13,18 +13,20 @@
 // per-chunk gradient kernel; dh0 (fp32) is the gradient at the sequence start.
 //
 // Same organisation as the forward kernel (gdn_fwd2.cu): one CTA per
-// (sequence, value head, 32-column slice of V) with 576 threads,
+// (sequence, value head, 32-column slice of V), w and P = M o Q K^T of every
+// chunk from the chunk-prep kernel through a TMA ring, 416 threads:
 //   warps 0-7   chain: dh' (128 x 32 fp32) in mma.sync fragments; per chunk
-//               A = K dh' then dh = e^{gamma_C} dh' + X + (-w)^T dDelta;
-//   warps 8-15  aux: P = scale (M o S) and dO' = scale e^gamma o dO into shared
-//               memory for issuer B; -w, Y, X from tensor memory into shared
-//               memory for the chain;
-//   warp 16     issuer A: TMA prologue, S = Q K^T and W = Aw K (tcgen05);
-//   warp 17     issuer B: Y = P^T dO and X = Q^T dO' (tcgen05), TMA refills.
-// None of the tcgen05 products depends on the chain, so they run ahead of it,
-// bounded by the double-buffered tensor memory and the 3-deep TMA ring.
-// Hand-over is by release/acquire counters and, where the hardware signals
-// completion, mbarriers with a single consumer; every wait is bounded.
+//               A = K dh', dDelta = e^{gamma_C - gamma} A + scale Y, then
+//               dh = e^{gamma_C} dh' + X - w^T dDelta, with Y and X read
+//               straight from tensor memory (the 16x256b load layout is the
+//               mma.sync accumulator layout, and chain warp p sits on TMEM
+//               sub-partition p);
+//   warps 8-11  aux: dO' = scale e^gamma o dO into shared memory;
+//   warp 12     issuer: TMA ring (q, k, w, P, dO per chunk) and, on tcgen05,
+//               Y = P^T dO and X = Q^T dO' into double-buffered TMEM.
+// Y and X do not depend on the chain, so they are ready one or two chunks
+// ahead of it. Hand-over by release/acquire counters and mbarriers; every wait
+// is bounded.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -37,51 +39,42 @@ namespace {
 using namespace sm100;
 using namespace warp;
 
-constexpr int kThreads = 576;
-constexpr int kRole = 256;
+constexpr int kThreads = 416;
+constexpr int kRole = 256;  // chain threads
+constexpr int kAux = 128;
 constexpr int kBV = 32;
 constexpr int kStages = 3;
 
 // ---- shared memory (bytes from a 1024-aligned base)
 constexpr int kHb = 0;          // 8192       dh' (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16, chain only
-constexpr int kDb = 8192;       // 4096       dDelta (bf16): (n/8)*1024 + (t/8)*128 + (t%8)*16, chain only
+constexpr int kDb = 8192;       // 4096       -dDelta (bf16): (n/8)*1024 + (t/8)*128 + (t%8)*16, chain only
 constexpr int kDO2 = 12288;     // 2 x 4096   dO' (bf16), layout of kDb (B of X)
-constexpr int kP = 20480;       // 2 x 8192   P [r][s], 128-byte swizzle (A of Y, read transposed)
-constexpr int kWs = 36864;      // 16384      -w (bf16) in the k tile's layout (two 64-column halves)
-constexpr int kY = 53248;       // 9216       Y (fp32) [t][36]
-constexpr int kX = 62464;       // 18432      X (fp32) [k][36]
-constexpr int kStage0 = 81920;  // TMA ring
-constexpr int kQ = 0, kK = 16384, kAw = 32768, kDO = 40960, kStageBytes = 45056;
-constexpr int kTxBytes = 16384 + 16384 + 8192 + 4096;
+constexpr int kStage0 = 20480;  // TMA ring
+// per stage: q, k, w [64][128] bf16 (two 64-column halves, 128-byte swizzle),
+// P [64][64] bf16 (128-byte swizzle), dO [64][32] bf16 (64-byte swizzle)
+constexpr int kQ = 0, kK = 16384, kW = 32768, kP = 49152, kDO = 57344, kStageBytes = 61440;
+constexpr int kTxBytes = 3 * 16384 + 8192 + 4096;
 constexpr int kSmall = kStage0 + kStages * kStageBytes;
-constexpr int kSmemBytes = kSmall + 2560 + 1024;
-static_assert(kX + 18432 <= kStage0 && kP % 1024 == 0 && kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 &&
-                  kSmemBytes <= 232448,
-              "shared memory layout");
+constexpr int kSmemBytes = kSmall + 2048 + 1024;
+static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory layout");
 
-// Tensor memory: two buffers of 256 columns, S | W | Y | X.
-constexpr uint32_t kColS = 0, kColW = 64, kColY = 192, kColX = 224, kABuf = 256, kTmemCols = 512;
+// Tensor memory: two buffers of 64 columns, Y (M = 64) | X (M = 128).
+constexpr uint32_t kColY = 0, kColX = 32, kYBuf = 64, kTmemCols = 128;
 
-struct __align__(16) Gates {
-    float gam[64], egam[64];
-};
-
-// Counters (number of iterations finished by the producer).
-enum Ctr { kTmemA, kPReady, kReady, kWFree, kStage, kNumCtr };
+enum Ctr { kPReady, kStage, kNumCtr };
 
 struct Small {
     uint64_t full[kStages];
-    uint64_t mmaA[2], mmaB[2];
+    uint64_t mmaB[2];
     uint32_t ctr[kNumCtr];
-    int loads_issued, loads_landed;
+    int loads_issued, loads_landed, mma_issued, mma_seen;
     uint32_t tmem_base;
     int abort_flag;
-    Gates gates[3];
 };
-static_assert(sizeof(Small) <= 2560, "small area");
-static_assert(kSmall % 16 == 0 && offsetof(Small, gates) % 16 == 0, "small area alignment");
+static_assert(sizeof(Small) <= 2048, "small area");
 
-__device__ __forceinline__ bool rsync(int id, bool pred) { return role_sync_and<kRole>(id, pred); }
+__device__ __forceinline__ bool chain_sync(bool pred) { return role_sync_and<kRole>(1, pred); }
+__device__ __forceinline__ bool aux_sync(bool pred) { return role_sync_and<kAux>(2, pred); }
 
 struct BwdDhParams {
     Dims d;
@@ -96,8 +89,8 @@ struct BwdDhParams {
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_wy,
-              const BwdDhParams prm) {
+              const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
+              const __grid_constant__ CUtensorMap tm_do, const BwdDhParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -114,16 +107,14 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm->full[s], 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm->mmaA[b], 1);
-            mbar_init(&sm->mmaB[b], 1);
-        }
+        mbar_init(&sm->mmaB[0], 1);
+        mbar_init(&sm->mmaB[1], 1);
         for (int c = 0; c < kNumCtr; ++c) sm->ctr[c] = 0;
-        sm->loads_issued = sm->loads_landed = 0;
+        sm->loads_issued = sm->loads_landed = sm->mma_issued = sm->mma_seen = 0;
         sm->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 16) {
+    if (warp == 12) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -135,26 +126,17 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // iteration it handles chunk nch - 1 - it of the sequence
     auto chunk_of = [&](int it) { return nch - 1 - it; };
-    auto issue_loads = [&](int it) {
-        const int s = it % kStages;
-        uint8_t *st = smem + kStage0 + s * kStageBytes;
-        const int ci = chunk_of(it);
-        const int t0 = sr.start + ci * kChunk;
-        const int cg = sr.chunk0 + ci;
-        mbar_arrive_expect_tx(&sm->full[s], kTxBytes);
-        atomicAdd(&sm->loads_issued, 1);
-        tma_load_3d(st + kQ, &tm_q, &sm->full[s], 0, hq, t0);
-        tma_load_3d(st + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
-        tma_load_3d(st + kK, &tm_k, &sm->full[s], 0, hq, t0);
-        tma_load_3d(st + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
-        tma_load_2d(st + kAw, &tm_wy, &sm->full[s], 0, ((cg * d.Hv + h) * 2 + 1) * kChunk);
-        tma_load_3d(st + kDO, &tm_do, &sm->full[s], c0, h, t0);
+    auto gamma_at = [&](int it, int r) {
+        const int ci = chunk_of(it), len = min(kChunk, sr.len - ci * kChunk);
+        return prm.gamma[(size_t)(sr.start + ci * kChunk + min(r, len - 1)) * d.Hv + h];
     };
 
     if (warp < 8) {
         // =========================================================== chain
         const int p = warp & 3, cb = (warp >> 2) * 2;  // state rows 32p.., n-tiles cb, cb+1
         const int g = lane >> 2, c4 = lane & 3;
+        const uint32_t lane_base = (uint32_t)(p * 32) << 16;
+        const float scl = prm.scale;
         float hf[2][2][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8(cb+nt)+2c4(+1)
         {
             const float *src = prm.dht ? prm.dht + ((size_t)n * d.Hv + h) * K * V : nullptr;
@@ -184,10 +166,19 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         };
         write_hb();
         bool ok = true;
+        float gl = 0.f, gt0 = 0.f, gt1 = 0.f;
+        if (nch > 0) gl = gamma_at(0, 63), gt0 = gamma_at(0, 16 * p + g), gt1 = gamma_at(0, 16 * p + g + 8);
         for (int it = 0; it < nch && ok; ++it) {
             const int ci = chunk_of(it);
             const int len = min(kChunk, sr.len - ci * kChunk);
             const int t0 = sr.start + ci * kChunk;
+            const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
+            // stage landed (and every warp's dh' is in kHb: the barrier orders them)
+            ok = chain_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag));
+            if (!ok) break;
+            if (tid == 0) sm->loads_landed = it + 1;
+            const float gC = gl, gtok[2] = {gt0, gt1};
+            if (it + 1 < nch) gl = gamma_at(it + 1, 63), gt0 = gamma_at(it + 1, 16 * p + g), gt1 = gamma_at(it + 1, 16 * p + g + 8);
             {  // dh' of this chunk, rounded as the products read it
                 __nv_bfloat16 *hc = prm.dh_chunks + ((size_t)(sr.chunk0 + ci) * d.Hv + h) * K * V + c0;
 #pragma unroll
@@ -201,16 +192,22 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                 pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
                     }
             }
-            // -w, Y, X of this chunk are in shared memory (and dh' in kHb from every warp)
-            ok = rsync(1, wait_ge(&ctr[kReady], it + 1, abort_flag));
+            // ---- Y and X of this chunk from tensor memory (issued now, waited after A)
+            ok = chain_sync(wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag));
             if (!ok) break;
-            const Gates &G = sm->gates[it % 3];
-            const float gl = G.gam[63];
-            const float gtok[2] = {G.gam[16 * p + g], G.gam[16 * p + g + 8]};
+            if (tid == 0) sm->mma_seen = it + 1;
+            tc_fence_after();
+            uint32_t yr[8], xr0[8], xr1[8];
+            {
+                const uint32_t tb = tmem + (it & 1) * kYBuf + 8 * cb;
+                tmem_ld16x256_x2_nowait(tb + lane_base + kColY, yr);                       // tokens 16p + (g, g+8)
+                tmem_ld16x256_x2_nowait(tb + lane_base + kColX, xr0);                      // state rows 32p + (g, g+8)
+                tmem_ld16x256_x2_nowait(tb + lane_base + ((uint32_t)16 << 16) + kColX, xr1);  // rows 32p + 16 + ..
+            }
             // ---- A = K dh' : tokens 16p..16p+15, columns of n-tiles cb, cb+1
             float acc[2][4] = {};
             {
-                const uint32_t kt = sb + kStage0 + (it % kStages) * kStageBytes + kK;
+                const uint32_t kt = st + kK;
                 const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int mi = lane >> 3;
                 uint32_t a[2][4], b[2][4];
@@ -227,56 +224,54 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     hmma(acc[1], a[ks & 1], b[ks & 1][2], b[ks & 1][3]);
                 }
             }
-            // ---- dDelta = e^{gamma_C - gamma} A + Y  -> ddelta (global) and kDb
+            tmem_wait_ld3(yr, xr0, xr1);
+            tc_fence_before();
+            // ---- dDelta = e^{gamma_C - gamma} A + scale Y  -> ddelta (global), -dDelta -> kDb
             {
-                const float *Y = reinterpret_cast<const float *>(smem + kY);
                 const uint32_t db = sb + kDb + c4 * 4;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int tok = 16 * p + g + half * 8;
                     const bool live = tok < len;
-                    const float sc = __expf(gl - gtok[half]);
+                    const float sc = __expf(gC - gtok[half]);
                     const uint32_t off = (tok >> 3) * 128 + (tok & 7) * 16;
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const int col = 8 * (cb + nt) + 2 * c4;
-                        const float2 y = *reinterpret_cast<const float2 *>(Y + tok * 36 + col);
-                        const float x0 = live ? fmaf(sc, acc[nt][2 * half], y.x) : 0.f;
-                        const float x1 = live ? fmaf(sc, acc[nt][2 * half + 1], y.y) : 0.f;
-                        const uint32_t pk = pack_bf16(x0, x1);
-                        st_shared_b32(db + (cb + nt) * 1024 + off, pk);
+                        const float y0 = __uint_as_float(yr[4 * nt + 2 * half]), y1 = __uint_as_float(yr[4 * nt + 2 * half + 1]);
+                        const float x0 = live ? fmaf(sc, acc[nt][2 * half], scl * y0) : 0.f;
+                        const float x1 = live ? fmaf(sc, acc[nt][2 * half + 1], scl * y1) : 0.f;
+                        st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(-x0, -x1));
                         if (live)
-                            *reinterpret_cast<uint32_t *>(prm.ddelta + ((size_t)(t0 + tok) * d.Hv + h) * V + c0 + col) = pk;
+                            *reinterpret_cast<uint32_t *>(prm.ddelta + ((size_t)(t0 + tok) * d.Hv + h) * V + c0 + col) =
+                                pack_bf16(x0, x1);
                     }
                 }
             }
-            rsync(1, true);  // every warp reads all 64 tokens of dDelta below
-            // ---- dh = e^{gamma_C} dh' + X + (-w)^T dDelta : rows 32p..+31, 16 columns, K = 64 tokens
+            chain_sync(true);  // every warp reads all 64 tokens of dDelta below
+            // ---- dh = e^{gamma_C} dh' + X + w^T (-dDelta) : rows 32p..+31, 16 columns, K = 64 tokens
             {
-                const float eC = __expf(gl);
-                const float *X = reinterpret_cast<const float *>(smem + kX);
+                const float eC = __expf(gC);
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint32_t(&xr)[8] = mt ? xr1 : xr0;
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int dim = 32 * p + 16 * mt + g + half * 8;
+                    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const float2 x = *reinterpret_cast<const float2 *>(X + dim * 36 + 8 * (cb + nt) + 2 * c4);
-                            hf[mt][nt][2 * half] = fmaf(eC, hf[mt][nt][2 * half], x.x);
-                            hf[mt][nt][2 * half + 1] = fmaf(eC, hf[mt][nt][2 * half + 1], x.y);
-                        }
-                    }
+                        for (int q = 0; q < 4; ++q) hf[mt][nt][q] = fmaf(eC, hf[mt][nt][q], __uint_as_float(xr[4 * nt + q]));
+                }
+                const uint32_t wt = st + kW;
                 const int mi = lane >> 3;
                 uint32_t b[2][4], a[2][2][4];
                 auto load = [&](int ks, int buf) {
                     ldsm_x4_t(b[buf], sb + kDb + (cb + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
-                        // A = (-w)^T rows (state rows) 32p+16mt.., cols (tokens) 16ks..
+                        // A = w^T rows (state rows) 32p+16mt.., cols (tokens) 16ks..: the
+                        // token-major, 128-byte-swizzled w tile read transposed
                         const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
                         const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
-                        ldsm_x4_t(a[buf][mt], sb + kWs + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
+                        ldsm_x4_t(a[buf][mt], wt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
                     }
                 };
                 load(0, 0);
@@ -290,11 +285,8 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
-            rsync(1, true);  // all reads of kHb, kDb, kWs, kX, kY and the k tile are done
-            if (tid == 0) {
-                publish(&ctr[kWFree], it + 1);
-                publish(&ctr[kStage], it + 1);
-            }
+            chain_sync(true);  // all reads of kHb, kDb, the stage and this TMEM buffer are done
+            if (tid == 0) publish(&ctr[kStage], it + 1);
             write_hb();
         }
         if (!ok) {
@@ -313,69 +305,32 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
                     }
         }
-    } else if (warp < 16) {
+    } else if (warp < 12) {
         // ============================================================= aux
-        const int atid = tid - kRole, aw = warp - 8;
-        const int ap = aw & 3, ah = aw >> 2;
-        const uint32_t lane_base = (uint32_t)(ap * 32) << 16;
-        const int ag = lane >> 2, ac = lane & 3;
-        const int ar0 = ap * 16 + ag, ar1 = ar0 + 8;
+        const int atid = tid - kRole;
         const float scl = prm.scale;
         bool ok = true;
-        float pg = 0.f;
-        auto fetch_gate = [&](int it) {
-            if (atid < kChunk && it < nch) {
-                const int ci = chunk_of(it);
-                const int t0 = sr.start + ci * kChunk, len = min(kChunk, sr.len - ci * kChunk);
-                pg = prm.gamma[(size_t)(t0 + min(atid, len - 1)) * d.Hv + h];
-            }
-        };
-        auto store_gate = [&](int it) {
-            if (atid < kChunk) {
-                sm->gates[it % 3].gam[atid] = pg;
-                sm->gates[it % 3].egam[atid] = __expf(pg);
-            }
-        };
-        // P and dO' of iteration it into buffer it & 1 (its previous readers, Y and X of
-        // iteration it - 2, have completed: this role saw mmaB of it - 2)
-        auto make_p = [&](int it) -> bool {
-            const int len = min(kChunk, sr.len - chunk_of(it) * kChunk);
-            if (!rsync(2, wait_bar(&sm->mmaA[it & 1], (it >> 1) & 1, abort_flag) &&
-                              wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag)))
-                return false;
-            tc_fence_after();
-            if (atid == 0) sm->loads_landed = it + 1;
-            store_gate(it);
-            fetch_gate(it + 1);
-            rsync(2, true);  // gates of this chunk visible to the role
-            const Gates &G = sm->gates[it % 3];
-            {
-                float v[16];
-                tmem_ld16x256_x4(tmem + lane_base + (it & 1) * kABuf + kColS + 32 * ah, v);
-                const float gr0 = G.gam[ar0], gr1 = G.gam[ar1];
-                const bool l0 = ar0 < len, l1 = ar1 < len;
-                const uint32_t pb = sb + kP + (it & 1) * 8192;
+        // thread: 16-byte chunks e = atid and atid + 128 of the 64 x 32 dO tile
+        const int ta = atid >> 2, tb2 = (atid + kAux) >> 2, cc = atid & 3;
+        float ga = 0.f, gb = 0.f;
+        if (nch > 0) ga = gamma_at(0, ta), gb = gamma_at(0, tb2);
+        for (int it = 0; it < nch && ok; ++it) {
+            const int ci = chunk_of(it);
+            const int len = min(kChunk, sr.len - ci * kChunk);
+            // the stage has landed; X of iteration it - 2 (the last reader of dO'[it % 2]) is done
+            ok = aux_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
+                          (it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag)));
+            if (!ok) break;
+            const float fa = ta < len ? scl * __expf(ga) : 0.f, fb = tb2 < len ? scl * __expf(gb) : 0.f;
+            if (it + 1 < nch) ga = gamma_at(it + 1, ta), gb = gamma_at(it + 1, tb2);
+            const uint32_t stg = sb + kStage0 + (it % kStages) * kStageBytes + kDO;
+            const uint32_t ob = sb + kDO2 + (it & 1) * 4096;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int s0 = 32 * ah + 8 * i + 2 * ac;
-                    const float2 gs = *reinterpret_cast<const float2 *>(&G.gam[s0]);
-                    const float x00 = (l0 && s0 <= ar0) ? scl * __expf(gr0 - gs.x) * v[4 * i] : 0.f;
-                    const float x01 = (l0 && s0 + 1 <= ar0) ? scl * __expf(gr0 - gs.y) * v[4 * i + 1] : 0.f;
-                    const float x10 = (l1 && s0 <= ar1) ? scl * __expf(gr1 - gs.x) * v[4 * i + 2] : 0.f;
-                    const float x11 = (l1 && s0 + 1 <= ar1) ? scl * __expf(gr1 - gs.y) * v[4 * i + 3] : 0.f;
-                    const int ch = 4 * ah + i;
-                    st_shared_b32(pb + (ar0 >> 3) * 1024 + (ar0 & 7) * 128 + ((ch ^ (ar0 & 7)) << 4) + 4 * ac,
-                                  pack_bf16(x00, x01));
-                    st_shared_b32(pb + (ar1 >> 3) * 1024 + (ar1 & 7) * 128 + ((ch ^ (ar1 & 7)) << 4) + 4 * ac,
-                                  pack_bf16(x10, x11));
-                }
-            }
-            {  // dO' = scale e^gamma dO (zero past the sequence end): one 16-byte chunk per thread
-                const int t = atid >> 2, c = atid & 3;
-                const uint32_t src = sb + kStage0 + (it % kStages) * kStageBytes + kDO + t * 64 +
-                                     ((c ^ ((t >> 1) & 3)) << 4);
-                const uint4 raw = ld_shared_v4(src);
-                const float f = t < len ? scl * G.egam[t] : 0.f;
+            for (int e2 = 0; e2 < 2; ++e2) {
+                const int t = e2 ? tb2 : ta;
+                const float f = e2 ? fb : fa;
+                // dO tile: 64-byte rows, 16-byte chunks XOR ((row / 2) % 4)
+                const uint4 raw = ld_shared_v4(stg + t * 64 + ((cc ^ ((t >> 1) & 3)) << 4));
                 const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
                 uint32_t o[4];
 #pragma unroll
@@ -383,129 +338,65 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const float2 x = unpack_bf16(w[e]);
                     o[e] = pack_bf16(f * x.x, f * x.y);
                 }
-                st_shared_v4(sb + kDO2 + (it & 1) * 4096 + c * 1024 + (t >> 3) * 128 + (t & 7) * 16, o[0], o[1], o[2],
-                             o[3]);
+                st_shared_v4(ob + cc * 1024 + (t >> 3) * 128 + (t & 7) * 16, o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async();
-            tc_fence_before();
-            rsync(2, true);
+            aux_sync(true);
             if (atid == 0) publish(&ctr[kPReady], it + 1);
-            return true;
-        };
-        if (nch > 0) {
-            fetch_gate(0);
-            ok = make_p(0);
-        }
-        for (int it = 0; it < nch && ok; ++it) {
-            const int len = min(kChunk, sr.len - chunk_of(it) * kChunk);
-            const uint32_t abuf = (it & 1) * kABuf;
-            // ---- -w, Y, X -> shared memory once the chain is done with the previous chunk's
-            ok = rsync(2, wait_ge(&ctr[kWFree], it, abort_flag) &&
-                              wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            {
-                float v[32];
-                tmem_ld16x256_x8(tmem + lane_base + abuf + kColW + ah * 64, v);  // columns 64 ah .. +63 of w
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int r = half ? ar1 : ar0;
-                    const bool live = r < len;
-                    const uint32_t rowb = sb + kWs + ah * 8192 + r * 128 + 4 * ac;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        st_shared_b32(rowb + ((i ^ (r & 7)) << 4),
-                                      live ? pack_bf16(-v[4 * i + 2 * half], -v[4 * i + 2 * half + 1]) : 0u);
-                }
-                float y[8];
-                tmem_ld16x256_x2(tmem + lane_base + abuf + kColY + 16 * ah, y);  // columns 16 ah .. +15 of Y
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int r = half ? ar1 : ar0;
-                    const bool live = r < len;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        st_shared_v2f(sb + kY + (r * 36 + 16 * ah + 8 * i + 2 * ac) * 4, live ? y[4 * i + 2 * half] : 0.f,
-                                      live ? y[4 * i + 2 * half + 1] : 0.f);
-                }
-                float x[16];
-                tmem_ld32x16(tmem + lane_base + abuf + kColX + 16 * ah, x);  // state row 32 ap + lane
-                const uint32_t xb = sb + kX + ((ap * 32 + lane) * 36 + 16 * ah) * 4;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) st_shared_v4f(xb + 16 * i, x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
-            }
-            tc_fence_before();
-            rsync(2, true);
-            if (atid == 0) {
-                publish(&ctr[kReady], it + 1);
-                publish(&ctr[kTmemA], it + 1);
-            }
-            if (it + 1 < nch) ok = make_p(it + 1);
         }
         if (!ok) {
             if (atid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
             *abort_flag = 1;
         }
-    } else if (warp == 16) {
-        // ================================================== MMA issuer A
-        if (lane == 0) {
-            bool ok = true;
-            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
-            const uint32_t id_S = idesc_bf16(64, 64, false, false);
-            const uint32_t id_W = idesc_bf16(64, 128, false, true);
-            for (int it = 0; it < nch && ok; ++it) {
-                const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
-                ok = wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
-                     wait_ge(&ctr[kTmemA], it >= 1 ? it - 1 : 0, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t tb = tmem + (it & 1) * kABuf;
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tb + kColW, smem_desc(st + kAw + ks * 32, 16, 1024, kSw128),
-                             smem_desc(st + kK + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16(tb + kColS, smem_desc(st + kQ + off, 16, 1024, kSw128),
-                             smem_desc(st + kK + off, 16, 1024, kSw128), id_S, ks > 0);
-                }
-                mma_commit(&sm->mmaA[it & 1]);
-            }
-            if (!ok) {
-                set_status(prm.status, GDN_ERR_TIMEOUT);
-                *abort_flag = 1;
-            }
-        }
-        __syncwarp();
     } else {
-        // ================================================== MMA issuer B
+        // ========================================================== issuer
         if (lane == 0) {
             bool ok = true;
+            auto issue_loads = [&](int it) {
+                const int s = it % kStages;
+                uint8_t *stg = smem + kStage0 + s * kStageBytes;
+                const int ci = chunk_of(it);
+                const int t0 = sr.start + ci * kChunk;
+                const int cg = sr.chunk0 + ci;
+                mbar_arrive_expect_tx(&sm->full[s], kTxBytes);
+                atomicAdd(&sm->loads_issued, 1);
+                tma_load_3d(stg + kQ, &tm_q, &sm->full[s], 0, hq, t0);
+                tma_load_3d(stg + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
+                tma_load_3d(stg + kK, &tm_k, &sm->full[s], 0, hq, t0);
+                tma_load_3d(stg + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
+                tma_load_3d(stg + kW, &tm_w, &sm->full[s], 0, h, t0);
+                tma_load_3d(stg + kW + 8192, &tm_w, &sm->full[s], 64, h, t0);
+                tma_load_2d(stg + kP, &tm_p, &sm->full[s], 0, (cg * d.Hv + h) * kChunk);
+                tma_load_3d(stg + kDO, &tm_do, &sm->full[s], c0, h, t0);
+            };
+            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
             const uint32_t id_Y = idesc_bf16(64, 32, true, true);
             const uint32_t id_X = idesc_bf16(128, 32, true, true);
             for (int it = 0; it < nch && ok; ++it) {
-                const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
-                ok = wait_ge(&ctr[kPReady], it + 1, abort_flag) &&
-                     wait_ge(&ctr[kTmemA], it >= 1 ? it - 1 : 0, abort_flag);
+                // refill the stage of iteration it - 1 with iteration it + 2 once the chain is
+                // done with it (which also means its Y, X and dO' are consumed)
+                if (it >= 1 && it + 2 < nch) {
+                    ok = wait_ge(&ctr[kStage], it, abort_flag);
+                    if (!ok) break;
+                    issue_loads(it + 2);
+                }
+                // Y, X of iteration it into buffer it % 2 once dO' is written and the chain
+                // has read that buffer's previous contents (iteration it - 2)
+                ok = wait_ge(&ctr[kPReady], it + 1, abort_flag) && wait_ge(&ctr[kStage], it >= 1 ? it - 1 : 0, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t tb = tmem + (it & 1) * kABuf;
-                const uint32_t pb = sb + kP + (it & 1) * 8192, ob = sb + kDO2 + (it & 1) * 4096;
+                const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
+                const uint32_t tb = tmem + (it & 1) * kYBuf, ob = sb + kDO2 + (it & 1) * 4096;
                 for (int ks = 0; ks < 4; ++ks) {
-                    // Y = P^T dO: A = P read transposed (MN-major), B = the dO tile; K = 16 rows of P per step
-                    mma_bf16(tb + kColY, smem_desc(pb + ks * 2048, 8192, 1024, kSw128),
+                    // Y = P^T dO: A = P read transposed (MN-major), B = the dO tile; 16 rows of P per step
+                    mma_bf16(tb + kColY, smem_desc(st + kP + ks * 2048, 8192, 1024, kSw128),
                              smem_desc(st + kDO + ks * 1024, 4096, 512, kSw64), id_Y, ks > 0);
                     // X = Q^T dO': A = the q tile read transposed (MN-major, two 64-row halves)
                     mma_bf16(tb + kColX, smem_desc(st + kQ + ks * 2048, 8192, 1024, kSw128),
                              smem_desc(ob + ks * 256, 128, 1024, kSwNone), id_X, ks > 0);
                 }
                 mma_commit(&sm->mmaB[it & 1]);
-                // refill the stage of iteration it - 1 with iteration it + 2 once the chain is done
-                // with its k tile and the aux role has seen this stage's products of it - 1 complete
-                if (it >= 1 && it + 2 < nch) {
-                    ok = wait_ge(&ctr[kStage], it, abort_flag) && wait_ge(&ctr[kTmemA], it, abort_flag);
-                    if (!ok) break;
-                    issue_loads(it + 2);
-                }
+                sm->mma_issued = it + 1;
             }
             if (!ok) {
                 set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -518,15 +409,17 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) {
-        // let every TMA load still in flight land (bounded) before the CTA exits
+        // let every TMA load and every MMA still in flight finish (bounded) before the CTA exits
         const uint64_t t0 = globaltimer();
         for (int c = sm->loads_landed; c < sm->loads_issued; ++c)
-            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) &&
-                   globaltimer() - t0 < kWaitNs) {
+            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
+            }
+        for (int c = sm->mma_seen; c < sm->mma_issued; ++c)
+            while (!mbar_try_wait(smem_u32(&sm->mmaB[c & 1]), (c >> 1) & 1) && globaltimer() - t0 < kWaitNs) {
             }
     }
     __syncthreads();
-    if (warp == 16) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -538,23 +431,27 @@ bool tc_bwd_supported(const Dims &d, int dtype) {
     return dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128;
 }
 
-cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *wy, void *dh_chunks16, void *ddelta16) {
+cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
-    CUtensorMap mq, mk, mdo, mw;
-    const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, (cuuint64_t)(d.T_total > 0 ? d.T_total : 1)};
+    CUtensorMap mq, mk, mw, mp, mdo;
+    const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
+    const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
-    const cuuint32_t bq[3] = {64, 1, 64};
-    const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, (cuuint64_t)(d.T_total > 0 ? d.T_total : 1)};
+    const cuuint32_t b64[3] = {64, 1, 64};
+    const cuuint64_t dw[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sw[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hv * d.K * 2};
+    const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
     const cuuint64_t sv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
     const cuuint32_t bv[3] = {kBV, 1, 64};
-    const cuuint64_t dw[2] = {64, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * 2 * 64};
-    const cuuint64_t sw[1] = {128};
-    const cuuint32_t bw[2] = {64, 64};
-    if (!make_bf16_map(&mq, a.q, 3, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_bf16_map(&mk, a.k, 3, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_bf16_map(&mdo, a.d_o, 3, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_bf16_map(&mw, wy, 2, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B))
+    const cuuint64_t dp[2] = {64, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * 64};
+    const cuuint64_t sp[1] = {128};
+    const cuuint32_t bp[2] = {64, 64};
+    if (!make_bf16_map(&mq, a.q, 3, dq, sq, b64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mk, a.k, 3, dq, sq, b64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mw, w16, 3, dw, sw, b64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mp, p16, 2, dp, sp, bp, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mdo, a.d_o, 3, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     BwdDhParams p;
     p.d = d;
@@ -567,7 +464,7 @@ cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *wy, void *dh_chunks16
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(bwd_dh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    bwd_dh_kernel<<<dim3(d.N, d.Hv, d.V / kBV), kThreads, kSmemBytes, a.stream>>>(mq, mk, mdo, mw, p);
+    bwd_dh_kernel<<<dim3(d.N, d.Hv, d.V / kBV), kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mp, mdo, p);
     return cudaGetLastError();
 }
 

@@ -32,16 +32,6 @@ using namespace warp;
 constexpr int kThreads = 256;  // 8 warps: warp w owns rows 16 (w % 4) .. +15, column half w / 4
 constexpr int C = 64, K = 128, V = 128;
 
-// bf16 tiles, row-major with 16-byte chunks XOR-permuted by (row % 8) so that
-// ldmatrix over 8 consecutive rows touches 8 distinct bank groups.
-struct Tile {
-    uint32_t base;
-    int pitch;  // bytes per row
-};
-__device__ __forceinline__ uint32_t toff(const Tile &t, int row, int col) {
-    return t.base + row * t.pitch + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2;
-}
-
 // ---- shared memory (bytes)
 constexpr int kSQ = 0, kSK = 16384, kSV = 32768 /* later dU */, kSdO = 49152, kSD = 65536, kSdD = 81920;
 constexpr int kSh = 98304, kSdh = 131072, kSA = 163840, kST1 = 172032, kSdG = 180224, kSvec = 188416;
@@ -54,54 +44,6 @@ struct Vecs {
     float scal[8];                     // per-warp partial of the chunk-level dgamma_C term
 };
 static_assert(sizeof(Vecs) <= 4096, "vector area");
-
-// C (16 x 8 NT) += A (16 x kdim) B (kdim x 8 NT) on one warp.
-// A_T: A stored [k][m] (read transposed); B_KN: B stored [k][n] (else [n][k]).
-template <int NT, bool A_T, bool B_KN>
-__device__ __forceinline__ void wgemm(float (&c)[NT][4], const Tile &A, const Tile &B, int m0, int n0, int kdim,
-                                      int lane) {
-    const int mi = lane >> 3, r8 = lane & 7;
-#pragma unroll 2
-    for (int k0 = 0; k0 < kdim; k0 += 16) {
-        uint32_t a[4];
-        if (!A_T) ldsm_x4(a, toff(A, m0 + r8 + (mi & 1) * 8, k0 + (mi >> 1) * 8));
-        else ldsm_x4_t(a, toff(A, k0 + (mi >> 1) * 8 + r8, m0 + (mi & 1) * 8));
-#pragma unroll
-        for (int j = 0; j < NT; j += 2) {
-            uint32_t b[4];
-            if (!B_KN) ldsm_x4(b, toff(B, n0 + j * 8 + (mi >> 1) * 8 + r8, k0 + (mi & 1) * 8));
-            else ldsm_x4_t(b, toff(B, k0 + (mi & 1) * 8 + r8, n0 + j * 8 + (mi >> 1) * 8));
-            hmma(c[j], a, b[0], b[1]);
-            hmma(c[j + 1], a, b[2], b[3]);
-        }
-    }
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_older() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
-// rows [0, rows) of a bf16 matrix with `cols` columns, global row stride `ld` elements;
-// rows >= valid are zero-filled.
-__device__ __forceinline__ void load_tile(const Tile &t, const __nv_bfloat16 *src, size_t ld, int rows, int cols,
-                                          int valid, int tid) {
-    const int cpr = cols / 8;
-    for (int e = tid; e < rows * cpr; e += kThreads) {
-        const int r = e / cpr, ch = e % cpr;
-        const bool ok = r < valid;
-        cp_async16(toff(t, r, ch * 8), src + (ok ? (size_t)r * ld + ch * 8 : 0), ok);
-    }
-}
-
-__device__ __forceinline__ float2 ld_pair(const Tile &t, int row, int col) {
-    uint32_t u;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(u) : "r"(toff(t, row, col)));
-    return unpack_bf16(u);
-}
 
 struct GradParams {
     Dims d;
@@ -142,16 +84,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
     // ---- loads (cp.async; rows past the chunk's end are zero). Two groups: the
     //      chunk tiles for phases A-C, then the two states, which land while A-C run.
     const size_t hbase = ((size_t)cg * d.Hv + h) * K * V;
-    load_tile(tQ, prm.q + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
-    load_tile(tK, prm.k + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
-    load_tile(tdO, prm.d_o + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
-    load_tile(tD, prm.delta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
-    load_tile(tdD, prm.ddelta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
-    load_tile(tA, prm.ainv + ((size_t)cg * d.Hv + h) * C * C, C, C, C, C, tid);
-    load_tile(tV, prm.v + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    load_tile<kThreads>(tQ, prm.q + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
+    load_tile<kThreads>(tK, prm.k + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
+    load_tile<kThreads>(tdO, prm.d_o + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    load_tile<kThreads>(tD, prm.delta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    load_tile<kThreads>(tdD, prm.ddelta + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
+    load_tile<kThreads>(tA, prm.ainv + ((size_t)cg * d.Hv + h) * C * C, C, C, C, C, tid);
+    load_tile<kThreads>(tV, prm.v + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
     cp_async_commit();
-    load_tile(th, prm.h_chunks + hbase, V, K, V, K, tid);
-    load_tile(tdh, prm.dh_chunks + hbase, V, K, V, K, tid);
+    load_tile<kThreads>(th, prm.h_chunks + hbase, V, K, V, K, tid);
+    load_tile<kThreads>(tdh, prm.dh_chunks + hbase, V, K, V, K, tid);
     cp_async_commit();
     if (tid < C) {
         const int r = tid, rr = min(r, len - 1);

@@ -1,46 +1,40 @@
-// gdn_fwd2.cu -- warp-specialised chunked forward (bf16, K = V = 128): the
-// state chain and the output on warp-level tensor-core MMAs, the bulk chunk
-// products on tcgen05.
+// gdn_fwd2.cu -- chunked forward of the gated delta rule (bf16, K = V = 128):
+// the sequential state chain on warp-level tensor-core MMAs, the output on
+// tcgen05. Everything that does not depend on the state (w, u and the
+// decay-masked P = M o Q K^T of every chunk) comes ready-made from the
+// chunk-prep kernel (gdn_prep3.cu) through a TMA ring.
 //
-// One CTA per (sequence, value head, 32-column slice of V). Per 64-token chunk
-// (notation of gdn_internal.cuh; Au = Ainv diag(beta), Aw = Ainv diag(beta e^gamma)
-// come ready-made from the chunk-prep kernel):
+// One CTA per (sequence or segment, value head, 32-column slice of V). Per
+// 64-token chunk (h the chunk-entry state, h = S^T, notation of gdn_internal.cuh):
 //
-//   tcgen05, TMEM accumulators:
-//     S = Q K^T,   W = Aw K,   U = Au V          (independent of h, one chunk ahead)
-//     DQ = Q h,    DP = P Delta                  (output, one chunk behind the chain)
-//     o = scale (e^gamma o DQ + DP),  P = causal decay mask o S
-//   mma.sync, fp32 state in registers (the chain):
-//     Delta = U + (-w) h,   h <- e^{gamma_C} h + K^T (e^{gamma_C - gamma} o Delta)
+//   chain (mma.sync, fp32 state in registers):
+//     Delta = u - w h,     h <- e^{gamma_C} h + K^T (e^{gamma_C - gamma} o Delta)
+//   output (tcgen05, TMEM accumulators, one chunk behind the chain):
+//     DQ = Q h,  DP = P Delta,   o = scale (e^gamma o DQ + DP)
 //
 // Why this split (measured on B200): a tcgen05 MMA takes ~450 cycles from
-// issue to a completed mbarrier, twice per chunk on the chain, whereas a
-// dependent mma.sync costs ~20 cycles, so the chain runs on mma.sync. The
-// output products stay on tcgen05 because there they read their operands once
-// from shared memory, whereas warp-level MMAs split across warps re-read them
-// and the shared-memory bandwidth (128 B/clk) is the next limit. The chain
-// publishes Delta_j and h_{j+1} together behind one generic-to-async proxy
-// fence per chunk.
+// issue to a completed mbarrier, and the chain has two dependent products per
+// chunk, whereas a dependent mma.sync costs ~20 cycles; the output products do
+// not feed the chain, so they run on tcgen05 off the critical path. Shared
+// memory bandwidth (128 B/clk/SM) is the next limit, which is why every
+// state-independent product is hoisted into the prep kernel.
 //
-// Warp roles (576 threads, two warps of each CUDA-core role per SM sub-partition):
+// Warp roles (416 threads):
 //   warps 0-7   chain: h (128 x 32 fp32) in mma fragments, warp w holding
 //               state rows 32 (w % 4) .. +31 and columns 16 (w / 4) .. +15.
-//   warps 8-15  aux: -w and u from TMEM into shared memory for the chain, P
-//               from S into shared memory, and o of the previous chunk from
-//               DQ/DP; warp 8 + w reads TMEM lanes 32 (w % 4) .. +31 and
-//               handles half (w / 4) of the columns.
-//   warp 16     MMA issuer A: TMA prologue, S/W/U MMAs.
-//   warp 17     MMA issuer B: DQ/DP MMAs, refills of the 3-deep TMA ring.
+//   warps 8-11  epilogue: o from the double-buffered DQ/DP accumulators;
+//               warp 8 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15).
+//   warp 12     issuer: 3-deep TMA ring (q, k, w, u, P per chunk) and the
+//               DQ/DP MMAs.
 // Roles hand over through monotonically increasing shared-memory counters
-// (release/acquire), which cannot alias the way mbarrier phase parities can
-// when a producer runs two phases ahead of a consumer. mbarriers are used only
-// where the hardware requires them: TMA completion (full[]) and tcgen05.commit
-// (mmaA[] for the aux warps, mmaO for issuer B), each with a single consumer
-// that its producer cannot lap. Every wait is
-// bounded in time; a wait that expires records GDN_ERR_TIMEOUT and winds the
-// CTA down.
-#include <cudaTypedefs.h>
-
+// (release/acquire), which cannot alias the way mbarrier parities can when a
+// producer runs ahead; mbarriers only where the hardware signals (TMA
+// completion, tcgen05.commit). Every wait is bounded in time; a wait that
+// expires records GDN_ERR_TIMEOUT and winds the CTA down.
+//
+// Modes: whole sequences from h0; the recompute for the backward (no output,
+// stores every chunk's entry state and Delta in bf16); and the two passes of
+// the sequence split (see Fwd2Mode).
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -53,56 +47,48 @@ namespace {
 using namespace sm100;
 using namespace warp;
 
-constexpr int kThreads = 576;  // 8 chain + 8 aux + 2 TMA/MMA warps
-constexpr int kRole = 256;     // threads per CUDA-core role
+constexpr int kThreads = 416;  // 8 chain + 4 epilogue + 1 issuer warps
+constexpr int kRole = 256;     // chain threads
+constexpr int kEpi = 128;      // epilogue threads
 constexpr int kBV = 32;
 constexpr int kStages = 3;
 
 // ---- shared memory (bytes from a 1024-aligned base)
 constexpr int kHb = 0;          // 2 x 8192   h (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16 (k = state row)
-constexpr int kDb = 16384;      // 3 x 4096   Delta (bf16), same layout with k = token
-constexpr int kDt = 28672;      // 4096       e^{gamma_C - gamma} Delta, chain only
-constexpr int kP = 32768;       // 8192       P, K-major SW128 (A of DP)
-constexpr int kWn = 40960;      // 16384      -w (bf16), row-major 256 B rows, 16-B chunks XOR (row % 8)
-constexpr int kU = 57344;       // 9216       u (fp32), row stride 36 floats
-constexpr int kStage0 = 66560;  // TMA ring
-constexpr int kQ = 0, kK = 16384, kAu = 32768, kAwS = 40960, kVt = 49152, kStageBytes = 53248;
-constexpr int kTxBytes = 16384 + 16384 + 8192 + 8192 + 4096;
+constexpr int kDb = 16384;      // 2 x 4096   Delta (bf16), same layout with k = token (B of DP)
+constexpr int kDt = 24576;      // 4096       e^{gamma_C - gamma} Delta, chain only
+constexpr int kStage0 = 28672;  // TMA ring
+// per stage: q [64][128] bf16 and k, w likewise (two 64-column halves, 128-byte
+// swizzle), u [64][32] fp32 (128-byte swizzle), P [64][64] bf16 (128-byte swizzle)
+constexpr int kQ = 0, kK = 16384, kW = 32768, kU = 49152, kP = 57344, kStageBytes = 65536;
+constexpr int kTxFull = 65536;                  // q, k, w, u, P
+constexpr int kTxChain = 16384 + 16384 + 8192;  // k, w, u (no output)
 constexpr int kSmall = kStage0 + kStages * kStageBytes;
-constexpr int kSmemBytes = kSmall + 2560 + 1024;
+constexpr int kSmemBytes = kSmall + 2048 + 1024;
 static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory layout");
 
-// S, W, U double-buffered in tensor memory (buffer b at column 224 b); DQ, DP single.
-constexpr uint32_t kColS = 0, kColW = 64, kColU = 192, kABuf = 224, kColQ = 448, kColP = 480, kTmemCols = 512;
+// DQ, DP double-buffered in tensor memory: buffer b at columns 64 b.
+constexpr uint32_t kColQ = 0, kColP = 32, kOBuf = 64, kTmemCols = 128;
 
-struct __align__(16) Gates {
-    float gam[64], egam[64];
-};
-
-// Hand-over counters: each holds the number of chunks (or states) its producer
-// has finished; consumers wait until it reaches the count they need.
-enum Ctr { kTmemA, kReady, kPReady, kWnFree, kDelta, kH, kStage, kODone, kTmemO, kNumCtr };
+// Hand-over counters (the number of chunks, or states, the producer has finished).
+enum Ctr { kH, kDelta, kStage, kODone, kTmemO, kNumCtr };
 
 struct Small {
     uint64_t full[kStages];
-    uint64_t mmaA[2], mmaO;
+    uint64_t mmaO[2];
     uint32_t ctr[kNumCtr];
-    int loads_issued, loads_landed;  // TMA chunk loads issued / observed complete
+    int loads_issued, loads_landed, mma_issued, mma_seen;
     uint32_t tmem_base;
     int abort_flag;
-    Gates gates[3];
 };
-static_assert(sizeof(Small) <= 2560, "small area");
-static_assert(kSmall % 16 == 0 && offsetof(Small, gates) % 16 == 0, "small area alignment");
+static_assert(sizeof(Small) <= 2048, "small area");
 
-template <int N = kRole>
-__device__ __forceinline__ bool role_sync_and(int id, bool pred) {
-    return warp::role_sync_and<N>(id, pred);
-}
+__device__ __forceinline__ bool chain_sync(bool pred) { return role_sync_and<kRole>(1, pred); }
+__device__ __forceinline__ bool epi_sync(bool pred) { return role_sync_and<kEpi>(2, pred); }
 
 // kWhole: one CTA column per sequence, from h0.
 // kSegPass: per segment, the chain on [c | P] with c from zero (V columns, u as
-//   input) and P from the identity (K more columns, whose v tile is read out of
+//   input) and P from the identity (K more columns, whose u tile is read out of
 //   range and so is zero): the segment maps a start state h to P h + c.
 // kSegOut: per segment, the chain and the output from the composed start state.
 enum Fwd2Mode { kWhole = 0, kSegPass = 1, kSegOut = 2 };
@@ -111,14 +97,14 @@ struct Fwd2Params {
     Dims d;
     const float *gamma;   // [T_total, Hv]
     const float *h0;      // [N, Hv, K, V] or null
-    __nv_bfloat16 *o;     // [T_total, Hv, V], or null: no output products (the backward's recompute)
+    __nv_bfloat16 *o;     // [T_total, Hv, V], or null: no output (the backward's recompute)
     float *final_state;   // [N, Hv, K, V] or null
     __nv_bfloat16 *h_chunks;  // [NC, Hv, K, V] entry state of every chunk (bf16, as the products read it) or null
     __nv_bfloat16 *delta;     // [T_total, Hv, V] Delta (bf16) or null
     // Sequence split: blockIdx.x = sequence * nseg + segment; a segment is a
     // contiguous run of ceil(chunks / nseg) chunks of its sequence.
     int nseg;
-    int mode;             // kWhole, kSegPass or kSegOut
+    int mode;             // Fwd2Mode
     const float *seg_h0;  // kSegOut: [N * nseg, Hv, K, V] start state of every segment
     float *seg_c;         // kSegPass: [N * nseg, Hv, K, V] end state from a zero start
     float *seg_P;         // kSegPass: [N * nseg, Hv, K, K] transition operator of the segment
@@ -127,8 +113,8 @@ struct Fwd2Params {
 
 __global__ void __launch_bounds__(kThreads, 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wy,
-            const Fwd2Params prm) {
+            const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
+            const __grid_constant__ CUtensorMap tm_p, const Fwd2Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -141,6 +127,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int K = 128, V = 128;
+    const bool want_o = prm.o != nullptr;
     // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
     const SeqRange seq = seq_range(d, n);
     const int nch_seq = (seq.len + kChunk - 1) / kChunk;
@@ -155,15 +142,14 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&sm->full[s], 1);
-        mbar_init(&sm->mmaA[0], 1);
-        mbar_init(&sm->mmaA[1], 1);
-        mbar_init(&sm->mmaO, 1);
+        mbar_init(&sm->mmaO[0], 1);
+        mbar_init(&sm->mmaO[1], 1);
         for (int c = 0; c < kNumCtr; ++c) sm->ctr[c] = 0;
-        sm->loads_issued = sm->loads_landed = 0;
+        sm->loads_issued = sm->loads_landed = sm->mma_issued = sm->mma_seen = 0;
         sm->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 16) {
+    if (warp == 12) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -173,20 +159,10 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = sm->tmem_base;
     uint32_t *ctr = sm->ctr;
 
-    auto issue_loads = [&](int ci) {
-        const int s = ci % kStages;
-        uint8_t *st = smem + kStage0 + s * kStageBytes;
-        const int t0 = sr.start + ci * kChunk;
-        const int cg = sr.chunk0 + ci;
-        mbar_arrive_expect_tx(&sm->full[s], kTxBytes);
-        atomicAdd(&sm->loads_issued, 1);
-        tma_load_3d(st + kQ, &tm_q, &sm->full[s], 0, hq, t0);
-        tma_load_3d(st + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
-        tma_load_3d(st + kK, &tm_k, &sm->full[s], 0, hq, t0);
-        tma_load_3d(st + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
-        tma_load_2d(st + kAu, &tm_wy, &sm->full[s], 0, ((cg * d.Hv + h) * 2) * kChunk);
-        tma_load_2d(st + kAwS, &tm_wy, &sm->full[s], 0, ((cg * d.Hv + h) * 2 + 1) * kChunk);
-        tma_load_3d(st + kVt, &tm_v, &sm->full[s], c0, h, t0);
+    // gamma of chunk j at in-chunk row r (rows past the end repeat the last live one)
+    auto gamma_at = [&](int j, int r) {
+        const int len = min(kChunk, sr.len - j * kChunk);
+        return prm.gamma[(size_t)(sr.start + j * kChunk + min(r, len - 1)) * d.Hv + h];
     };
 
     if (warp < 8) {
@@ -225,16 +201,20 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         };
         write_hb(0);
         fence_proxy_async();
-        bool ok = role_sync_and(1, true);
+        bool ok = chain_sync(true);
         if (tid == 0) publish(&ctr[kH], 1);  // h_0
+        // gates of the current chunk, prefetched one chunk ahead
+        float gl = 0.f, gt0 = 0.f, gt1 = 0.f;
+        if (nch > 0) gl = gamma_at(0, 63), gt0 = gamma_at(0, 16 * p + g), gt1 = gamma_at(0, 16 * p + g + 8);
 
         for (int j = 0; j < nch && ok; ++j) {
             const int len = min(kChunk, sr.len - j * kChunk);
-            ok = role_sync_and(1, wait_ge(&ctr[kReady], j + 1, abort_flag));
+            const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
+            ok = chain_sync(wait_bar(&sm->full[j % kStages], (j / kStages) & 1, abort_flag));
             if (!ok) break;
-            // gate scalars of chunk j (its slot is refilled only after this chunk's -w is consumed)
-            const Gates &G = sm->gates[j % 3];
-            const float gl = G.gam[63];
+            if (tid == 0) sm->loads_landed = j + 1;
+            const float gC = gl, gtok[2] = {gt0, gt1};
+            if (j + 1 < nch) gl = gamma_at(j + 1, 63), gt0 = gamma_at(j + 1, 16 * p + g), gt1 = gamma_at(j + 1, 16 * p + g + 8);
             if (prm.h_chunks) {  // entry state of chunk j, rounded as the products read it
                 __nv_bfloat16 *hc = prm.h_chunks + ((size_t)(sr.chunk0 + j) * d.Hv + h) * K * V + c0;
 #pragma unroll
@@ -248,25 +228,17 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                 pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
                     }
             }
-            const float gtok[2] = {G.gam[16 * p + g], G.gam[16 * p + g + 8]};
-            // ---- Delta = u + (-w) h : tokens 16p..16p+15, columns of n-tiles cb, cb+1
-            float acc[2][4];
+            // ---- w h : tokens 16p..16p+15, columns of n-tiles cb, cb+1 (A = w tile, B = h)
+            float acc[2][4] = {};
             {
-                const float *U = reinterpret_cast<const float *>(smem + kU);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int r0 = 16 * p + g, col = 8 * (cb + nt) + 2 * c4;
-                    const float2 a = *reinterpret_cast<const float2 *>(U + r0 * 36 + col);
-                    const float2 b = *reinterpret_cast<const float2 *>(U + (r0 + 8) * 36 + col);
-                    acc[nt][0] = a.x; acc[nt][1] = a.y; acc[nt][2] = b.x; acc[nt][3] = b.y;
-                }
+                const uint32_t wt = st + kW;
                 const uint32_t hb = sb + kHb + (j & 1) * 8192;
                 const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int mi = lane >> 3;  // (kg, nb): (2ks,cb) (2ks+1,cb) (2ks,cb+1) (2ks+1,cb+1)
+                const int mi = lane >> 3;
                 uint32_t a[2][4], b[2][4];
                 auto load = [&](int ks, int buf) {
-                    const int ch = 2 * ks + (lane >> 4);
-                    ldsm_x4(a[buf], sb + kWn + arow * 256 + ((ch ^ (arow & 7)) << 4));
+                    const int d0 = 16 * ks + (lane >> 4) * 8;
+                    ldsm_x4(a[buf], wt + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
                     ldsm_x4_t(b[buf], hb + (cb + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
                 };
                 load(0, 0);
@@ -277,41 +249,44 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     hmma(acc[1], a[ks & 1], b[ks & 1][2], b[ks & 1][3]);
                 }
             }
-            role_sync_and(1, true);
-            if (tid == 0) publish(&ctr[kWnFree], j + 1);
-            // ---- Delta -> Db[j%3] (read by the output) ; e^{gamma_C - gamma} Delta -> Dt
-            ok = role_sync_and(1, j < 3 || wait_ge(&ctr[kODone], j - 2, abort_flag));  // DP of j-3 read Db[j%3]
+            // ---- Delta = u - w h -> Db[j%2] (read by DP) ; e^{gamma_C - gamma} Delta -> Dt
+            ok = chain_sync(!want_o || j < 2 || wait_ge(&ctr[kODone], j - 1, abort_flag));  // DP of j-2 read Db[j%2]
             if (!ok) break;
             {
-                const uint32_t db = sb + kDb + (j % 3) * 4096 + c4 * 4, dt = sb + kDt + c4 * 4;
+                const uint32_t db = sb + kDb + (j & 1) * 4096 + c4 * 4, dt = sb + kDt + c4 * 4;
+                const float *ut = reinterpret_cast<const float *>(smem + kStage0 + (j % kStages) * kStageBytes + kU);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int tok = 16 * p + g + half * 8;
                     const bool live = tok < len;
-                    const float sc = __expf(gl - gtok[half]);
+                    const float sc = __expf(gC - gtok[half]);
                     const uint32_t off = (tok >> 3) * 128 + (tok & 7) * 16;
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        const float x0 = live ? acc[nt][2 * half] : 0.f, x1 = live ? acc[nt][2 * half + 1] : 0.f;
+                        const int col = 8 * (cb + nt) + 2 * c4;  // u tile: 32 fp32 per row, 16-B chunks XOR (row % 8)
+                        const float2 uu = *reinterpret_cast<const float2 *>(
+                            ut + tok * 32 + ((((col >> 2) ^ (tok & 7))) << 2) + (col & 3));
+                        const float x0 = live ? uu.x - acc[nt][2 * half] : 0.f;
+                        const float x1 = live ? uu.y - acc[nt][2 * half + 1] : 0.f;
                         st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(x0, x1));
                         st_shared_b32(dt + (cb + nt) * 1024 + off, pack_bf16(sc * x0, sc * x1));
                         if (prm.delta && live)
                             *reinterpret_cast<uint32_t *>(prm.delta + ((size_t)(sr.start + j * kChunk + tok) * d.Hv + h) * V +
-                                                          c0 + 8 * (cb + nt) + 2 * c4) = pack_bf16(x0, x1);
+                                                          c0 + col) = pack_bf16(x0, x1);
                     }
                 }
             }
-            role_sync_and(1, true);  // every warp reads all 64 tokens of Dt below
+            chain_sync(true);  // every warp reads all 64 tokens of Dt below
             // ---- h <- e^{gamma_C} h + K^T Dt : rows 32p..32p+31, 16 columns, K = 64 tokens
             {
-                const float eC = __expf(gl);
+                const float eC = __expf(gC);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) hf[mt][nt][q] *= eC;
-                const uint32_t kt = sb + kStage0 + (j % kStages) * kStageBytes + kK;
+                const uint32_t kt = st + kK;
                 const int mi = lane >> 3;
                 uint32_t b[2][4], a[2][2][4];
                 auto load = [&](int ks, int buf) {
@@ -336,15 +311,15 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
                 }
             }
-            role_sync_and(1, true);
+            chain_sync(true);
             if (tid == 0) publish(&ctr[kStage], j + 1);
             // ---- h_{j+1} -> Hb[(j+1)%2] once DQ of chunk j-1 (which read it) is done; then
             //      Delta_j and h_{j+1} go to the output MMAs behind one proxy fence
-            ok = role_sync_and(1, j < 1 || wait_ge(&ctr[kODone], j, abort_flag));
+            ok = chain_sync(!want_o || j < 1 || wait_ge(&ctr[kODone], j, abort_flag));
             if (!ok) break;
             write_hb((j + 1) & 1);
             fence_proxy_async();
-            role_sync_and(1, true);
+            chain_sync(true);
             if (tid == 0) {
                 publish(&ctr[kDelta], j + 1);
                 publish(&ctr[kH], j + 2);
@@ -377,220 +352,102 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         }
             }
         }
-    } else if (warp < 16) {
-        // ============================================================= aux
-        const int atid = tid - kRole, aw = warp - 8;
-        const int ap = aw & 3, ah = aw >> 2;  // TMEM sub-partition (rows 16ap..), output column half
-        const uint32_t lane_base = (uint32_t)(ap * 32) << 16;
-        const int ag = lane >> 2, ac = lane & 3;
-        const int ar0 = ap * 16 + ag, ar1 = ar0 + 8;  // rows of M=64 results this thread holds
-        bool ok = true;
-        const bool want_o = prm.o != nullptr;
-        auto output = [&](int jo) -> bool {  // o of chunk jo from DQ, DP (16 columns per warp)
-            if (!wait_ge(&ctr[kODone], jo + 1, abort_flag)) return false;
-            if (!want_o) return true;
-            tc_fence_after();
-            const Gates &G = sm->gates[jo % 3];
-            const int len = min(kChunk, sr.len - jo * kChunk);
-            const int t0 = sr.start + jo * kChunk;
-            float dq[8], dp[8];
-            tmem_ld16x256_x2(tmem + lane_base + kColQ + 16 * ah, dq);
-            tmem_ld16x256_x2(tmem + lane_base + kColP + 16 * ah, dp);
-            tc_fence_before();
+    } else if (warp < 12) {
+        // ======================================================== epilogue
+        if (want_o) {
+            const int et = tid - kRole, q = warp & 3;  // TMEM lanes 32q.. = rows 16q..16q+15
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            const int eg = lane >> 2, ec = lane & 3;
+            const int rr[2] = {16 * q + eg, 16 * q + eg + 8};
             const float scl = d.scale;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = half ? ar1 : ar0;
-                if (r < len) {
-                    const float er = G.egam[r];
-                    __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + r) * d.Hv + h) * V + c0 + 16 * ah + 2 * ac;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const int k = 4 * i + 2 * half;
-                        *reinterpret_cast<uint32_t *>(dst + 8 * i) =
-                            pack_bf16(scl * fmaf(er, dq[k], dp[k]), scl * fmaf(er, dq[k + 1], dp[k + 1]));
-                    }
-                }
-            }
-            return true;
-        };
-        float pg = 0.f;
-        auto fetch_gate = [&](int jj) {  // gamma of chunk jj, one value per thread < 64
-            if (atid < kChunk && jj < nch) {
-                const int t0 = sr.start + jj * kChunk, len = min(kChunk, sr.len - jj * kChunk);
-                pg = prm.gamma[(size_t)(t0 + min(atid, len - 1)) * d.Hv + h];
-            }
-        };
-        auto store_gate = [&](int jj) {
-            if (atid < kChunk) {
-                sm->gates[jj % 3].gam[atid] = pg;
-                sm->gates[jj % 3].egam[atid] = __expf(pg);
-            }
-        };
-        if (nch > 0) {
-            fetch_gate(0);
-            store_gate(0);
-            fetch_gate(1);
-        }
-        for (int j = 0; j < nch && ok; ++j) {
-            const int len = min(kChunk, sr.len - j * kChunk);
-            const uint32_t abuf = (j & 1) * kABuf;
-            // ---- S, W, U of chunk j have landed (the S/W/U MMAs also saw the stage land)
-            ok = role_sync_and(2, wait_bar(&sm->mmaA[j & 1], (j >> 1) & 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            if (atid == 0) sm->loads_landed = j + 1;
-            if (j + 1 < nch) {  // gates of chunk j+1 into their slot (chunk j-2 is fully done with it)
-                store_gate(j + 1);
-                fetch_gate(j + 2);
-            }
-            // ---- W, U -> -w and u for the chain, once it is done with chunk j-1's
-            ok = role_sync_and(2, wait_ge(&ctr[kWnFree], j, abort_flag));
-            if (!ok) break;
-            {
-                float v[32];
-                tmem_ld16x256_x8(tmem + lane_base + abuf + kColW + ah * 64, v);  // columns 64 ah .. +63 of -w
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int r = half ? ar1 : ar0;
-                    const uint32_t rowb = sb + kWn + r * 256 + 4 * ac;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int ch = 8 * ah + i;
-                        st_shared_b32(rowb + ((ch ^ (r & 7)) << 4), pack_bf16(-v[4 * i + 2 * half], -v[4 * i + 2 * half + 1]));
-                    }
-                }
-                float u[8];
-                tmem_ld16x256_x2(tmem + lane_base + abuf + kColU + 16 * ah, u);  // columns 16 ah .. +15 of u
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int r = half ? ar1 : ar0;
-                    const bool live = r < len;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        st_shared_v2f(sb + kU + (r * 36 + 16 * ah + 8 * i + 2 * ac) * 4, live ? u[4 * i + 2 * half] : 0.f,
-                                      live ? u[4 * i + 2 * half + 1] : 0.f);
-                }
-            }
-            role_sync_and(2, true);
-            if (atid == 0) publish(&ctr[kReady], j + 1);
-            // ---- P = causal decay mask o S -> SW128 tile for DP, once DP of chunk j-1 is done with it
-            ok = role_sync_and(2, j < 1 || wait_ge(&ctr[kODone], j, abort_flag));
-            if (!ok) break;
-            if (want_o) {
-                const Gates &G = sm->gates[j % 3];
-                float v[16];
-                tmem_ld16x256_x4(tmem + lane_base + abuf + kColS + 32 * ah, v);  // key columns 32 ah .. +31
-                const float gr0 = G.gam[ar0], gr1 = G.gam[ar1];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int s0 = 32 * ah + 8 * i + 2 * ac;
-                    const float2 gs = *reinterpret_cast<const float2 *>(&G.gam[s0]);
-                    const float x00 = s0 <= ar0 ? __expf(gr0 - gs.x) * v[4 * i] : 0.f;
-                    const float x01 = s0 + 1 <= ar0 ? __expf(gr0 - gs.y) * v[4 * i + 1] : 0.f;
-                    const float x10 = s0 <= ar1 ? __expf(gr1 - gs.x) * v[4 * i + 2] : 0.f;
-                    const float x11 = s0 + 1 <= ar1 ? __expf(gr1 - gs.y) * v[4 * i + 3] : 0.f;
-                    const int ch = 4 * ah + i;
-                    st_shared_b32(sb + kP + (ar0 >> 3) * 1024 + (ar0 & 7) * 128 + ((ch ^ (ar0 & 7)) << 4) + 4 * ac,
-                                  pack_bf16(x00, x01));
-                    st_shared_b32(sb + kP + (ar1 >> 3) * 1024 + (ar1 & 7) * 128 + ((ch ^ (ar1 & 7)) << 4) + 4 * ac,
-                                  pack_bf16(x10, x11));
-                }
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            role_sync_and(2, true);
-            if (atid == 0) {
-                publish(&ctr[kPReady], j + 1);
-                publish(&ctr[kTmemA], j + 1);
-            }
-            // ---- output of the previous chunk
-            if (j >= 1) {
-                ok = role_sync_and(2, output(j - 1));
-                if (!ok) break;
-                if (atid == 0) publish(&ctr[kTmemO], j);
-            }
-        }
-        if (ok && nch > 0) {
-            ok = role_sync_and(2, output(nch - 1));
-            if (ok && atid == 0) publish(&ctr[kTmemO], nch);
-        }
-        if (!ok) {
-            if (atid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
-            *abort_flag = 1;
-        }
-    } else if (warp == 16) {
-        // ==================================================== MMA issuer
-        if (lane == 0) {
             bool ok = true;
-            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
-            const uint32_t id_S = idesc_bf16(64, 64, false, false);
-            const uint32_t id_W = idesc_bf16(64, 128, false, true);
-            const uint32_t id_U = idesc_bf16(64, 32, false, true);
             for (int j = 0; j < nch && ok; ++j) {
-                const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
-                // stage landed; accumulator buffer j%2 was last read (by the aux warps) for chunk j-2
-                ok = wait_bar(&sm->full[j % kStages], (j / kStages) & 1, abort_flag) &&
-                     wait_ge(&ctr[kTmemA], j >= 1 ? j - 1 : 0, abort_flag);
+                const int len = min(kChunk, sr.len - j * kChunk);
+                const float g0 = gamma_at(j, rr[0]), g1 = gamma_at(j, rr[1]);
+                ok = epi_sync(wait_bar(&sm->mmaO[j & 1], (j >> 1) & 1, abort_flag));
                 if (!ok) break;
+                if (et == 0) {
+                    sm->mma_seen = j + 1;
+                    publish(&ctr[kODone], j + 1);
+                }
                 tc_fence_after();
-                const uint32_t tb = tmem + (j & 1) * kABuf;
-                for (int ks = 0; ks < 4; ++ks) {
-                    mma_bf16(tb + kColW, smem_desc(st + kAwS + ks * 32, 16, 1024, kSw128),
-                             smem_desc(st + kK + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
-                    mma_bf16(tb + kColU, smem_desc(st + kAu + ks * 32, 16, 1024, kSw128),
-                             smem_desc(st + kVt + ks * 1024, 4096, 512, kSw64), id_U, ks > 0);
+                float dq[16], dp[16];
+                const uint32_t tb = tmem + lane_base + (j & 1) * kOBuf;
+                tmem_ld16x256_x4(tb + kColQ, dq);
+                tmem_ld16x256_x4(tb + kColP, dp);
+                tc_fence_before();
+                epi_sync(true);
+                if (et == 0) publish(&ctr[kTmemO], j + 1);
+                const float er[2] = {__expf(g0), __expf(g1)};
+                const int t0 = sr.start + j * kChunk;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (rr[half] < len) {
+                        __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + rr[half]) * d.Hv + h) * V + c0 + 2 * ec;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int k = 4 * i + 2 * half;
+                            *reinterpret_cast<uint32_t *>(dst + 8 * i) =
+                                pack_bf16(scl * fmaf(er[half], dq[k], dp[k]), scl * fmaf(er[half], dq[k + 1], dp[k + 1]));
+                        }
+                    }
                 }
-                for (int ks = 0; ks < 8 && prm.o; ++ks) {
-                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16(tb + kColS, smem_desc(st + kQ + off, 16, 1024, kSw128),
-                             smem_desc(st + kK + off, 16, 1024, kSw128), id_S, ks > 0);
-                }
-                mma_commit(&sm->mmaA[j & 1]);
             }
             if (!ok) {
-                set_status(prm.status, GDN_ERR_TIMEOUT);
+                if (et == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
         }
-        __syncwarp();
     } else {
-        // ================================================== MMA issuer B
+        // ========================================================== issuer
         if (lane == 0) {
             bool ok = true;
+            auto issue_loads = [&](int j) {
+                const int s = j % kStages;
+                uint8_t *stg = smem + kStage0 + s * kStageBytes;
+                const int t0 = sr.start + j * kChunk;
+                const int cg = sr.chunk0 + j;
+                mbar_arrive_expect_tx(&sm->full[s], want_o ? kTxFull : kTxChain);
+                atomicAdd(&sm->loads_issued, 1);
+                if (want_o) {
+                    tma_load_3d(stg + kQ, &tm_q, &sm->full[s], 0, hq, t0);
+                    tma_load_3d(stg + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
+                    tma_load_2d(stg + kP, &tm_p, &sm->full[s], 0, (cg * d.Hv + h) * kChunk);
+                }
+                tma_load_3d(stg + kK, &tm_k, &sm->full[s], 0, hq, t0);
+                tma_load_3d(stg + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
+                tma_load_3d(stg + kW, &tm_w, &sm->full[s], 0, h, t0);
+                tma_load_3d(stg + kW + 8192, &tm_w, &sm->full[s], 64, h, t0);
+                tma_load_3d(stg + kU, &tm_u, &sm->full[s], c0, h, t0);  // out of range (zero) for operator columns
+            };
+            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
             const uint32_t id_O = idesc_bf16(64, 32, false, true);
-            int issued = min(kStages, nch);
             for (int j = 0; j < nch && ok; ++j) {
-                const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
+                // refill the stage of chunk j-1 with chunk j+2 once the chain and DQ/DP are done with it
+                if (j >= 1 && j + 2 < nch) {
+                    ok = wait_ge(&ctr[kStage], j, abort_flag) && (!want_o || wait_ge(&ctr[kODone], j, abort_flag));
+                    if (!ok) break;
+                    issue_loads(j + 2);
+                }
+                if (!want_o) continue;
+                // DQ = Q h_j, DP = P Delta_j into buffer j%2 once the epilogue has read chunk j-2's
                 ok = wait_ge(&ctr[kH], j + 1, abort_flag) && wait_ge(&ctr[kDelta], j + 1, abort_flag) &&
-                     wait_ge(&ctr[kPReady], j + 1, abort_flag) && wait_ge(&ctr[kTmemO], j, abort_flag);
+                     wait_ge(&ctr[kTmemO], j >= 1 ? j - 1 : 0, abort_flag);
                 if (!ok) break;
-                if (!prm.o) {  // recompute for the backward: no output products
-                    publish(&ctr[kODone], j + 1);
-                } else {
                 tc_fence_after();
-                const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j % 3) * 4096;
+                const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
+                const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
+                const uint32_t tb = tmem + (j & 1) * kOBuf;
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t aoff = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16(tmem + kColQ, smem_desc(st + kQ + aoff, 16, 1024, kSw128),
+                    mma_bf16(tb + kColQ, smem_desc(st + kQ + aoff, 16, 1024, kSw128),
                              smem_desc(hb + ks * 256, 128, 2048, kSwNone), id_O, ks > 0);
                 }
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + kColP, smem_desc(sb + kP + ks * 32, 16, 1024, kSw128),
+                    mma_bf16(tb + kColP, smem_desc(st + kP + ks * 32, 16, 1024, kSw128),
                              smem_desc(db + ks * 256, 128, 1024, kSwNone), id_O, ks > 0);
-                mma_commit(&sm->mmaO);
-                ok = wait_bar(&sm->mmaO, j & 1, abort_flag);
-                if (!ok) break;
-                tc_fence_before();
-                publish(&ctr[kODone], j + 1);
-                }
-                // refill the stage of chunk j with chunk j + 3 once the chain is done with its k tile
-                if (issued < nch) {
-                    ok = wait_ge(&ctr[kStage], j + 1, abort_flag);
-                    if (!ok) break;
-                    issue_loads(issued);
-                    ++issued;
-                }
+                mma_commit(&sm->mmaO[j & 1]);
+                sm->mma_issued = j + 1;
             }
             if (!ok) {
                 set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -606,21 +463,27 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // let every TMA load still in flight land (bounded) before the CTA exits
         const uint64_t t0 = globaltimer();
         for (int c = sm->loads_landed; c < sm->loads_issued; ++c)
-            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) &&
-                   globaltimer() - t0 < 2000000000ull) {
+            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
+            }
+        for (int c = sm->mma_seen; c < sm->mma_issued; ++c)  // and every output MMA
+            while (!mbar_try_wait(smem_u32(&sm->mmaO[c & 1]), (c >> 1) & 1) && globaltimer() - t0 < kWaitNs) {
             }
     }
     __syncthreads();
-    if (warp == 16) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-// ------------------------------------------------------------------ host side
-bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
-              const cuuint32_t *box, CUtensorMapSwizzle sw) {
-    return warp::make_bf16_map(m, base, rank, dims, strides, box, sw);
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank, const cuuint64_t *dims,
+              const cuuint64_t *strides, const cuuint32_t *box) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, rank, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -628,21 +491,24 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims
 cudaError_t launch_fwd2(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
-    if (!a.wy) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv, mw;
-    const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, (cuuint64_t)(d.T_total > 0 ? d.T_total : 1)};
+    if (!a.w16 || !a.u32 || (a.o && !a.p16)) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mw, mu, mp;
+    const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
+    const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
-    const cuuint32_t bq[3] = {64, 1, 64};
-    const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, (cuuint64_t)(d.T_total > 0 ? d.T_total : 1)};
-    const cuuint64_t sv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
-    const cuuint32_t bv[3] = {kBV, 1, 64};
-    const cuuint64_t dw[2] = {64, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * 2 * 64};
-    const cuuint64_t sw[1] = {128};
-    const cuuint32_t bw[2] = {64, 64};
-    if (!make_map(&mq, a.q, 3, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, a.k, 3, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, 3, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map(&mw, a.wy, 2, dw, sw, bw, CU_TENSOR_MAP_SWIZZLE_128B))
+    const cuuint32_t b64[3] = {64, 1, 64};
+    const cuuint64_t dw[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sw[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hv * d.K * 2};
+    const cuuint64_t du[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
+    const cuuint64_t su[2] = {(cuuint64_t)d.V * 4, (cuuint64_t)d.Hv * d.V * 4};
+    const cuuint32_t bu[3] = {kBV, 1, 64};
+    const cuuint64_t dp[2] = {64, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * 64};
+    const cuuint64_t sp[1] = {128};
+    const cuuint32_t bp[2] = {64, 64};
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (!make_map(&mq, BF, a.q, 3, dq, sq, b64) || !make_map(&mk, BF, a.k, 3, dq, sq, b64) ||
+        !make_map(&mw, BF, a.w16, 3, dw, sw, b64) || !make_map(&mu, F32, a.u32, 3, du, su, bu) ||
+        !make_map(&mp, BF, a.p16 ? a.p16 : a.w16, 2, dp, sp, bp))
         return cudaErrorInvalidValue;
     Fwd2Params p;
     p.d = d;
@@ -657,15 +523,14 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     p.seg_h0 = a.seg_h0;
     p.seg_c = a.seg_c;
     p.seg_P = a.seg_P;
-    if (p.mode != kWhole && (p.nseg < 1 || (p.mode == kSegOut && !p.seg_h0) ||
-                             (p.mode == kSegPass && (!p.seg_c || !p.seg_P || p.o))))
+    if (p.mode != kWhole && ((p.mode == kSegOut && !p.seg_h0) || (p.mode == kSegPass && (!p.seg_c || !p.seg_P || p.o))))
         return cudaErrorInvalidValue;
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(fwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
     dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
-    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, mw, p);
+    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, p);
     return cudaGetLastError();
 }
 

@@ -104,7 +104,11 @@ struct FwdArgs {
     float *gamma;    // [T_total, Hv] fp32
     void *ainv;      // [NC, Hv, 64, 64], fp32 (F32 problems) or bf16 (BF16 problems); may be null
                      // for the tensor-core forward when nothing is saved
-    void *wy;        // [NC, Hv, 2, 64, 64] bf16: Ainv diag(beta), Ainv diag(beta e^gamma) (tensor-core forward)
+    void *wy;        // [NC, Hv, 2, 64, 64] bf16: Ainv diag(beta), Ainv diag(beta e^gamma) (optional prep output)
+    // Chunk-prep outputs of the tensor-core path (bf16, K = V = 128):
+    void *w16;       // [T_total, Hv, K] bf16  w = Ainv diag(beta e^gamma) K
+    float *u32;      // [T_total, Hv, V] fp32  u = Ainv diag(beta) V
+    void *p16;       // [NC, Hv, 64, 64] bf16  P = M o Q K^T
     unsigned *status;
     cudaStream_t stream;
     // Per-chunk entry states and Delta for the backward's recompute (nullable).
@@ -143,12 +147,15 @@ bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
 cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_fwd2(const FwdArgs &a);
+// Chunk prep of the tensor-core path: gamma, Ainv (optional), w, u, P.
+bool prep3_supported(const FwdArgs &a);
+cudaError_t launch_prep3(const FwdArgs &a);
 // Sequence split: start state of every segment from h0 and the segments' (c, P).
 cudaError_t launch_split_compose(const FwdArgs &a);
 // Tensor-core backward (bf16, K = V = 128): reverse dh scan, per-chunk gradients,
 // and the GQA reduction of the dq / dk partials.
 bool tc_bwd_supported(const Dims &d, int dtype);
-cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *wy, void *dh_chunks16, void *ddelta16);
+cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16);
 cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const void *dh_chunks16,
                                const void *delta16, const void *ddelta16, float *dq_part, float *dk_part);
 cudaError_t launch_bwd_final(const BwdArgs &a, const float *dq_part, const float *dk_part);

@@ -132,6 +132,65 @@ __device__ __forceinline__ void hmma(float (&c)[4], const uint32_t (&a)[4], uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// bf16 tiles, row-major with 16-byte chunks XOR-permuted by (row % 8) so that
+// ldmatrix over 8 consecutive rows touches 8 distinct bank groups.
+struct Tile {
+    uint32_t base;
+    int pitch;  // bytes per row
+};
+__device__ __forceinline__ uint32_t toff(const Tile &t, int row, int col) {
+    return t.base + row * t.pitch + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2;
+}
+
+// C (16 x 8 NT) += A (16 x kdim) B (kdim x 8 NT) on one warp.
+// A_T: A stored [k][m] (read transposed); B_KN: B stored [k][n] (else [n][k]).
+template <int NT, bool A_T, bool B_KN>
+__device__ __forceinline__ void wgemm(float (&c)[NT][4], const Tile &A, const Tile &B, int m0, int n0, int kdim,
+                                      int lane) {
+    const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll 2
+    for (int k0 = 0; k0 < kdim; k0 += 16) {
+        uint32_t a[4];
+        if (!A_T) ldsm_x4(a, toff(A, m0 + r8 + (mi & 1) * 8, k0 + (mi >> 1) * 8));
+        else ldsm_x4_t(a, toff(A, k0 + (mi >> 1) * 8 + r8, m0 + (mi & 1) * 8));
+#pragma unroll
+        for (int j = 0; j < NT; j += 2) {
+            uint32_t b[4];
+            if (!B_KN) ldsm_x4(b, toff(B, n0 + j * 8 + (mi >> 1) * 8 + r8, k0 + (mi & 1) * 8));
+            else ldsm_x4_t(b, toff(B, k0 + (mi & 1) * 8 + r8, n0 + j * 8 + (mi >> 1) * 8));
+            hmma(c[j], a, b[0], b[1]);
+            hmma(c[j + 1], a, b[2], b[3]);
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_older() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// rows [0, rows) of a bf16 matrix with `cols` columns, global row stride `ld` elements;
+// rows >= valid are zero-filled.
+template <int kThreads>
+__device__ __forceinline__ void load_tile(const Tile &t, const __nv_bfloat16 *src, size_t ld, int rows, int cols,
+                                          int valid, int tid) {
+    const int cpr = cols / 8;
+    for (int e = tid; e < rows * cpr; e += kThreads) {
+        const int r = e / cpr, ch = e % cpr;
+        const bool ok = r < valid;
+        cp_async16(toff(t, r, ch * 8), src + (ok ? (size_t)r * ld + ch * 8 : 0), ok);
+    }
+}
+
+__device__ __forceinline__ float2 ld_pair(const Tile &t, int row, int col) {
+    uint32_t u;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(u) : "r"(toff(t, row, col)));
+    return unpack_bf16(u);
+}
+
 // ------------------------------------------------------------------ host side
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
