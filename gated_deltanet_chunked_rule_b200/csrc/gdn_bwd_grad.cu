@@ -29,7 +29,14 @@ namespace {
 
 using namespace warp;
 
-constexpr int kThreads = 256;  // 8 warps: warp w owns rows 16 (w % 4) .. +15, column half w / 4
+// 8 warps: warp w owns rows 16 (w % 4) .. +15 of every product and column
+// group w / 4 (32 columns of the 64 x 64 products, 64 of the 64 x 128 ones).
+// (More warps re-read the same operand fragments; the kernel is bound by
+// shared-memory load bandwidth, measured slower with 16.)
+constexpr int kThreads = 256;
+constexpr int kWN = 2;                       // column groups
+constexpr int NT_CC = 64 / (8 * kWN);        // n-tiles per warp, 64 x 64 products
+constexpr int NT_CK = 128 / (8 * kWN);       // n-tiles per warp, 64 x 128 products
 constexpr int C = 64, K = 128, V = 128;
 
 // ---- shared memory (bytes)
@@ -39,9 +46,9 @@ constexpr int kSmemBytes = kSvec + 4096;
 
 struct Vecs {
     float gam[64], egam[64], bet[64];
-    float rowdg[2][64], rowdb[2][64];  // per column-half partial row sums
-    float coldg[4][64];                // per row-quarter partial column sums
-    float scal[8];                     // per-warp partial of the chunk-level dgamma_C term
+    float rowdg[kWN][64], rowdb[kWN][64];  // per column-group partial row sums
+    float coldg[4][64];                    // per row-quarter partial column sums
+    float scal[kThreads / 32];             // per-warp partial of the chunk-level dgamma_C term
 };
 static_assert(sizeof(Vecs) <= 4096, "vector area");
 
@@ -110,20 +117,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
     const float er[2] = {vec.egam[r0], vec.egam[r1]};
     const float br[2] = {vec.bet[r0], vec.bet[r1]};
     const bool lr[2] = {r0 < len, r1 < len};
-    float rdg[2] = {0.f, 0.f}, rdb[2] = {0.f, 0.f}, cdg[8] = {}, sdg = 0.f;
+    float rdg[2] = {0.f, 0.f}, rdb[2] = {0.f, 0.f}, cdg[2 * NT_CC] = {}, sdg = 0.f;
+    const int cc0 = 8 * NT_CC * wn, ck0 = 8 * NT_CK * wn;  // this warp's first column (C x C, C x K)
 
-    // ---- phase A: S = Q K^T, G = K K^T, P1 = dO Delta^T (16 x 32 per warp)
-    float sacc[4][4] = {}, gacc[4][4] = {};
+    // ---- phase A: S = Q K^T, G = K K^T, P1 = dO Delta^T
+    float sacc[NT_CC][4] = {}, gacc[NT_CC][4] = {};
     {
-        float pacc[4][4] = {};
-        wgemm<4, false, false>(sacc, tQ, tK, 16 * wm, 32 * wn, K, lane);
-        wgemm<4, false, false>(gacc, tK, tK, 16 * wm, 32 * wn, K, lane);
-        wgemm<4, false, false>(pacc, tdO, tD, 16 * wm, 32 * wn, V, lane);
+        float pacc[NT_CC][4] = {};
+        wgemm<NT_CC, false, false>(sacc, tQ, tK, 16 * wm, cc0, K, lane);
+        wgemm<NT_CC, false, false>(gacc, tK, tK, 16 * wm, cc0, K, lane);
+        wgemm<NT_CC, false, false>(pacc, tdO, tD, 16 * wm, cc0, V, lane);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NT_CC; ++j)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int hi = q >> 1, s = 32 * wn + 8 * j + 2 * c4 + (q & 1), r = hi ? r1 : r0;
+                const int hi = q >> 1, s = cc0 + 8 * j + 2 * c4 + (q & 1), r = hi ? r1 : r0;
                 const bool on = lr[hi] && s <= r;  // s < len follows
                 const float E = on ? __expf(gr[hi] - vec.gam[s]) : 0.f;
                 const float t1 = scale * E * pacc[j][q];
@@ -135,20 +143,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
             }
         // T1 -> shared memory (bf16)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int s = 32 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CC; ++j) {
+            const int s = cc0 + 8 * j + 2 * c4;
             st_shared_b32(toff(tT1, r0, s), pack_bf16(pacc[j][0], pacc[j][1]));
             st_shared_b32(toff(tT1, r1, s), pack_bf16(pacc[j][2], pacc[j][3]));
         }
     }
 
-    // ---- phase B: dU = Ainv^T dDelta (16 x 64 per warp); dv, dbeta (dU.v); dU -> (V's space)
+    // ---- phase B: dU = Ainv^T dDelta; dv, dbeta (dU.v); dU -> (V's space)
     {
-        float uacc[8][4] = {};
-        wgemm<8, true, true>(uacc, tA, tdD, 16 * wm, 64 * wn, C, lane);
+        float uacc[NT_CK][4] = {};
+        wgemm<NT_CK, true, true>(uacc, tA, tdD, 16 * wm, ck0, C, lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi) {
                 const int r = hi ? r1 : r0;
@@ -161,8 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
         }
         __syncthreads();  // every warp is done reading v
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
             st_shared_b32(toff(tV, r0, col), pack_bf16(uacc[j][0], uacc[j][1]));
             st_shared_b32(toff(tV, r1, col), pack_bf16(uacc[j][2], uacc[j][3]));
         }
@@ -172,10 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
 
     // ---- phase C: dAkk = -dU Delta^T (s < r); dbeta, Zr, dG
     {
-        float aacc[4][4] = {};
-        wgemm<4, false, false>(aacc, tU, tD, 16 * wm, 32 * wn, V, lane);
+        float aacc[NT_CC][4] = {};
+        wgemm<NT_CC, false, false>(aacc, tU, tD, 16 * wm, cc0, V, lane);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < NT_CC; ++j) {
             float dgv[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
                 cdg[2 * j + (q & 1)] -= zr;
                 dgv[q] = dA * br[hi] * E;
             }
-            const int s = 32 * wn + 8 * j + 2 * c4;
+            const int s = cc0 + 8 * j + 2 * c4;
             st_shared_b32(toff(tdG, r0, s), pack_bf16(dgv[0], dgv[1]));
             st_shared_b32(toff(tdG, r1, s), pack_bf16(dgv[2], dgv[3]));
         }
@@ -197,13 +205,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
     cp_async_wait_all();  // the two states
     __syncthreads();      // dG and the states visible
 
-    // ---- phase D: dq = scale diag(e^gamma) dO h^T + T1 K  (16 x 64 per warp)
+    // ---- phase D: dq = scale diag(e^gamma) dO h^T + T1 K
     {
-        float acc[8][4] = {};
-        wgemm<8, false, false>(acc, tdO, th, 16 * wm, 64 * wn, V, lane);
+        float acc[NT_CK][4] = {};
+        wgemm<NT_CK, false, false>(acc, tdO, th, 16 * wm, ck0, V, lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi) {
                 const float2 qq = ld_pair(tQ, hi ? r1 : r0, col);
@@ -213,10 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
                 acc[j][2 * hi + 1] *= f;
             }
         }
-        wgemm<8, false, true>(acc, tT1, tK, 16 * wm, 64 * wn, C, lane);
+        wgemm<NT_CK, false, true>(acc, tT1, tK, 16 * wm, ck0, C, lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi)
                 if (lr[hi])
@@ -227,12 +235,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
 
     // ---- phase E: dk
     {
-        float kacc[8][4], tacc[8][4] = {};
+        float kacc[NT_CK][4], tacc[NT_CK][4] = {};
         // -dU h^T = dKb: dk += beta e^gamma dKb; dbeta += e^gamma dKb.k; dgamma += beta e^gamma dKb.k
-        wgemm<8, false, false>(tacc, tU, th, 16 * wm, 64 * wn, V, lane);
+        wgemm<NT_CK, false, false>(tacc, tU, th, 16 * wm, ck0, V, lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi) {
                 const float2 kk = ld_pair(tK, hi ? r1 : r0, col);
@@ -247,15 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
             }
         }
         // Delta dh'^T: dk += e^{gamma_C - gamma} (.); Z3
-        wgemm<8, false, false>(tacc, tD, tdh, 16 * wm, 64 * wn, V, lane);
+        wgemm<NT_CK, false, false>(tacc, tD, tdh, 16 * wm, ck0, V, lane);
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
             const int r = hi ? r1 : r0;
             const float f = lr[hi] ? __expf(gC - gr[hi]) : 0.f;
             float z3 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int col = 64 * wn + 8 * j + 2 * c4;
+            for (int j = 0; j < NT_CK; ++j) {
+                const int col = ck0 + 8 * j + 2 * c4;
                 const float2 kk = ld_pair(tK, r, col);
                 z3 += tacc[j][2 * hi] * kk.x + tacc[j][2 * hi + 1] * kk.y;
                 kacc[j][2 * hi] += f * tacc[j][2 * hi];
@@ -265,12 +273,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
             rdg[hi] -= z3;
             sdg += z3;
         }
-        wgemm<8, true, true>(kacc, tT1, tQ, 16 * wm, 64 * wn, C, lane);   // T1^T Q
-        wgemm<8, false, true>(kacc, tdG, tK, 16 * wm, 64 * wn, C, lane);  // dG K
-        wgemm<8, true, true>(kacc, tdG, tK, 16 * wm, 64 * wn, C, lane);   // dG^T K
+        wgemm<NT_CK, true, true>(kacc, tT1, tQ, 16 * wm, ck0, C, lane);   // T1^T Q
+        wgemm<NT_CK, false, true>(kacc, tdG, tK, 16 * wm, ck0, C, lane);  // dG K
+        wgemm<NT_CK, true, true>(kacc, tdG, tK, 16 * wm, ck0, C, lane);   // dG^T K
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int j = 0; j < NT_CK; ++j) {
+            const int col = ck0 + 8 * j + 2 * c4;
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi)
                 if (lr[hi])
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
         rdb[hi] += __shfl_xor_sync(0xffffffffu, rdb[hi], 2);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 2 * NT_CC; ++i) {
         cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 4);
         cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 8);
         cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 16);
@@ -318,9 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
     }
     if (g == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            vec.coldg[wm][32 * wn + 8 * j + 2 * c4] = cdg[2 * j];
-            vec.coldg[wm][32 * wn + 8 * j + 2 * c4 + 1] = cdg[2 * j + 1];
+        for (int j = 0; j < NT_CC; ++j) {
+            vec.coldg[wm][cc0 + 8 * j + 2 * c4] = cdg[2 * j];
+            vec.coldg[wm][cc0 + 8 * j + 2 * c4 + 1] = cdg[2 * j + 1];
         }
     }
     if (lane == 0) vec.scal[warp] = sdg;
@@ -331,14 +339,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const GradParams 
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
             const int r = lane + 32 * hi;
-            float a = vec.rowdg[0][r] + vec.rowdg[1][r];
+            float a = 0.f, b = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWN; ++w) a += vec.rowdg[w][r], b += vec.rowdb[w][r];
             a += ((vec.coldg[0][r] + vec.coldg[1][r]) + vec.coldg[2][r]) + vec.coldg[3][r];
             dgr[hi] = r < len ? a : 0.f;
-            dbr[hi] = vec.rowdb[0][r] + vec.rowdb[1][r];
+            dbr[hi] = b;
         }
         float tot = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) tot += vec.scal[w];
+        for (int w = 0; w < kThreads / 32; ++w) tot += vec.scal[w];
         // the chunk-level term belongs to the last live token
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi)

@@ -231,23 +231,47 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             // ---- w h : tokens 16p..16p+15, columns of n-tiles cb, cb+1 (A = w tile, B = h)
             float acc[2][4] = {};
             {
+                // all of this warp's w fragments up front (they do not depend on h),
+                // the h fragments streamed three k-steps ahead
                 const uint32_t wt = st + kW;
                 const uint32_t hb = sb + kHb + (j & 1) * 8192;
                 const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int mi = lane >> 3;
-                uint32_t a[2][4], b[2][4];
-                auto load = [&](int ks, int buf) {
-                    const int d0 = 16 * ks + (lane >> 4) * 8;
-                    ldsm_x4(a[buf], wt + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
-                    ldsm_x4_t(b[buf], hb + (cb + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
-                };
-                load(0, 0);
+                uint32_t a[8][4], b[4][4];
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    if (ks + 1 < 8) load(ks + 1, (ks + 1) & 1);
-                    hmma(acc[0], a[ks & 1], b[ks & 1][0], b[ks & 1][1]);
-                    hmma(acc[1], a[ks & 1], b[ks & 1][2], b[ks & 1][3]);
+                    const int d0 = 16 * ks + (lane >> 4) * 8;
+                    ldsm_x4(a[ks], wt + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
                 }
+                auto load_b = [&](int ks) {
+                    ldsm_x4_t(b[ks & 3], hb + (cb + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
+                };
+                load_b(0);
+                load_b(1);
+                load_b(2);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    if (ks + 3 < 8) load_b(ks + 3);
+                    hmma(acc[0], a[ks], b[ks & 3][0], b[ks & 3][1]);
+                    hmma(acc[1], a[ks], b[ks & 3][2], b[ks & 3][3]);
+                }
+            }
+            // K^T fragments of the state update (independent of the chain): issued now so that
+            // their latency overlaps the Delta step. A = K^T rows (state rows) 32p+16mt..,
+            // cols (tokens) 16ks..: 8x8 blocks of the token-major, 128-byte-swizzled k tile
+            // read transposed.
+            uint32_t ka[4][2][4];
+            {
+                const uint32_t kt = st + kK;
+                const int mi = lane >> 3;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
+                        const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
+                        ldsm_x4_t(ka[ks][mt], kt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
+                    }
             }
             // ---- Delta = u - w h -> Db[j%2] (read by DP) ; e^{gamma_C - gamma} Delta -> Dt
             ok = chain_sync(!want_o || j < 2 || wait_ge(&ctr[kODone], j - 1, abort_flag));  // DP of j-2 read Db[j%2]
@@ -286,30 +310,18 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) hf[mt][nt][q] *= eC;
-                const uint32_t kt = st + kK;
                 const int mi = lane >> 3;
-                uint32_t b[2][4], a[2][2][4];
-                auto load = [&](int ks, int buf) {
-                    ldsm_x4_t(b[buf], sb + kDt + (cb + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
+                uint32_t b[4][4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    ldsm_x4_t(b[ks], sb + kDt + (cb + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
                     for (int mt = 0; mt < 2; ++mt) {
-                        // A = K^T rows (state rows) 32p+16mt.., cols (tokens) 16ks..: 8x8
-                        // blocks of the token-major, 128-byte-swizzled k tile read transposed
-                        const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
-                        const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
-                        ldsm_x4_t(a[buf][mt], kt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
+                        hmma(hf[mt][0], ka[ks][mt], b[ks][0], b[ks][1]);
+                        hmma(hf[mt][1], ka[ks][mt], b[ks][2], b[ks][3]);
                     }
-                };
-                load(0, 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    if (ks + 1 < 4) load(ks + 1, (ks + 1) & 1);
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        hmma(hf[mt][0], a[ks & 1][mt], b[ks & 1][0], b[ks & 1][1]);
-                        hmma(hf[mt][1], a[ks & 1][mt], b[ks & 1][2], b[ks & 1][3]);
-                    }
-                }
             }
             chain_sync(true);
             if (tid == 0) publish(&ctr[kStage], j + 1);
