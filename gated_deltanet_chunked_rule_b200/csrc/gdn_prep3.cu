@@ -14,33 +14,46 @@
 //   Ainv  (bf16 [NC, Hv, 64, 64], for the backward; optional)
 //
 // (the WY form of the chunk: Delta = u - w h, o = scale (diag(e^gamma) Q h + P Delta).)
-// Products on warp-level bf16 MMAs from swizzled shared-memory tiles; the unit
-// lower-triangular inverse block-wise on 16 x 16 blocks: diagonal blocks by
-// forward substitution, off-diagonal blocks one block diagonal at a time on
-// tf32 MMAs. Rows past the end of a sequence have k = q = v = 0 and beta = 0,
-// so their rows of A vanish and the inverse is the identity there.
+// The four bulk products (S, G, u, w) run on tcgen05 from TMA-loaded,
+// 128-byte-swizzled tiles, so their operands never pass through the
+// load/store unit, which the warp-level version of this kernel saturated.
+// The unit lower-triangular inverse is taken block-wise on 16 x 16 blocks in
+// fp32: diagonal blocks by forward substitution, off-diagonal blocks one block
+// diagonal at a time on tf32 MMAs. Rows past the end of a sequence have
+// beta = 0, so their rows of A vanish, the inverse is the identity there and
+// their columns of Ainv diag(beta) are zero: whatever the TMA reads past the
+// end (the next sequence, or zeros) never reaches an output.
+#include <cstddef>
+
 #include "gdn_internal.cuh"
 #include "gdn_warp.cuh"
+#include "sm100_ptx.cuh"
 
 namespace gdn {
 namespace {
 
+using namespace sm100;
 using namespace warp;
 
 constexpr int kThreads = 256;
 constexpr int C = 64, K = 128, V = 128;
+constexpr int kLd = 68;  // row pitch (floats) of the fp32 work matrices
 
-// ---- shared memory (bytes)
-constexpr int kSK = 0;          // k tile [64][128] bf16
-constexpr int kSQV = 16384;     // q tile, then the current value head's v tile
-constexpr int kSA = 32768;      // float [64][65]
-constexpr int kSX = kSA + 16640;
-constexpr int kST = kSX + 16640;
-constexpr int kSAw = kST + 16640;  // bf16 [64][64] Ainv diag(beta e^gamma)
-constexpr int kSAu = kSAw + 8192;  // bf16 [64][64] Ainv diag(beta)
-constexpr int kSvec = kSAu + 8192;
-constexpr int kSmemBytes = kSvec + 1024;
-static_assert(kSAw % 16 == 0 && kSmemBytes <= 113 * 1024, "two CTAs per SM");
+// ---- shared memory (bytes from a 1024-aligned base)
+constexpr int kQV = 0;          // q tile, then the current value head's v tile: [64][128] bf16, 128-byte swizzle, two halves
+constexpr int kKt = 16384;      // k tile, same layout
+constexpr int kAu = 32768;      // Ainv diag(beta): [64][64] bf16, 128-byte swizzle (K-major A operand)
+constexpr int kAw = 40960;      // Ainv diag(beta e^gamma)
+constexpr int kA = 49152;       // float [64][kLd]
+constexpr int kX = kA + 64 * kLd * 4;
+constexpr int kT = kX + 64 * kLd * 4;      // float [3][16][17]: one 16 x 16 block product per warp
+constexpr int kVec = kT + 3 * 16 * 17 * 4;
+constexpr int kBar = kVec + 1024;
+constexpr int kSmemBytes = kBar + 64 + 1024;
+static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+
+// tensor memory: S | G (64 columns each), later u | w (128 columns each)
+constexpr uint32_t kColS = 0, kColG = 64, kColU = 0, kColW = 128, kTmemCols = 256;
 
 __device__ __forceinline__ uint32_t tf32(float x) {
     uint32_t r;
@@ -55,24 +68,36 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Bounded wait on an mbarrier phase by every thread of the CTA.
+__device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer() - t0 > kWaitNs) return false;
+    return true;
+}
+
 struct Prep3Params {
     Dims d;
-    const __nv_bfloat16 *q, *k, *v;
     const float *g, *beta;
     float *gamma_out;
     __nv_bfloat16 *ainv_out;  // nullable
     __nv_bfloat16 *w_out;
     float *u_out;
     __nv_bfloat16 *p_out;
+    unsigned *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params prm) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kThreads, 2)
+prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_v, const Prep3Params prm) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
     const Dims &d = prm.d;
     const int cg = blockIdx.x, hq = blockIdx.y;
     const int n = chunk_owner(d, cg);
-    if (n < 0) return;
+    if (n < 0) return;  // whole CTA, before any allocation
     const SeqRange sr = seq_range(d, n);
     const int ci = cg - sr.chunk0;
     const int t0 = sr.start + ci * C, len = min(C, sr.len - ci * C);
@@ -81,35 +106,88 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
     const int r0 = 16 * wm + g8, r1 = r0 + 8;
     const int G = d.Hv / d.Hq;
 
-    float(*A)[65] = reinterpret_cast<float(*)[65]>(smem + kSA);
-    float(*X)[65] = reinterpret_cast<float(*)[65]>(smem + kSX);
-    float(*T)[65] = reinterpret_cast<float(*)[65]>(smem + kST);
-    float *gam = reinterpret_cast<float *>(smem + kSvec);
+    float(*A)[kLd] = reinterpret_cast<float(*)[kLd]>(smem + kA);
+    float(*X)[kLd] = reinterpret_cast<float(*)[kLd]>(smem + kX);
+    float(*T)[16][17] = reinterpret_cast<float(*)[16][17]>(smem + kT);
+    float *gam = reinterpret_cast<float *>(smem + kVec);
     float *egam = gam + 64, *bet = gam + 128, *scan = gam + 192;
-    const Tile tK{sb + kSK, 256}, tQV{sb + kSQV, 256}, tAw{sb + kSAw, 128}, tAu{sb + kSAu, 128};
+    uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + kBar);
+    uint64_t *mma_bar = tma_bar + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
 
-    // ---- k, q tiles; g, beta of the first value head (prefetched one head ahead)
-    load_tile<kThreads>(tK, prm.k + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
-    load_tile<kThreads>(tQV, prm.q + ((size_t)t0 * d.Hq + hq) * K, (size_t)d.Hq * K, C, K, len, tid);
-    cp_async_commit();
-    float g_next = 0.f, b_next = 0.f;
+    if (tid == 0) {
+        mbar_init(tma_bar, 1);
+        mbar_init(mma_bar, 1);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)(wm * 32) << 16;  // TMEM lanes of this warp's rows (M = 64 layout)
+    uint32_t tma_phase = 0, mma_phase = 0;  // phases consumed so far
+    bool tma_pending = false, mma_pending = false;  // (thread 0) issued and not yet consumed
+    bool ok = true;
+
+    // ---- q, k tiles by TMA; S = Q K^T and G = K K^T on tcgen05
+    if (tid == 0) {
+        mbar_arrive_expect_tx(tma_bar, 4 * 8192);
+        tma_load_3d(smem + kQV, &tm_q, tma_bar, 0, hq, t0);
+        tma_load_3d(smem + kQV + 8192, &tm_q, tma_bar, 64, hq, t0);
+        tma_load_3d(smem + kKt, &tm_k, tma_bar, 0, hq, t0);
+        tma_load_3d(smem + kKt + 8192, &tm_k, tma_bar, 64, hq, t0);
+        tma_pending = true;
+    }
+    float g_next = 0.f, b_next = 0.f;  // g, beta of the next value head, prefetched
     if (tid < C && tid < len) {
         g_next = prm.g[(size_t)(t0 + tid) * d.Hv + hq * G];
         b_next = prm.beta[(size_t)(t0 + tid) * d.Hv + hq * G];
     }
-    cp_async_wait_all();
-    __syncthreads();
+    ok = cta_wait(tma_bar, tma_phase & 1);
+    if (ok) ++tma_phase, tma_pending = false;
+    if (ok && tid == 0) {
+        tc_fence_after();
+        const uint32_t id_S = idesc_bf16(64, 64, false, false);
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+            mma_bf16(tmem + kColS, smem_desc(sb + kQV + off, 16, 1024, kSw128), smem_desc(sb + kKt + off, 16, 1024, kSw128),
+                     id_S, ks > 0);
+            mma_bf16(tmem + kColG, smem_desc(sb + kKt + off, 16, 1024, kSw128), smem_desc(sb + kKt + off, 16, 1024, kSw128),
+                     id_S, ks > 0);
+        }
+        mma_commit(mma_bar);
+        mma_pending = true;
+    }
+    ok = ok && cta_wait(mma_bar, mma_phase & 1);
+    if (ok) ++mma_phase, mma_pending = false;
+    tc_fence_after();
+    // S, G: rows r0, r1, columns 32 wn + 8 j + 2 c4 (+1) -- the warp MMA fragment layout
+    float sacc[4][4], gacc[4][4];
+    {
+        float v[16];
+        tmem_ld16x256_x4(tmem + lane_base + kColS + 32 * wn, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sacc[i >> 2][i & 3] = v[i];
+        tmem_ld16x256_x4(tmem + lane_base + kColG + 32 * wn, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) gacc[i >> 2][i & 3] = v[i];
+    }
+    tc_fence_before();
+    __syncthreads();  // q tile and S, G columns free
+    auto load_v = [&](int h) {
+        mbar_arrive_expect_tx(tma_bar, 2 * 8192);
+        tma_load_3d(smem + kQV, &tm_v, tma_bar, 0, h, t0);
+        tma_load_3d(smem + kQV + 8192, &tm_v, tma_bar, 64, h, t0);
+        tma_pending = true;
+    };
+    if (ok && tid == 0) load_v(hq * G);
 
-    // ---- S = Q K^T, G = K K^T: 16 x 32 per warp, kept in registers for every value head
-    float sacc[4][4] = {}, gacc[4][4] = {};
-    wgemm<4, false, false>(sacc, tQV, tK, 16 * wm, 32 * wn, K, lane);
-    wgemm<4, false, false>(gacc, tK, tK, 16 * wm, 32 * wn, K, lane);
-    __syncthreads();  // q tile no longer read: its space takes v
-
-    for (int gi = 0; gi < G; ++gi) {
+    for (int gi = 0; gi < G && ok; ++gi) {
         const int h = hq * G + gi;
-        load_tile<kThreads>(tQV, prm.v + ((size_t)t0 * d.Hv + h) * V, (size_t)d.Hv * V, C, V, len, tid);
-        cp_async_commit();
         // ---- gamma: two warps scan 32 rows each, then combine
         if (tid < C) {
             float x = g_next;
@@ -148,10 +226,9 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
                     const int r = hi ? r1 : r0;
                     const float e0 = s <= r ? __expf(gr[hi] - gs0) : 0.f;
                     const float e1 = s + 1 <= r ? __expf(gr[hi] - gs1) : 0.f;
-                    A[r][s] = s < r ? br[hi] * e0 * gacc[j][2 * hi] : 0.f;
-                    A[r][s + 1] = s + 1 < r ? br[hi] * e1 * gacc[j][2 * hi + 1] : 0.f;
-                    X[r][s] = 0.f;
-                    X[r][s + 1] = 0.f;
+                    *reinterpret_cast<float2 *>(&A[r][s]) =
+                        make_float2(s < r ? br[hi] * e0 * gacc[j][2 * hi] : 0.f, s + 1 < r ? br[hi] * e1 * gacc[j][2 * hi + 1] : 0.f);
+                    *reinterpret_cast<float2 *>(&X[r][s]) = make_float2(0.f, 0.f);
                     const bool live = r < len;
                     *reinterpret_cast<uint32_t *>(pout + r * C + s) =
                         pack_bf16(live ? e0 * sacc[j][2 * hi] : 0.f, live ? e1 * sacc[j][2 * hi + 1] : 0.f);
@@ -193,13 +270,14 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
                         }
                     }
                 }
+                float(*Tw)[17] = T[warp];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    const int col = j * 16 + nt * 8 + 2 * c4;
-                    T[i * 16 + g8][col] = t[nt][0];
-                    T[i * 16 + g8][col + 1] = t[nt][1];
-                    T[i * 16 + g8 + 8][col] = t[nt][2];
-                    T[i * 16 + g8 + 8][col + 1] = t[nt][3];
+                    const int col = nt * 8 + 2 * c4;
+                    Tw[g8][col] = t[nt][0];
+                    Tw[g8][col + 1] = t[nt][1];
+                    Tw[g8 + 8][col] = t[nt][2];
+                    Tw[g8 + 8][col + 1] = t[nt][3];
                 }
                 __syncwarp();
                 float x[2][4] = {};
@@ -210,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
                                            tf32(X[i * 16 + g8][ac + 4]), tf32(X[i * 16 + g8 + 8][ac + 4])};
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        const int bc = j * 16 + nt * 8 + g8;
-                        mma_tf32(x[nt], a, tf32(T[i * 16 + kk * 8 + c4][bc]), tf32(T[i * 16 + kk * 8 + c4 + 4][bc]));
+                        const int bc = nt * 8 + g8;
+                        mma_tf32(x[nt], a, tf32(Tw[kk * 8 + c4][bc]), tf32(Tw[kk * 8 + c4 + 4][bc]));
                     }
                 }
 #pragma unroll
@@ -225,49 +303,85 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
             }
             __syncthreads();
         }
-        // ---- Ainv diag(beta), Ainv diag(beta e^gamma) -> bf16 tiles; Ainv -> global (optional)
+        // ---- Ainv diag(beta), Ainv diag(beta e^gamma) -> 128-byte-swizzled bf16 tiles
+        //      (the K-major A operands of the u and w products); Ainv -> global (optional)
         for (int e = tid; e < C * C / 2; e += kThreads) {
             const int r = e >> 5, s = (e & 31) * 2;
             const float x0 = X[r][s], x1 = X[r][s + 1];
             const float u0 = x0 * bet[s], u1 = x1 * bet[s + 1];
-            st_shared_b32(toff(tAu, r, s), pack_bf16(u0, u1));
-            st_shared_b32(toff(tAw, r, s), pack_bf16(u0 * egam[s], u1 * egam[s + 1]));
+            const uint32_t off = (r >> 3) * 1024 + (r & 7) * 128 + ((((s >> 3) ^ (r & 7))) << 4) + (s & 7) * 2;
+            st_shared_b32(sb + kAu + off, pack_bf16(u0, u1));
+            st_shared_b32(sb + kAw + off, pack_bf16(u0 * egam[s], u1 * egam[s + 1]));
             if (prm.ainv_out)
                 *reinterpret_cast<uint32_t *>(prm.ainv_out + ((size_t)cg * d.Hv + h) * C * C + r * C + s) =
                     pack_bf16(x0, x1);
         }
-        cp_async_wait_all();  // this head's v tile
+        fence_proxy_async();
         __syncthreads();
-        // ---- u = Au V (fp32), w = Aw K (bf16): 16 x 64 per warp
-        {
-            float acc[8][4] = {};
-            wgemm<8, false, true>(acc, tAu, tQV, 16 * wm, 64 * wn, C, lane);
+        // ---- u = Au V, w = Aw K on tcgen05 once this head's v tile has landed
+        ok = cta_wait(tma_bar, tma_phase & 1);
+        if (ok) ++tma_phase, tma_pending = false;
+        if (ok && tid == 0) {
+            tc_fence_after();
+            const uint32_t id_W = idesc_bf16(64, 128, false, true);
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(tmem + kColU, smem_desc(sb + kAu + ks * 32, 16, 1024, kSw128),
+                         smem_desc(sb + kQV + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
+                mma_bf16(tmem + kColW, smem_desc(sb + kAw + ks * 32, 16, 1024, kSw128),
+                         smem_desc(sb + kKt + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
+            }
+            mma_commit(mma_bar);
+            mma_pending = true;
+        }
+        ok = ok && cta_wait(mma_bar, mma_phase & 1);
+        if (ok) ++mma_phase, mma_pending = false;
+        tc_fence_after();
+        if (ok && tid == 0 && gi + 1 < G) load_v(h + 1);  // the v tile is free again
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int col = 64 * wn + 8 * j + 2 * c4;
+        for (int part = 0; part < 2; ++part) {  // columns 64 wn + 32 part .. +31, 16 values at a time
+            float v[16];
+            const int cb = 64 * wn + 32 * part;
+            tmem_ld16x256_x4(tmem + lane_base + kColU + cb, v);  // u
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int col = cb + 8 * i + 2 * c4;
                 if (r0 < len)
                     *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r0) * d.Hv + h) * V + col) =
-                        make_float2(acc[j][0], acc[j][1]);
+                        make_float2(v[4 * i], v[4 * i + 1]);
                 if (r1 < len)
                     *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r1) * d.Hv + h) * V + col) =
-                        make_float2(acc[j][2], acc[j][3]);
+                        make_float2(v[4 * i + 2], v[4 * i + 3]);
             }
-        }
-        {
-            float acc[8][4] = {};
-            wgemm<8, false, true>(acc, tAw, tK, 16 * wm, 64 * wn, C, lane);
+            tmem_ld16x256_x4(tmem + lane_base + kColW + cb, v);  // w
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int col = 64 * wn + 8 * j + 2 * c4;
+            for (int i = 0; i < 4; ++i) {
+                const int col = cb + 8 * i + 2 * c4;
                 if (r0 < len)
                     *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r0) * d.Hv + h) * K + col) =
-                        pack_bf16(acc[j][0], acc[j][1]);
+                        pack_bf16(v[4 * i], v[4 * i + 1]);
                 if (r1 < len)
                     *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r1) * d.Hv + h) * K + col) =
-                        pack_bf16(acc[j][2], acc[j][3]);
+                        pack_bf16(v[4 * i + 2], v[4 * i + 3]);
             }
         }
-        __syncthreads();  // v tile, Au, Aw, A, X free for the next value head
+        tc_fence_before();
+        __syncthreads();  // u, w columns, Au, Aw, A, X free for the next value head
+    }
+    if (!ok) {
+        if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
+        // a TMA load or MMA that has not completed may still be in flight: wait (bounded) for it
+        if (tid == 0) {
+            const uint64_t t1 = globaltimer();
+            while (tma_pending && !mbar_try_wait(smem_u32(tma_bar), tma_phase & 1) && globaltimer() - t1 < kWaitNs) {
+            }
+            while (mma_pending && !mbar_try_wait(smem_u32(mma_bar), mma_phase & 1) && globaltimer() - t1 < kWaitNs) {
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -276,13 +390,22 @@ __global__ void __launch_bounds__(kThreads, 2) prep3_kernel(const Prep3Params pr
 bool prep3_supported(const FwdArgs &a) { return a.dtype == GDN_DTYPE_BF16 && a.d.K == 128 && a.d.V == 128; }
 
 cudaError_t launch_prep3(const FwdArgs &a) {
-    if (a.d.NC == 0) return cudaSuccess;
+    const Dims &d = a.d;
+    if (d.NC == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || !a.p16 || !a.gamma) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
+    const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
+    const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
+    const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    if (!make_bf16_map(&mq, a.q, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mk, a.k, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mv, a.v, 3, dv, sv, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     Prep3Params p;
-    p.d = a.d;
-    p.q = (const __nv_bfloat16 *)a.q;
-    p.k = (const __nv_bfloat16 *)a.k;
-    p.v = (const __nv_bfloat16 *)a.v;
+    p.d = d;
     p.g = a.g;
     p.beta = a.beta;
     p.gamma_out = a.gamma;
@@ -290,9 +413,10 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     p.w_out = (__nv_bfloat16 *)a.w16;
     p.u_out = a.u32;
     p.p_out = (__nv_bfloat16 *)a.p16;
+    p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(prep3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    prep3_kernel<<<dim3(a.d.NC, a.d.Hq), kThreads, kSmemBytes, a.stream>>>(p);
+    prep3_kernel<<<dim3(d.NC, d.Hq), kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 
