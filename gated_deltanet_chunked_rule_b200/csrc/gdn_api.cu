@@ -93,6 +93,8 @@ struct Plan {
     size_t gamma_bytes, ainv_bytes, saved_bytes, seq_info_bytes;
     bool tc_ok;       // bf16 with K = V = 128: the tensor-core path
     size_t w_bytes, u_bytes, p_bytes;  // its chunk-prep outputs w (bf16), u (fp32), P (bf16)
+    size_t hs_bytes, ds_bytes;         // per-chunk entry states, Delta (bf16): saved for the backward
+    size_t core_bytes;                 // gamma | Ainv | w | u | P (what the forward itself needs)
     int max_chunks;   // chunks of the longest sequence
     int nseg;         // forward sequence split: segments per sequence (1 = none)
     size_t seg_bytes; // split scratch: c, P, start states of every segment
@@ -175,9 +177,15 @@ int make_plan(const gdn_problem *p, Plan *out) {
         P.u_bytes = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.V);
         P.p_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * kChunk * kChunk);
     }
-    // saved = gamma | Ainv | (bf16 K = V = 128) w, u, P, so that a backward
-    // given `saved` needs no chunk prep of its own
-    P.saved_bytes = P.gamma_bytes + P.ainv_bytes + P.w_bytes + P.u_bytes + P.p_bytes;
+    // saved = gamma | Ainv | (bf16 K = V = 128) w, u, P | every chunk's entry state
+    // and Delta, so that a backward given `saved` runs neither the chunk prep nor
+    // the recompute of the states
+    if (P.tc_ok) {
+        P.hs_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
+        P.ds_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
+    }
+    P.core_bytes = P.gamma_bytes + P.ainv_bytes + P.w_bytes + P.u_bytes + P.p_bytes;
+    P.saved_bytes = P.core_bytes + P.hs_bytes + P.ds_bytes;
     if (P.varlen) {
         for (int n = 0; n < p->num_seqs; ++n)
             P.max_chunks = std::max(P.max_chunks, (p->cu_seqlens_host[n + 1] - p->cu_seqlens_host[n] + kChunk - 1) / kChunk);
@@ -190,11 +198,23 @@ int make_plan(const gdn_problem *p, Plan *out) {
     return GDN_OK;
 }
 
-size_t fwd_ws_bytes(const Plan &P) {
-    // sequence table | gamma, Ainv, scaled inverses (used when the caller passes no `saved`)
-    // | sequence-split scratch
-    return P.seq_info_bytes + P.saved_bytes + P.seg_bytes;
+// Forward workspace: sequence table | gamma, Ainv, w, u, P (used when the caller
+// passes no `saved`) | sequence-split scratch. The size and the offsets come
+// from this one function.
+struct FwdLayout {
+    size_t seq, core, seg, total;
+};
+
+FwdLayout fwd_layout(const Plan &P) {
+    FwdLayout L;
+    L.seq = 0;
+    L.core = L.seq + P.seq_info_bytes;
+    L.seg = L.core + P.core_bytes;
+    L.total = L.seg + P.seg_bytes;
+    return L;
 }
+
+size_t fwd_ws_bytes(const Plan &P) { return fwd_layout(P).total; }
 
 // Backward workspace: sequence table | gamma, Ainv (when no `saved`) | per-chunk
 // entry states h | per-chunk exit-state gradients dh' | Delta | dDelta |
@@ -211,7 +231,7 @@ BwdLayout bwd_layout(const Plan &P) {
     const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
-    L.hc = L.saved + P.saved_bytes;
+    L.hc = L.saved + P.core_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dl;
@@ -237,7 +257,7 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
-    L.hc = L.saved + P.saved_bytes;
+    L.hc = L.saved + P.core_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dl;
@@ -252,8 +272,9 @@ bool tc_bwd_path(const Plan &P) {
            tc_bwd_supported(P.d, P.dtype) && P.tc_ok;
 }
 
-// Pointers into a saved buffer (or the workspace's copy of one): gamma | Ainv | w | u | P.
-void set_saved_ptrs(FwdArgs &a, char *sv, const Plan &P) {
+// Pointers into a saved buffer (or the workspace's copy of its core): gamma | Ainv |
+// w | u | P [| chunk entry states | Delta, only in a caller's saved buffer].
+void set_saved_ptrs(FwdArgs &a, char *sv, const Plan &P, bool with_states) {
     a.gamma = (float *)sv;
     a.ainv = sv + P.gamma_bytes;
     if (P.tc_ok) {
@@ -261,6 +282,10 @@ void set_saved_ptrs(FwdArgs &a, char *sv, const Plan &P) {
         a.w16 = x;
         a.u32 = (float *)(x + P.w_bytes);
         a.p16 = x + P.w_bytes + P.u_bytes;
+        if (with_states) {
+            a.h_chunks16 = sv + P.core_bytes;
+            a.delta16 = sv + P.core_bytes + P.hs_bytes;
+        }
     }
 }
 
@@ -400,7 +425,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     if (!status) return GDN_ERR_CUDA;
     char *ws = (char *)workspace;
     if ((rc = launch_plan(p, P, ws, status, st)) != GDN_OK) return rc;
-    char *sv = saved ? (char *)saved : ws + P.seq_info_bytes;
+    char *sv = saved ? (char *)saved : ws + fwd_layout(P).core;
 
     FwdArgs a;
     memset(&a, 0, sizeof(a));
@@ -408,7 +433,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.dtype = P.dtype;
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0;
     a.o = o; a.final_state = final_state;
-    set_saved_ptrs(a, sv, P);
+    set_saved_ptrs(a, sv, P, saved != nullptr);
     a.status = status;
     a.stream = st;
     a.nseg = 1;
@@ -428,7 +453,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     }
     if (hybrid && P.nseg > 1) {
         // sequence split: segment pass (c, P) -> composition of start states -> output pass
-        float *seg = (float *)(ws + P.seq_info_bytes + P.saved_bytes);
+        float *seg = (float *)(ws + fwd_layout(P).seg);
         const size_t per = (size_t)P.d.N * P.nseg * P.d.Hv * P.d.K;
         a.nseg = P.nseg;
         a.seg_c = seg;
@@ -437,6 +462,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
         FwdArgs s1 = a;
         s1.o = nullptr;
         s1.final_state = nullptr;
+        s1.h_chunks16 = s1.delta16 = nullptr;  // the output pass stores the true states
         s1.fwd_mode = 1;
         {
             TimedLaunch t("fwd_split_seg", st);
@@ -458,6 +484,16 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     } else {
         TimedLaunch t("fwd_simt", st);
         if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
+    }
+    if (saved && P.tc_ok && !hybrid) {
+        // keep `saved` complete for a tensor-core backward: the chunk states and Delta
+        FwdArgs r = a;
+        r.o = nullptr;
+        r.final_state = nullptr;
+        r.nseg = 1;
+        r.fwd_mode = 0;
+        TimedLaunch t("fwd_states", st);
+        if (launch_fwd2(r) != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;
 }
@@ -501,20 +537,23 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         f.nseg = 1;
         // gamma | Ainv | w | u | P: from the forward's `saved`, else made here
         char *sv = saved ? (char *)saved : ws + T.saved;
-        set_saved_ptrs(f, sv, P);
+        set_saved_ptrs(f, sv, P, saved != nullptr);
         const void *ainv = f.ainv;
         if (!saved) {
-            TimedLaunch t("bwd_prep3", st);
-            if (launch_prep3(f) != cudaSuccess) return GDN_ERR_CUDA;
-        }
-        f.o = nullptr;
-        f.final_state = nullptr;
-        f.h_chunks16 = ws + T.hc;
-        f.delta16 = ws + T.delta;
-        {
+            // no saved forward: chunk prep, then the recompute of every chunk's entry
+            // state and Delta
+            {
+                TimedLaunch t("bwd_prep3", st);
+                if (launch_prep3(f) != cudaSuccess) return GDN_ERR_CUDA;
+            }
+            f.o = nullptr;
+            f.final_state = nullptr;
+            f.h_chunks16 = ws + T.hc;
+            f.delta16 = ws + T.delta;
             TimedLaunch t("bwd_recompute", st);
             if (launch_fwd2(f) != cudaSuccess) return GDN_ERR_CUDA;
         }
+        char *hcs = (char *)f.h_chunks16, *dls = (char *)f.delta16;
         BwdArgs b;
         memset(&b, 0, sizeof(b));
         b.d = P.d;
@@ -532,7 +571,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         }
         {
             TimedLaunch t("bwd_grad", st);
-            if (launch_bwd_grad_tc(b, ws + T.hc, ws + T.dhc, ws + T.delta, ws + T.ddelta, (float *)(ws + T.dqp),
+            if (launch_bwd_grad_tc(b, hcs, ws + T.dhc, dls, ws + T.ddelta, (float *)(ws + T.dqp),
                                    (float *)(ws + T.dkp)) != cudaSuccess)
                 return GDN_ERR_CUDA;
         }

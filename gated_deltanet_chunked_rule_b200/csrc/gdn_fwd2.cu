@@ -535,7 +535,8 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     p.seg_h0 = a.seg_h0;
     p.seg_c = a.seg_c;
     p.seg_P = a.seg_P;
-    if (p.mode != kWhole && ((p.mode == kSegOut && !p.seg_h0) || (p.mode == kSegPass && (!p.seg_c || !p.seg_P || p.o))))
+    if (p.mode != kWhole && ((p.mode == kSegOut && !p.seg_h0) ||
+                             (p.mode == kSegPass && (!p.seg_c || !p.seg_P || p.o || p.h_chunks || p.delta))))
         return cudaErrorInvalidValue;
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(fwd2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

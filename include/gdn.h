@@ -92,10 +92,14 @@ size_t gdn_bwd_workspace_size(const gdn_problem *p);
  * ([num_chunks, Hv, 64, 64], fp32 for GDN_DTYPE_F32 problems, bf16 for
  * GDN_DTYPE_BF16), i.e. the "g, A" that page 1's low-level forward returns
  * and its backward takes back ("底层 API" section of the FlashQLA write-up).
- * For bf16 problems with K = V = 128 the buffer continues with the two
- * scaled inverses Ainv diag(beta) and Ainv diag(beta e^gamma) (bf16,
- * [num_chunks, Hv, 2, 64, 64]) that the tensor-core kernels consume, so a
- * backward given `saved` runs no chunk prep. Each 256-byte aligned. */
+ * For bf16 problems with K = V = 128 the buffer continues with what the
+ * tensor-core backward needs from the forward: w = Ainv diag(beta e^gamma) K
+ * (bf16 [B*T, Hv, K]), u = Ainv diag(beta) V (fp32 [B*T, Hv, V]), the
+ * decay-masked P = M o Q K^T of every chunk (bf16 [num_chunks, Hv, 64, 64]),
+ * and every chunk's entry state (bf16 [num_chunks, Hv, K, V]) and Delta (bf16
+ * [B*T, Hv, V]) -- the per-chunk states h that page 1's low-level forward also
+ * returns -- so that a backward given `saved` runs neither the chunk prep nor
+ * a recompute of the states. Each part 256-byte aligned. */
 size_t gdn_saved_size(const gdn_problem *p);
 
 /* Forward. h0 may be NULL (zero initial state); final_state may be NULL (not

@@ -51,19 +51,27 @@ def prob(B_=1, T=256, Hq=2, Hv=4, K=128, V=128, ns=0, cu=None, dtype=1, scale=0.
     return p
 
 
+def saved_bf16_k128(ntok, nc, Hv=4, K=128, V=128):
+    # gamma | Ainv | w | u | P | chunk entry states | Delta (include/gdn.h)
+    return (ntok * Hv * 4 + nc * Hv * 64 * 64 * 2 + ntok * Hv * K * 2 + ntok * Hv * V * 4
+            + nc * Hv * 64 * 64 * 2 + nc * Hv * K * V * 2 + ntok * Hv * V * 2)
+
+
 def test_workspace_sizes(L):
     p = prob()
     nc = 4  # 256 tokens -> 4 chunks
     gamma = 256 * 4 * 4
     ainv = nc * 4 * 64 * 64 * 2
-    assert L.gdn_saved_size(ctypes.byref(p)) == gamma + ainv
+    assert L.gdn_saved_size(ctypes.byref(p)) == saved_bf16_k128(256, nc)
     assert L.gdn_fwd_workspace_size(ctypes.byref(p)) >= gamma + ainv
     assert L.gdn_bwd_workspace_size(ctypes.byref(p)) > L.gdn_fwd_workspace_size(ctypes.byref(p))
-    p32 = prob(dtype=0)
+    p32 = prob(dtype=0)  # fp32: gamma and Ainv (fp32) only
     assert L.gdn_saved_size(ctypes.byref(p32)) == gamma + 2 * ainv
+    p64 = prob(K=64, V=64)  # bf16 but not the tensor-core shape: gamma and Ainv only
+    assert L.gdn_saved_size(ctypes.byref(p64)) == gamma + ainv
     # ragged varlen: lengths 100, 0, 28, 128 -> 2 + 0 + 1 + 2 chunks
     pv = prob(T=256, ns=4, cu=[0, 100, 100, 128, 256])
-    assert L.gdn_saved_size(ctypes.byref(pv)) == gamma + 5 * 4 * 64 * 64 * 2
+    assert L.gdn_saved_size(ctypes.byref(pv)) == saved_bf16_k128(256, 5)
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -149,3 +149,15 @@ def test_backward_deterministic():
     b = gpu_bwd(x)
     for n in NAMES:
         torch.testing.assert_close(a[n], b[n], rtol=0, atol=0)
+
+
+def test_backward_from_states_saved_by_a_split_forward(oracle_mod, monkeypatch):
+    # the forward stores every chunk's entry state and Delta in `saved`; with the
+    # sequence split the output pass stores them, and the backward reuses them
+    w = Workload("bwd_split_saved", B=1, T=1100, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, grads=True,
+                 seed=17)
+    x = make_inputs(w)
+    monkeypatch.setenv("GDN_NSEG", "3")
+    g = gpu_bwd(x, use_saved=True)
+    monkeypatch.delenv("GDN_NSEG")
+    check(oracle_mod, x, g, "bwd from split-forward states")
