@@ -71,7 +71,7 @@ static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 23
 constexpr uint32_t kColQ = 0, kColP = 32, kOBuf = 64, kTmemCols = 128;
 
 // Hand-over counters (the number of chunks, or states, the producer has finished).
-enum Ctr { kH, kDelta, kStage, kODone, kTmemO, kNumCtr };
+enum Ctr { kH, kDelta, kStage, kODone, kTmemO, kStored, kNumCtr };
 
 struct Small {
     uint64_t full[kStages];
@@ -114,7 +114,8 @@ struct Fwd2Params {
 __global__ void __launch_bounds__(kThreads, 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
-            const __grid_constant__ CUtensorMap tm_p, const Fwd2Params prm) {
+            const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_hs,
+            const __grid_constant__ CUtensorMap tm_ds, const Fwd2Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -128,6 +129,8 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int K = 128, V = 128;
     const bool want_o = prm.o != nullptr;
+    // chunk entry states and Delta go to global memory by TMA stores from kHb / kDb
+    const bool states = prm.h_chunks != nullptr;
     // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
     const SeqRange seq = seq_range(d, n);
     const int nch_seq = (seq.len + kChunk - 1) / kChunk;
@@ -215,19 +218,6 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (tid == 0) sm->loads_landed = j + 1;
             const float gC = gl, gtok[2] = {gt0, gt1};
             if (j + 1 < nch) gl = gamma_at(j + 1, 63), gt0 = gamma_at(j + 1, 16 * p + g), gt1 = gamma_at(j + 1, 16 * p + g + 8);
-            if (prm.h_chunks) {  // entry state of chunk j, rounded as the products read it
-                __nv_bfloat16 *hc = prm.h_chunks + ((size_t)(sr.chunk0 + j) * d.Hv + h) * K * V + c0;
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int dim = 32 * p + 16 * mt + g + half * 8;
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-                            *reinterpret_cast<uint32_t *>(hc + (size_t)dim * V + 8 * (cb + nt) + 2 * c4) =
-                                pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
-                    }
-            }
             // ---- w h : tokens 16p..16p+15, columns of n-tiles cb, cb+1 (A = w tile, B = h)
             float acc[2][4] = {};
             {
@@ -274,7 +264,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     }
             }
             // ---- Delta = u - w h -> Db[j%2] (read by DP) ; e^{gamma_C - gamma} Delta -> Dt
-            ok = chain_sync(!want_o || j < 2 || wait_ge(&ctr[kODone], j - 1, abort_flag));  // DP of j-2 read Db[j%2]
+            // DP and the state store of chunk j-2 read Db[j%2]
+            ok = chain_sync(j < 2 || ((!want_o || wait_ge(&ctr[kODone], j - 1, abort_flag)) &&
+                                      (!states || wait_ge(&ctr[kStored], j - 1, abort_flag))));
             if (!ok) break;
             {
                 const uint32_t db = sb + kDb + (j & 1) * 4096 + c4 * 4, dt = sb + kDt + c4 * 4;
@@ -294,7 +286,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         const float x1 = live ? uu.y - acc[nt][2 * half + 1] : 0.f;
                         st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(x0, x1));
                         st_shared_b32(dt + (cb + nt) * 1024 + off, pack_bf16(sc * x0, sc * x1));
-                        if (prm.delta && live)
+                        if (states && len < kChunk && live)  // ragged last chunk: no TMA store past its end
                             *reinterpret_cast<uint32_t *>(prm.delta + ((size_t)(sr.start + j * kChunk + tok) * d.Hv + h) * V +
                                                           c0 + col) = pack_bf16(x0, x1);
                     }
@@ -327,7 +319,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (tid == 0) publish(&ctr[kStage], j + 1);
             // ---- h_{j+1} -> Hb[(j+1)%2] once DQ of chunk j-1 (which read it) is done; then
             //      Delta_j and h_{j+1} go to the output MMAs behind one proxy fence
-            ok = chain_sync(!want_o || j < 1 || wait_ge(&ctr[kODone], j, abort_flag));
+            // DQ and the state store of chunk j-1 read Hb[(j+1)%2]
+            ok = chain_sync(j < 1 || ((!want_o || wait_ge(&ctr[kODone], j, abort_flag)) &&
+                                      (!states || wait_ge(&ctr[kStored], j, abort_flag))));
             if (!ok) break;
             write_hb((j + 1) & 1);
             fence_proxy_async();
@@ -441,10 +435,26 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (!ok) break;
                     issue_loads(j + 2);
                 }
+                if (!want_o && !states) continue;
+                // h_j and Delta_j are in kHb[j%2], kDb[j%2]
+                ok = wait_ge(&ctr[kH], j + 1, abort_flag) && wait_ge(&ctr[kDelta], j + 1, abort_flag);
+                if (!ok) break;
+                if (states) {
+                    // entry state (four 8-column boxes of 128 rows) and, for a full chunk, Delta
+                    const int len = min(kChunk, sr.len - j * kChunk);
+                    const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
+                    const int row = ((sr.chunk0 + j) * d.Hv + h) * K;
+                    for (int nb = 0; nb < 4; ++nb) {
+                        tma_store_2d(&tm_hs, hb + nb * 2048, c0 + 8 * nb, row);
+                        if (len == kChunk) tma_store_3d(&tm_ds, db + nb * 1024, c0 + 8 * nb, h, sr.start + j * kChunk);
+                    }
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                    publish(&ctr[kStored], j + 1);
+                }
                 if (!want_o) continue;
                 // DQ = Q h_j, DP = P Delta_j into buffer j%2 once the epilogue has read chunk j-2's
-                ok = wait_ge(&ctr[kH], j + 1, abort_flag) && wait_ge(&ctr[kDelta], j + 1, abort_flag) &&
-                     wait_ge(&ctr[kTmemO], j >= 1 ? j - 1 : 0, abort_flag);
+                ok = wait_ge(&ctr[kTmemO], j >= 1 ? j - 1 : 0, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
@@ -465,6 +475,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 set_status(prm.status, GDN_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
+            bulk_wait_all();  // state stores complete before the CTA's shared memory goes away
         }
         __syncwarp();
     }
@@ -489,13 +500,13 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 }
 
 bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank, const cuuint64_t *dims,
-              const cuuint64_t *strides, const cuuint32_t *box) {
+              const cuuint64_t *strides, const cuuint32_t *box,
+              CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, dt, rank, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, dt, rank, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -504,7 +515,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || (a.o && !a.p16)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mw, mu, mp;
+    CUtensorMap mq, mk, mw, mu, mp, mhs, mds;
     const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
     const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
@@ -521,6 +532,18 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     if (!make_map(&mq, BF, a.q, 3, dq, sq, b64) || !make_map(&mk, BF, a.k, 3, dq, sq, b64) ||
         !make_map(&mw, BF, a.w16, 3, dw, sw, b64) || !make_map(&mu, F32, a.u32, 3, du, su, bu) ||
         !make_map(&mp, BF, a.p16 ? a.p16 : a.w16, 2, dp, sp, bp))
+        return cudaErrorInvalidValue;
+    // state stores: entry states as [NC * Hv * K rows][V], Delta as [T][Hv][V]; 16-byte boxes
+    const bool st = a.h_chunks16 != nullptr;
+    if (st != (a.delta16 != nullptr)) return cudaErrorInvalidValue;
+    const cuuint64_t dhs[2] = {(cuuint64_t)d.V, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * d.K};
+    const cuuint64_t shs[1] = {(cuuint64_t)d.V * 2};
+    const cuuint32_t bhs[2] = {8, 128};
+    const cuuint64_t dds[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sds[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
+    const cuuint32_t bds[3] = {8, 1, 64};
+    if (!make_map(&mhs, BF, st ? a.h_chunks16 : a.w16, 2, dhs, shs, bhs, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mds, BF, st ? a.delta16 : a.w16, 3, dds, sds, bds, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     Fwd2Params p;
     p.d = d;
@@ -543,7 +566,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
     dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
-    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, p);
+    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, mhs, mds, p);
     return cudaGetLastError();
 }
 
