@@ -121,6 +121,45 @@ def kernel_bytes(name, w, saved=False):
     return table.get(name)
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, bytes per launch)
+# of one ncu capture per kernel (summaries under profiles/), valid only for the
+# workload and step they were taken on and only while the kernel's sources are
+# byte-identical to the captured build (sha256 over the listed files).
+NCU_TRAFFIC = {
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=645888256 + 307320576,
+                     sources=["gdn_bwd_grad.cu"],
+                     sha256="7f74d3569aa5c14ce7c2e7a3f9055bc055fc8ae4206c046e9c8382433567aeb8"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072320 + 167649792,
+                   sources=["gdn_bwd_dh.cu"],
+                   sha256="dffa02f93180ece98e9e3ec45634479026cc213ef9376735daccfff066b3a7f8"),
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd", bytes=303084544 + 57421312,
+                       sources=["gdn_fwd2.cu"],
+                       sha256="ab1104a6ecb3bdf74902b31d96f0c64569529bf335816f6523efb0a37159c919"),
+    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd", bytes=138035200 + 187329280,
+                  sources=["gdn_prep3.cu"],
+                  sha256="c40c7df4f99dbc4efa75743e164771cbd04d313a0c62cb0c1ae93d5875554097"),
+}
+TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
+
+
+def measured_traffic(kernel, workload, step):
+    """ncu DRAM bytes per launch for this kernel, or None if not captured for this
+    workload and step or if the kernel's sources changed since the capture."""
+    rec = NCU_TRAFFIC.get(kernel)
+    if not rec or rec["workload"] != workload or rec["step"] != step:
+        return None
+    import hashlib
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "gated_deltanet_chunked_rule_b200", "csrc")
+    h = hashlib.sha256()
+    try:
+        for f in rec["sources"] + TRAFFIC_COMMON_SOURCES:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return rec["bytes"] if h.hexdigest() == rec["sha256"] else None
+
+
 class Clocks:
     """Samples SM clocks and throttle reasons with nvidia-smi while running."""
 
@@ -371,7 +410,8 @@ def main():
     roofline = {"kernel": dom, "bound": "hbm", "unit": "GB/s",
                 "achieved": dom_bytes / dom_avg_s / 1e9 if dom_bytes else None,
                 "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)",
-                "traffic": None}
+                "traffic": measured_traffic(dom, w.name, "fwd+bwd" if do_bwd else "fwd"),
+                "algorithmic_bytes": dom_bytes}
     if roofline["achieved"]:
         roofline["frac"] = roofline["achieved"] / roofline["peak"]
 
