@@ -21,7 +21,9 @@
 //               straight from tensor memory (the 16x256b load layout is the
 //               mma.sync accumulator layout, and chain warp p sits on TMEM
 //               sub-partition p);
-//   warps 8-11  aux: dO' = scale e^gamma o dO into shared memory;
+//   warps 8-11  aux: dO' = scale e^gamma o dO into shared memory, one chunk
+//               ahead of the chain, and the copies of dh' and dDelta from
+//               shared memory to global memory, off the chain's path;
 //   warp 12     issuer: TMA ring (q, k, w, P, dO per chunk) and, on tcgen05,
 //               Y = P^T dO and X = Q^T dO' into double-buffered TMEM.
 // Y and X do not depend on the chain, so they are ready one or two chunks
@@ -46,8 +48,8 @@ constexpr int kBV = 32;
 constexpr int kStages = 3;
 
 // ---- shared memory (bytes from a 1024-aligned base)
-constexpr int kHb = 0;          // 8192       dh' (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16, chain only
-constexpr int kDb = 8192;       // 4096       -dDelta (bf16): (n/8)*1024 + (t/8)*128 + (t%8)*16, chain only
+constexpr int kHb = 0;          // 8192       dh' (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16
+constexpr int kDb = 8192;       // 4096       -dDelta (bf16): (n/8)*1024 + (t/8)*128 + (t%8)*16
 constexpr int kDO2 = 12288;     // 2 x 4096   dO' (bf16), layout of kDb (B of X)
 constexpr int kStage0 = 20480;  // TMA ring
 // per stage: q, k, w [64][128] bf16 (two 64-column halves, 128-byte swizzle),
@@ -61,7 +63,9 @@ static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 23
 // Tensor memory: two buffers of 64 columns, Y (M = 64) | X (M = 128).
 constexpr uint32_t kColY = 0, kColX = 32, kYBuf = 64, kTmemCols = 128;
 
-enum Ctr { kPReady, kStage, kNumCtr };
+// kHbFull / kDbFull: the chain has put dh' / -dDelta of an iteration in kHb / kDb;
+// kHbRead / kDbRead: the aux warps have copied them to global memory.
+enum Ctr { kPReady, kStage, kHbFull, kDbFull, kHbRead, kDbRead, kNumCtr };
 
 struct Small {
     uint64_t full[kStages];
@@ -171,29 +175,20 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int it = 0; it < nch && ok; ++it) {
             const int ci = chunk_of(it);
             const int len = min(kChunk, sr.len - ci * kChunk);
-            const int t0 = sr.start + ci * kChunk;
             const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
             // stage landed (and every warp's dh' is in kHb: the barrier orders them)
             ok = chain_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag));
             if (!ok) break;
-            if (tid == 0) sm->loads_landed = it + 1;
+            if (tid == 0) {
+                sm->loads_landed = it + 1;
+                publish(&ctr[kHbFull], it + 1);  // kHb holds dh' of this chunk (written before the barrier)
+            }
             const float gC = gl, gtok[2] = {gt0, gt1};
             if (it + 1 < nch) gl = gamma_at(it + 1, 63), gt0 = gamma_at(it + 1, 16 * p + g), gt1 = gamma_at(it + 1, 16 * p + g + 8);
-            {  // dh' of this chunk, rounded as the products read it
-                __nv_bfloat16 *hc = prm.dh_chunks + ((size_t)(sr.chunk0 + ci) * d.Hv + h) * K * V + c0;
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int dim = 32 * p + 16 * mt + g + half * 8;
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-                            *reinterpret_cast<uint32_t *>(hc + (size_t)dim * V + 8 * (cb + nt) + 2 * c4) =
-                                pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
-                    }
-            }
             // ---- Y and X of this chunk from tensor memory (issued now, waited after A)
-            ok = chain_sync(wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag));
+            // Y, X of this chunk computed; the aux has copied the previous -dDelta out of kDb
+            ok = chain_sync(wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag) &&
+                            (it < 1 || wait_ge(&ctr[kDbRead], it, abort_flag)));
             if (!ok) break;
             if (tid == 0) sm->mma_seen = it + 1;
             tc_fence_after();
@@ -226,7 +221,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             tmem_wait_ld3(yr, xr0, xr1);
             tc_fence_before();
-            // ---- dDelta = e^{gamma_C - gamma} A + scale Y  -> ddelta (global), -dDelta -> kDb
+            // ---- dDelta = e^{gamma_C - gamma} A + scale Y; -dDelta -> kDb
             {
                 const uint32_t db = sb + kDb + c4 * 4;
 #pragma unroll
@@ -237,18 +232,15 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint32_t off = (tok >> 3) * 128 + (tok & 7) * 16;
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        const int col = 8 * (cb + nt) + 2 * c4;
                         const float y0 = __uint_as_float(yr[4 * nt + 2 * half]), y1 = __uint_as_float(yr[4 * nt + 2 * half + 1]);
                         const float x0 = live ? fmaf(sc, acc[nt][2 * half], scl * y0) : 0.f;
                         const float x1 = live ? fmaf(sc, acc[nt][2 * half + 1], scl * y1) : 0.f;
                         st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(-x0, -x1));
-                        if (live)
-                            *reinterpret_cast<uint32_t *>(prm.ddelta + ((size_t)(t0 + tok) * d.Hv + h) * V + c0 + col) =
-                                pack_bf16(x0, x1);
                     }
                 }
             }
             chain_sync(true);  // every warp reads all 64 tokens of dDelta below
+            if (tid == 0) publish(&ctr[kDbFull], it + 1);
             // ---- dh = e^{gamma_C} dh' + X + w^T (-dDelta) : rows 32p..+31, 16 columns, K = 64 tokens
             {
                 const float eC = __expf(gC);
@@ -285,7 +277,10 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
-            chain_sync(true);  // all reads of kHb, kDb, the stage and this TMEM buffer are done
+            // all reads of kHb, kDb, the stage and this TMEM buffer are done; dh' of this
+            // chunk has been copied out of kHb
+            ok = chain_sync(wait_ge(&ctr[kHbRead], it + 1, abort_flag));
+            if (!ok) break;
             if (tid == 0) publish(&ctr[kStage], it + 1);
             write_hb();
         }
@@ -314,13 +309,14 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int ta = atid >> 2, tb2 = (atid + kAux) >> 2, cc = atid & 3;
         float ga = 0.f, gb = 0.f;
         if (nch > 0) ga = gamma_at(0, ta), gb = gamma_at(0, tb2);
-        for (int it = 0; it < nch && ok; ++it) {
+        // dO' of iteration it into dO'[it % 2] once its stage has landed and X of
+        // iteration it - 2 (the buffer's last reader) is done
+        auto make_do = [&](int it) -> bool {
             const int ci = chunk_of(it);
             const int len = min(kChunk, sr.len - ci * kChunk);
-            // the stage has landed; X of iteration it - 2 (the last reader of dO'[it % 2]) is done
-            ok = aux_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
-                          (it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag)));
-            if (!ok) break;
+            if (!aux_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
+                          (it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag))))
+                return false;
             const float fa = ta < len ? scl * __expf(ga) : 0.f, fb = tb2 < len ? scl * __expf(gb) : 0.f;
             if (it + 1 < nch) ga = gamma_at(it + 1, ta), gb = gamma_at(it + 1, tb2);
             const uint32_t stg = sb + kStage0 + (it % kStages) * kStageBytes + kDO;
@@ -343,6 +339,45 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             fence_proxy_async();
             aux_sync(true);
             if (atid == 0) publish(&ctr[kPReady], it + 1);
+            return true;
+        };
+        if (nch > 0) ok = make_do(0);
+        for (int it = 0; it < nch && ok; ++it) {
+            const int ci = chunk_of(it);
+            const int len = min(kChunk, sr.len - ci * kChunk);
+            const int t0 = sr.start + ci * kChunk;
+            if (it + 1 < nch) {
+                ok = make_do(it + 1);  // one iteration ahead of the chain
+                if (!ok) break;
+            }
+            // dh' of this iteration: kHb -> dh_chunks (16-byte rows of 8 columns)
+            ok = aux_sync(wait_ge(&ctr[kHbFull], it + 1, abort_flag));
+            if (!ok) break;
+            {
+                __nv_bfloat16 *hc = prm.dh_chunks + ((size_t)(sr.chunk0 + ci) * d.Hv + h) * K * V + c0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int e = atid + kAux * i, k = e & 127, nb = e >> 7;
+                    const uint4 v4 = ld_shared_v4(sb + kHb + nb * 2048 + k * 16);
+                    *reinterpret_cast<uint4 *>(hc + (size_t)k * V + 8 * nb) = v4;
+                }
+            }
+            aux_sync(true);
+            if (atid == 0) publish(&ctr[kHbRead], it + 1);
+            // dDelta of this iteration: kDb holds -dDelta -> ddelta (live tokens), sign restored
+            ok = aux_sync(wait_ge(&ctr[kDbFull], it + 1, abort_flag));
+            if (!ok) break;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int e = atid + kAux * i, t = e & 63, nb = e >> 6;
+                if (t < len) {
+                    uint4 v4 = ld_shared_v4(sb + kDb + nb * 1024 + t * 16);
+                    v4.x ^= 0x80008000u, v4.y ^= 0x80008000u, v4.z ^= 0x80008000u, v4.w ^= 0x80008000u;
+                    *reinterpret_cast<uint4 *>(prm.ddelta + ((size_t)(t0 + t) * d.Hv + h) * V + c0 + 8 * nb) = v4;
+                }
+            }
+            aux_sync(true);
+            if (atid == 0) publish(&ctr[kDbRead], it + 1);
         }
         if (!ok) {
             if (atid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -373,15 +408,10 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t id_Y = idesc_bf16(64, 32, true, true);
             const uint32_t id_X = idesc_bf16(128, 32, true, true);
             for (int it = 0; it < nch && ok; ++it) {
-                // refill the stage of iteration it - 1 with iteration it + 2 once the chain is
-                // done with it (which also means its Y, X and dO' are consumed)
-                if (it >= 1 && it + 2 < nch) {
-                    ok = wait_ge(&ctr[kStage], it, abort_flag);
-                    if (!ok) break;
-                    issue_loads(it + 2);
-                }
                 // Y, X of iteration it into buffer it % 2 once dO' is written and the chain
-                // has read that buffer's previous contents (iteration it - 2)
+                // has read that buffer's previous contents (iteration it - 2). They depend on
+                // loaded tiles only, so they are issued before the refill below, which waits
+                // for the chain to finish iteration it - 1.
                 ok = wait_ge(&ctr[kPReady], it + 1, abort_flag) && wait_ge(&ctr[kStage], it >= 1 ? it - 1 : 0, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -397,6 +427,13 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 mma_commit(&sm->mmaB[it & 1]);
                 sm->mma_issued = it + 1;
+                // refill the stage of iteration it - 1 with iteration it + 2 once the chain is
+                // done with it (which also means its Y, X and dO' are consumed)
+                if (it >= 1 && it + 2 < nch) {
+                    ok = wait_ge(&ctr[kStage], it, abort_flag);
+                    if (!ok) break;
+                    issue_loads(it + 2);
+                }
             }
             if (!ok) {
                 set_status(prm.status, GDN_ERR_TIMEOUT);
