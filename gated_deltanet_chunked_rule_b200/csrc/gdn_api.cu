@@ -243,10 +243,9 @@ BwdLayout bwd_layout(const Plan &P) {
 
 // Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv,
 // scaled inverses (when no `saved`) |
-// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta |
-// fp32 dq, dk partials per value head.
+// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta.
 struct TcBwdLayout {
-    size_t seq, saved, hc, dhc, delta, ddelta, dqp, dkp, total;
+    size_t seq, saved, hc, dhc, delta, ddelta, total;
 };
 
 TcBwdLayout tc_bwd_layout(const Plan &P) {
@@ -254,16 +253,13 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     TcBwdLayout L;
     const size_t hc = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
     const size_t dl = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
-    const size_t qp = align_up(sizeof(float) * (size_t)d.T_total * d.Hv * d.K);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
     L.hc = L.saved + P.core_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dl;
-    L.dqp = L.ddelta + dl;
-    L.dkp = L.dqp + qp;
-    L.total = L.dkp + qp;
+    L.total = L.ddelta + dl;
     return L;
 }
 
@@ -525,7 +521,8 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
 
     if (tc_bwd_path(P)) {
         // tensor-core path: prep (gamma, Ainv when not saved, scaled inverses) ->
-        // recompute of h, Delta (bf16) -> reverse dh scan -> per-chunk gradients -> GQA sum
+        // recompute of h, Delta (bf16) -> reverse dh scan -> per-chunk gradients (which
+        // also sum dq, dk over each qk head's group of value heads)
         const TcBwdLayout T = tc_bwd_layout(P);
         FwdArgs f;
         memset(&f, 0, sizeof(f));
@@ -571,14 +568,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         }
         {
             TimedLaunch t("bwd_grad", st);
-            if (launch_bwd_grad_tc(b, hcs, ws + T.dhc, dls, ws + T.ddelta, (float *)(ws + T.dqp),
-                                   (float *)(ws + T.dkp)) != cudaSuccess)
-                return GDN_ERR_CUDA;
-        }
-        {
-            TimedLaunch t("bwd_final", st);
-            if (launch_bwd_final(b, (const float *)(ws + T.dqp), (const float *)(ws + T.dkp)) != cudaSuccess)
-                return GDN_ERR_CUDA;
+            if (launch_bwd_grad_tc(b, hcs, ws + T.dhc, dls, ws + T.ddelta) != cudaSuccess) return GDN_ERR_CUDA;
         }
         return GDN_OK;
     }

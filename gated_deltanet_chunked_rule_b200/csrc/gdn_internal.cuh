@@ -152,12 +152,11 @@ bool prep3_supported(const FwdArgs &a);
 cudaError_t launch_prep3(const FwdArgs &a);
 // Sequence split: start state of every segment from h0 and the segments' (c, P).
 cudaError_t launch_split_compose(const FwdArgs &a);
-// Tensor-core backward (bf16, K = V = 128): reverse dh scan, per-chunk gradients,
-// and the GQA reduction of the dq / dk partials.
+// Tensor-core backward (bf16, K = V = 128): reverse dh scan, then the per-chunk
+// gradients, which sum dq and dk over each qk head's group of value heads.
 bool tc_bwd_supported(const Dims &d, int dtype);
 cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16);
 cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const void *dh_chunks16,
-                               const void *delta16, const void *ddelta16, float *dq_part, float *dk_part);
-cudaError_t launch_bwd_final(const BwdArgs &a, const float *dq_part, const float *dk_part);
+                               const void *delta16, const void *ddelta16);
 
 }  // namespace gdn

@@ -500,46 +500,6 @@ cudaError_t bwd_dispatch(const BwdArgs &a, float *dq_part, float *dk_part) {
 
 }  // namespace
 
-// bf16 outputs, four consecutive elements per thread (16-byte partial loads).
-__global__ void __launch_bounds__(kThreads) bwd_final_bf16x4(Dims d, const float4 *__restrict__ dq_part,
-                                                           const float4 *__restrict__ dk_part,
-                                                           uint2 *__restrict__ dq, uint2 *__restrict__ dk) {
-    const int G = d.Hv / d.Hq, K4 = d.K / 4;
-    const size_t total = (size_t)d.T_total * d.Hq * K4;
-    for (size_t e = (size_t)blockIdx.x * kThreads + threadIdx.x; e < total; e += (size_t)gridDim.x * kThreads) {
-        const int j = (int)(e % K4);
-        const size_t th = e / K4;  // t * Hq + hq
-        const int hq = (int)(th % d.Hq);
-        const size_t t = th / d.Hq;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-        for (int g = 0; g < G; ++g) {
-            const size_t off = (t * d.Hv + (size_t)hq * G + g) * K4 + j;
-            const float4 x = __ldcs(dq_part + off), y = __ldcs(dk_part + off);
-            a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
-            b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
-        }
-        __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w);
-        __nv_bfloat162 k0 = __floats2bfloat162_rn(b.x, b.y), k1 = __floats2bfloat162_rn(b.z, b.w);
-        dq[e] = make_uint2(*reinterpret_cast<uint32_t *>(&q0), *reinterpret_cast<uint32_t *>(&q1));
-        dk[e] = make_uint2(*reinterpret_cast<uint32_t *>(&k0), *reinterpret_cast<uint32_t *>(&k1));
-    }
-}
-
-cudaError_t launch_bwd_final(const BwdArgs &a, const float *dq_part, const float *dk_part) {
-    const size_t total = (size_t)a.d.T_total * a.d.Hq * a.d.K;
-    if (total == 0) return cudaSuccess;
-    if (a.dtype == GDN_DTYPE_BF16) {
-        const size_t n4 = total / 4;
-        const int blocks = (int)((n4 + kThreads - 1) / kThreads < 148 * 8 ? (n4 + kThreads - 1) / kThreads : 148 * 8);
-        bwd_final_bf16x4<<<blocks, kThreads, 0, a.stream>>>(a.d, (const float4 *)dq_part, (const float4 *)dk_part,
-                                                           (uint2 *)a.dq, (uint2 *)a.dk);
-        return cudaGetLastError();
-    }
-    const int blocks = (int)((total + kThreads - 1) / kThreads < 148 * 16 ? (total + kThreads - 1) / kThreads : 148 * 16);
-    bwd_final<float><<<blocks, kThreads, 0, a.stream>>>(a.d, dq_part, dk_part, (float *)a.dq, (float *)a.dk);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part) {
     const int kv = (a.d.K == 64 ? 0 : 2) + (a.d.V == 64 ? 0 : 1);
     if (a.dtype == GDN_DTYPE_F32) {

@@ -236,6 +236,23 @@ __device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Stores 16 fp32 per thread in the 16x256b.x4 layout (the layout tmem_ld16x256_x4
+// reads back) and waits until the store has completed.
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+        "tcgen05.wait::st.sync.aligned;"
+        :
+        : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
 // The same 16x256b.x2 load without the wait, so that its latency can overlap
 // other work; the registers are valid only after tmem_wait_ld().
 __device__ __forceinline__ void tmem_ld16x256_x2_nowait(uint32_t taddr, uint32_t (&r)[8]) {
