@@ -60,6 +60,9 @@ constexpr int kThreads = 256;
 constexpr int kWN = 2;  // column groups: warp w owns column half w / 4
 constexpr int C = 64, K = 128, V = 128;
 constexpr int kStoreTid = 32;  // issues the TMA stores and the loads of the buffers they read
+// The products of a round are issued by two threads (thread 0 and kStoreTid), each
+// committing to the round's mbarrier (two arrivals): a single issuing thread spends
+// about 70 cycles per tcgen05.mma.
 
 // ---- shared memory (bytes from a 1024-aligned base); [64][128] tiles are two
 //      64-column halves of [64 rows][128 B], 128-byte swizzle
@@ -111,14 +114,17 @@ __device__ __forceinline__ float2 ld_pair_sw(uint32_t base, int r, int c) {
     return unpack_bf16(u);
 }
 
+// Operand descriptors are built once per tile; a k-step only moves the start
+// address (descriptor bits 0..13, in 16-byte units), by a constant once the
+// issue loops are unrolled.
 // K-major operand over a tile of 64-column halves: 16 columns per k-step.
-__device__ __forceinline__ uint64_t kdesc(uint32_t base, int ks, int half_bytes) {
-    return smem_desc(base + (ks >> 2) * half_bytes + (ks & 3) * 32, 16, 1024, kSw128);
+__device__ __forceinline__ uint64_t kbase(uint32_t base) { return smem_desc(base, 16, 1024, kSw128); }
+__device__ __forceinline__ constexpr uint64_t kstep(int ks, int half_bytes) {
+    return (uint64_t)(((ks >> 2) * half_bytes + (ks & 3) * 32) >> 4);
 }
 // MN-major operand (K runs down the rows): 16 rows per k-step; halves 8192 bytes apart.
-__device__ __forceinline__ uint64_t mdesc(uint32_t base, int ks) {
-    return smem_desc(base + ks * 2048, 8192, 1024, kSw128);
-}
+__device__ __forceinline__ uint64_t mbase(uint32_t base) { return smem_desc(base, 8192, 1024, kSw128); }
+__device__ __forceinline__ constexpr uint64_t mstep(int ks) { return (uint64_t)(ks * 2048 >> 4); }
 
 struct GradParams {
     Dims d;
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBar);
 
     if (tid == 0) {
-        for (int i = 0; i < kNumBar; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kNumBar; ++i) mbar_init(&bars[i], i == kBarMma ? 2 : 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -274,6 +280,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
             load_v(cur);
         }
     }
+    float pg = 0.f, pb = 0.f;  // threads < C: gamma and beta of row tid of the coming step
+    auto fetch_gate = [&](const Step &s) {
+        if (tid < C) {
+            const int rr = min(tid, s.len - 1);
+            pg = prm.gamma[(size_t)(s.t0 + rr) * d.Hv + head(s)];
+            pb = tid < s.len ? prm.beta[(size_t)(s.t0 + tid) * d.Hv + head(s)] : 0.f;
+        }
+    };
+    if (cur.valid) fetch_gate(cur);
     bool ok = true;
     for (int j = 0; cur.valid; ++j) {
         Step nxt = cur;
@@ -287,11 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         // previous step, has completed)
         if (tid == 0 && nxt.valid) load_delta(nxt, db ^ 1);
         if (tid < C) {
-            const int r = tid, rr = min(r, len - 1);
-            const float gm = prm.gamma[(size_t)(t0 + rr) * d.Hv + h];
-            vec.gam[r] = gm;
-            vec.egam[r] = __expf(gm);
-            vec.bet[r] = r < len ? prm.beta[(size_t)(t0 + r) * d.Hv + h] : 0.f;
+            vec.gam[tid] = pg;  // padded rows repeat the last live gamma
+            vec.egam[tid] = __expf(pg);
+            vec.bet[tid] = pb;
         }
         ok = ok && (!first || (wait_bar(kBarQ) && wait_bar(kBarK))) && wait_bar(kBarD0 + db) &&
              wait_bar(kBarDO) && wait_bar(kBarA);
@@ -299,18 +312,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         // ---- round 1: S, G, P1 (64 x 64) and dU (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
-            const uint32_t idCC = idesc_bf16(64, 64, false, false), idU = idesc_bf16(64, 128, true, true);
+            const uint32_t idCC = idesc_bf16(64, 64, false, false);
+            const uint64_t q = kbase(sb + kQ), k = kbase(sb + kKt);
+#pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16(tmem + kCS, kdesc(sb + kQ, ks, 8192), kdesc(sb + kKt, ks, 8192), idCC, ks > 0);
-                mma_bf16(tmem + kCG, kdesc(sb + kKt, ks, 8192), kdesc(sb + kKt, ks, 8192), idCC, ks > 0);
-                mma_bf16(tmem + kCP1, kdesc(sb + kdO, ks, 8192), kdesc(sD, ks, 8192), idCC, ks > 0);
+                mma_bf16(tmem + kCS, q + kstep(ks, 8192), k + kstep(ks, 8192), idCC, ks > 0);
+                mma_bf16(tmem + kCG, k + kstep(ks, 8192), k + kstep(ks, 8192), idCC, ks > 0);
             }
-            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCU, mdesc(sb + kA, ks), mdesc(sb + kdD, ks), idU, ks > 0);
+            commit_mma();
+        } else if (ok && tid == kStoreTid) {
+            tc_fence_after();
+            const uint32_t idCC = idesc_bf16(64, 64, false, false), idU = idesc_bf16(64, 128, true, true);
+            const uint64_t o = kbase(sb + kdO), dl = kbase(sD), ai = mbase(sb + kA), dd = mbase(sb + kdD);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCP1, o + kstep(ks, 8192), dl + kstep(ks, 8192), idCC, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCU, ai + mstep(ks), dd + mstep(ks), idU, ks > 0);
             commit_mma();
         }
         if (tid == kStoreTid) bulk_wait_read<0>();  // the previous dk store has read T1 | dG
         ok = __syncthreads_and(ok);                 // the gate vectors
         if (!ok) break;
+        if (nxt.valid) fetch_gate(nxt);
         const float gC = vec.gam[63];  // gamma at the chunk's last token (padded rows repeat it)
         const float gr[2] = {vec.gam[r0], vec.gam[r1]};
         const float er[2] = {vec.egam[r0], vec.egam[r1]};
@@ -394,22 +417,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         // ---- round 2: dAkk (64 x 64), T1 K, T1^T Q onto dk, dO h^T (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
-            const uint32_t idCC = idesc_bf16(64, 64, false, false);
-            const uint32_t idKM = idesc_bf16(64, 128, false, true), idMM = idesc_bf16(64, 128, true, true);
-            const uint32_t idKK = idesc_bf16(64, 128, false, false);
-            for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16(tmem + kCAkk, kdesc(sb + kdU, ks, 8192), kdesc(sD, ks, 8192), idCC, ks > 0);
-                mma_bf16(tmem + kCQ1, kdesc(sb + kdO, ks, 8192), kdesc(sb + kH, ks, 16384), idKK, ks > 0);
-            }
-            for (int ks = 0; ks < 4; ++ks) {
-                mma_bf16(tmem + kCTK, kdesc(sb + kT1, ks, 8192), mdesc(sb + kKt, ks), idKM, ks > 0);
-                mma_bf16(tmem + kCDK, mdesc(sb + kT1, ks), mdesc(sb + kQ, ks), idMM, ks > 0 || !first);
-            }
+            const uint32_t idCC = idesc_bf16(64, 64, false, false), idKM = idesc_bf16(64, 128, false, true);
+            const uint64_t du = kbase(sb + kdU), dl = kbase(sD), t1 = kbase(sb + kT1), km = mbase(sb + kKt);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCAkk, du + kstep(ks, 8192), dl + kstep(ks, 8192), idCC, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCTK, t1 + kstep(ks, 8192), km + mstep(ks), idKM, ks > 0);
             commit_mma();
-        }
-        if (ok && tid == kStoreTid && nxt.valid) {
-            bulk_wait_read<0>();  // dv has left the v tile
-            load_v(nxt);
+        } else if (ok && tid == kStoreTid) {
+            tc_fence_after();
+            const uint32_t idMM = idesc_bf16(64, 128, true, true), idKK = idesc_bf16(64, 128, false, false);
+            const uint64_t o = kbase(sb + kdO), hh = kbase(sb + kH), t1m = mbase(sb + kT1), qm = mbase(sb + kQ);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCQ1, o + kstep(ks, 8192), hh + kstep(ks, 16384), idKK, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCDK, t1m + mstep(ks), qm + mstep(ks), idMM, ks > 0 || !first);
+            commit_mma();
+            if (nxt.valid) {
+                bulk_wait_read<0>();  // dv has left the v tile
+                load_v(nxt);
+            }
         }
         ok = ok && wait_bar(kBarMma);
         tc_fence_after();
@@ -479,17 +506,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idKK = idesc_bf16(64, 128, false, false);
-            const uint32_t idKM = idesc_bf16(64, 128, false, true), idMM = idesc_bf16(64, 128, true, true);
+            const uint64_t du = kbase(sb + kdU), hh = kbase(sb + kH), dl = kbase(sD), dh = kbase(sb + kdH);
+#pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16(tmem + kCKb, kdesc(sb + kdU, ks, 8192), kdesc(sb + kH, ks, 16384), idKK, ks > 0);
-                mma_bf16(tmem + kCK2, kdesc(sD, ks, 8192), kdesc(sb + kdH, ks, 16384), idKK, ks > 0);
-            }
-            for (int ks = 0; ks < 4; ++ks) {
-                mma_bf16(tmem + kCDK, kdesc(sb + kdG, ks, 8192), mdesc(sb + kKt, ks), idKM, true);
-                mma_bf16(tmem + kCDK, mdesc(sb + kdG, ks), mdesc(sb + kKt, ks), idMM, true);
+                mma_bf16(tmem + kCKb, du + kstep(ks, 8192), hh + kstep(ks, 16384), idKK, ks > 0);
+                mma_bf16(tmem + kCK2, dl + kstep(ks, 8192), dh + kstep(ks, 16384), idKK, ks > 0);
             }
             commit_mma();
-        } else if (tid == kStoreTid && last) {
+        } else if (tid == kStoreTid) {
+            tc_fence_after();
+            const uint32_t idKM = idesc_bf16(64, 128, false, true), idMM = idesc_bf16(64, 128, true, true);
+            const uint64_t dg = kbase(sb + kdG), dgm = mbase(sb + kdG), km = mbase(sb + kKt);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_bf16(tmem + kCDK, dg + kstep(ks, 8192), km + mstep(ks), idKM, true);
+                mma_bf16(tmem + kCDK, dgm + mstep(ks), km + mstep(ks), idMM, true);
+            }
+            commit_mma();
+        }
+        if (tid == kStoreTid && last) {
             if (full) {
                 tma_store_3d(&tm.dq, sb + kQ, 0, cur.hq, t0);
                 tma_store_3d(&tm.dq, sb + kQ + 8192, 64, cur.hq, t0);
