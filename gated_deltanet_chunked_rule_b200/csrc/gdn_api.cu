@@ -182,7 +182,7 @@ int make_plan(const gdn_problem *p, Plan *out) {
     // the recompute of the states
     if (P.tc_ok) {
         P.hs_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
-        P.ds_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
+        P.ds_bytes = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * kChunk * d.Hv * d.V);  // per chunk, blocked
     }
     P.core_bytes = P.gamma_bytes + P.ainv_bytes + P.w_bytes + P.u_bytes + P.p_bytes;
     P.saved_bytes = P.core_bytes + P.hs_bytes + P.ds_bytes;
@@ -252,13 +252,14 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     const Dims &d = P.d;
     TcBwdLayout L;
     const size_t hc = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
+    const size_t dlb = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * kChunk * d.Hv * d.V);  // blocked per chunk
     const size_t dl = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
     L.hc = L.saved + P.core_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
-    L.ddelta = L.delta + dl;
+    L.ddelta = L.delta + dlb;
     L.total = L.ddelta + dl;
     return L;
 }

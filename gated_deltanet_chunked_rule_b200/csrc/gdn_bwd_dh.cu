@@ -84,7 +84,8 @@ struct BwdDhParams {
     Dims d;
     const float *gamma;          // [T_total, Hv]
     const float *dht;            // [N, Hv, K, V] or null
-    __nv_bfloat16 *dh_chunks;    // [NC, Hv, K, V]: gradient w.r.t. each chunk's exit state
+    __nv_bfloat16 *dh_chunks;    // gradient w.r.t. each chunk's exit state, blocked: per (chunk, head)
+                                 // V/32 slices of [4][128][8] (the tile layout of kHb)
     __nv_bfloat16 *ddelta;       // [T_total, Hv, V]
     float *dh0;                  // [N, Hv, K, V] or null
     float scale;
@@ -188,7 +189,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- Y and X of this chunk from tensor memory (issued now, waited after A)
             // Y, X of this chunk computed; the aux has copied the previous -dDelta out of kDb
             ok = chain_sync(wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag) &&
-                            (it < 1 || wait_ge(&ctr[kDbRead], it, abort_flag)));
+                            (tid != 0 || it < 1 || wait_ge(&ctr[kDbRead], it, abort_flag)));
             if (!ok) break;
             if (tid == 0) sm->mma_seen = it + 1;
             tc_fence_after();
@@ -279,7 +280,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             // all reads of kHb, kDb, the stage and this TMEM buffer are done; dh' of this
             // chunk has been copied out of kHb
-            ok = chain_sync(wait_ge(&ctr[kHbRead], it + 1, abort_flag));
+            ok = chain_sync(tid != 0 || wait_ge(&ctr[kHbRead], it + 1, abort_flag));
             if (!ok) break;
             if (tid == 0) publish(&ctr[kStage], it + 1);
             write_hb();
@@ -315,7 +316,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int ci = chunk_of(it);
             const int len = min(kChunk, sr.len - ci * kChunk);
             if (!aux_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
-                          (it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag))))
+                          (atid != 0 || it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag))))
                 return false;
             const float fa = ta < len ? scl * __expf(ga) : 0.f, fb = tb2 < len ? scl * __expf(gb) : 0.f;
             if (it + 1 < nch) ga = gamma_at(it + 1, ta), gb = gamma_at(it + 1, tb2);
@@ -350,22 +351,22 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 ok = make_do(it + 1);  // one iteration ahead of the chain
                 if (!ok) break;
             }
-            // dh' of this iteration: kHb -> dh_chunks (16-byte rows of 8 columns)
-            ok = aux_sync(wait_ge(&ctr[kHbFull], it + 1, abort_flag));
+            // dh' of this iteration: kHb -> dh_chunks, one contiguous block per (chunk, head,
+            // column slice) in the tile layout
+            ok = aux_sync(atid != 0 || wait_ge(&ctr[kHbFull], it + 1, abort_flag));
             if (!ok) break;
             {
-                __nv_bfloat16 *hc = prm.dh_chunks + ((size_t)(sr.chunk0 + ci) * d.Hv + h) * K * V + c0;
+                __nv_bfloat16 *hc = prm.dh_chunks + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + blockIdx.z) * (K * kBV);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int e = atid + kAux * i, k = e & 127, nb = e >> 7;
-                    const uint4 v4 = ld_shared_v4(sb + kHb + nb * 2048 + k * 16);
-                    *reinterpret_cast<uint4 *>(hc + (size_t)k * V + 8 * nb) = v4;
+                    const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 128 + k
+                    *reinterpret_cast<uint4 *>(hc + 8 * e) = ld_shared_v4(sb + kHb + e * 16);
                 }
             }
             aux_sync(true);
             if (atid == 0) publish(&ctr[kHbRead], it + 1);
             // dDelta of this iteration: kDb holds -dDelta -> ddelta (live tokens), sign restored
-            ok = aux_sync(wait_ge(&ctr[kDbFull], it + 1, abort_flag));
+            ok = aux_sync(atid != 0 || wait_ge(&ctr[kDbFull], it + 1, abort_flag));
             if (!ok) break;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {

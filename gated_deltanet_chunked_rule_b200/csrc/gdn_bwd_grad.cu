@@ -33,6 +33,9 @@
 // column half w / 4), and do the elementwise terms and the row and column sums
 // in a fixed order.
 //
+// Delta, h and dh' arrive in the blocked layout the chain kernels keep them in
+// (per 32-column slice: 8-column blocks of 16-byte rows), which is the K-major
+// operand layout without swizzle; each is one contiguous bulk copy per step.
 // Each input tile of the next step is loaded by TMA as soon as the current
 // step is done with its buffer (Ainv and dDelta after round 1, dO after round
 // 2, h and dh' after round 3; Delta has two buffers), so that only a new
@@ -68,15 +71,15 @@ constexpr int kStoreTid = 32;  // issues the TMA stores and the loads of the buf
 //      64-column halves of [64 rows][128 B], 128-byte swizzle
 constexpr int kQ = 0, kKt = 16384;  // per item; dq goes out through the q tile
 constexpr int kdO = 32768;
-constexpr int kD = 49152;           // Delta, two buffers (step parity)
+constexpr int kD = 49152;           // Delta, two buffers (step parity): (v/8)*1024 + t*16
 constexpr int kdD = 81920;
 constexpr int kVt = 98304;          // v; dv goes out through it
 constexpr int kA = 114688;          // Ainv [64 s][64 r]
 constexpr int kT1 = 122880;         // T1 [64 r][64 s]   } dk goes out through these two:
 constexpr int kdG = 131072;         // dG [64 r][64 s]   } one [64][128] tile
 constexpr int kdU = 139264;         // dU [64 r][128 v]
-constexpr int kH = 155648;          // h [128 k][128 v]: two halves of [128 rows][128 B]
-constexpr int kdH = 188416;         // dh'
+constexpr int kH = 155648;          // h [128 k][128 v]: (v/8)*2048 + k*16
+constexpr int kdH = 188416;         // dh', same layout
 constexpr int kVec = 221184;
 constexpr int kBar = kVec + 4096;
 constexpr int kSmemBytes = kBar + 128 + 1024;
@@ -125,9 +128,15 @@ __device__ __forceinline__ constexpr uint64_t kstep(int ks, int half_bytes) {
 // MN-major operand (K runs down the rows): 16 rows per k-step; halves 8192 bytes apart.
 __device__ __forceinline__ uint64_t mbase(uint32_t base) { return smem_desc(base, 8192, 1024, kSw128); }
 __device__ __forceinline__ constexpr uint64_t mstep(int ks) { return (uint64_t)(ks * 2048 >> 4); }
+// K-major operand without swizzle, the blocked layout: core matrices of 8 rows x
+// 16 bytes, 128 bytes apart down the rows, kblk bytes apart along K (Delta 1024,
+// h and dh' 2048); a k-step of 16 is two core matrices along K.
+__device__ __forceinline__ uint64_t bbase(uint32_t base, uint32_t kblk) { return smem_desc(base, kblk, 128, kSwNone); }
+__device__ __forceinline__ constexpr uint64_t bstep(int ks, int kblk) { return (uint64_t)(ks * 2 * kblk >> 4); }
 
 struct GradParams {
     Dims d;
+    const __nv_bfloat16 *delta, *h, *dh;  // blocked: per (chunk, head) 4 slices of [4][64][8] / [4][128][8]
     const float *gamma, *beta;
     __nv_bfloat16 *dq, *dk;  // [T, Hq, K]
     __nv_bfloat16 *dv;       // [T, Hv, V]
@@ -137,8 +146,8 @@ struct GradParams {
 };
 
 struct GradMaps {
-    CUtensorMap q, k, v, d_o, delta, ddelta, h, dh, ainv;  // loads
-    CUtensorMap dq, dk, dv;                               // stores
+    CUtensorMap q, k, v, d_o, ddelta, ainv;  // loads
+    CUtensorMap dq, dk, dv;                 // stores
 };
 
 // One step: value head g of the group of qk head hq, on chunk cg.
@@ -235,8 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
     auto load_delta = [&](const Step &s, int buf) {
         const int b = kBarD0 + buf;
         expect(b, 16384);
-        tma_load_3d(smem + kD + buf * 16384, &tm.delta, &bars[b], 0, head(s), s.t0);
-        tma_load_3d(smem + kD + buf * 16384 + 8192, &tm.delta, &bars[b], 64, head(s), s.t0);
+        bulk_load(smem + kD + buf * 16384, prm.delta + ((size_t)s.cg * d.Hv + head(s)) * (C * V), 16384, &bars[b]);
     };
     auto load_do = [&](const Step &s) {
         expect(kBarDO, 16384);
@@ -255,12 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         tma_load_3d(smem + kVt + 8192, &tm.v, &bars[kBarV], 64, head(s), s.t0);
     };
     auto load_st = [&](const Step &s) {  // h and dh'
-        const int krow = (s.cg * d.Hv + head(s)) * K;
-        expect(kBarSt, 4 * 16384);
-        tma_load_2d(smem + kH, &tm.h, &bars[kBarSt], 0, krow);
-        tma_load_2d(smem + kH + 16384, &tm.h, &bars[kBarSt], 64, krow);
-        tma_load_2d(smem + kdH, &tm.dh, &bars[kBarSt], 0, krow);
-        tma_load_2d(smem + kdH + 16384, &tm.dh, &bars[kBarSt], 64, krow);
+        const size_t off = ((size_t)s.cg * d.Hv + head(s)) * (K * V);
+        expect(kBarSt, 2 * 32768);
+        bulk_load(smem + kH, prm.h + off, 32768, &bars[kBarSt]);
+        bulk_load(smem + kdH, prm.dh + off, 32768, &bars[kBarSt]);
     };
     auto commit_mma = [&]() {
         mma_commit(&bars[kBarMma]);
@@ -323,9 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         } else if (ok && tid == kStoreTid) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false), idU = idesc_bf16(64, 128, true, true);
-            const uint64_t o = kbase(sb + kdO), dl = kbase(sD), ai = mbase(sb + kA), dd = mbase(sb + kdD);
+            const uint64_t o = kbase(sb + kdO), dl = bbase(sD, 1024), ai = mbase(sb + kA), dd = mbase(sb + kdD);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCP1, o + kstep(ks, 8192), dl + kstep(ks, 8192), idCC, ks > 0);
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCP1, o + kstep(ks, 8192), dl + bstep(ks, 1024), idCC, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCU, ai + mstep(ks), dd + mstep(ks), idU, ks > 0);
             commit_mma();
@@ -418,18 +424,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false), idKM = idesc_bf16(64, 128, false, true);
-            const uint64_t du = kbase(sb + kdU), dl = kbase(sD), t1 = kbase(sb + kT1), km = mbase(sb + kKt);
+            const uint64_t du = kbase(sb + kdU), dl = bbase(sD, 1024), t1 = kbase(sb + kT1), km = mbase(sb + kKt);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCAkk, du + kstep(ks, 8192), dl + kstep(ks, 8192), idCC, ks > 0);
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCAkk, du + kstep(ks, 8192), dl + bstep(ks, 1024), idCC, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCTK, t1 + kstep(ks, 8192), km + mstep(ks), idKM, ks > 0);
             commit_mma();
         } else if (ok && tid == kStoreTid) {
             tc_fence_after();
             const uint32_t idMM = idesc_bf16(64, 128, true, true), idKK = idesc_bf16(64, 128, false, false);
-            const uint64_t o = kbase(sb + kdO), hh = kbase(sb + kH), t1m = mbase(sb + kT1), qm = mbase(sb + kQ);
+            const uint64_t o = kbase(sb + kdO), hh = bbase(sb + kH, 2048), t1m = mbase(sb + kT1), qm = mbase(sb + kQ);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCQ1, o + kstep(ks, 8192), hh + kstep(ks, 16384), idKK, ks > 0);
+            for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCQ1, o + kstep(ks, 8192), hh + bstep(ks, 2048), idKK, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCDK, t1m + mstep(ks), qm + mstep(ks), idMM, ks > 0 || !first);
             commit_mma();
@@ -506,11 +512,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idKK = idesc_bf16(64, 128, false, false);
-            const uint64_t du = kbase(sb + kdU), hh = kbase(sb + kH), dl = kbase(sD), dh = kbase(sb + kdH);
+            const uint64_t du = kbase(sb + kdU), hh = bbase(sb + kH, 2048), dl = bbase(sD, 1024), dh = bbase(sb + kdH, 2048);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                mma_bf16(tmem + kCKb, du + kstep(ks, 8192), hh + kstep(ks, 16384), idKK, ks > 0);
-                mma_bf16(tmem + kCK2, dl + kstep(ks, 8192), dh + kstep(ks, 16384), idKK, ks > 0);
+                mma_bf16(tmem + kCKb, du + kstep(ks, 8192), hh + bstep(ks, 2048), idKK, ks > 0);
+                mma_bf16(tmem + kCK2, dl + bstep(ks, 1024), dh + bstep(ks, 2048), idKK, ks > 0);
             }
             commit_mma();
         } else if (tid == kStoreTid) {
@@ -711,24 +717,22 @@ cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const v
     const cuuint64_t dvv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
     const cuuint64_t svv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
     const cuuint32_t b3[3] = {64, 1, 64};
-    const cuuint64_t dst[2] = {(cuuint64_t)d.V, (cuuint64_t)d.NC * d.Hv * d.K};
-    const cuuint64_t sst[1] = {(cuuint64_t)d.V * 2};
-    const cuuint32_t bst[2] = {64, 128};
     const cuuint64_t dai[2] = {64, (cuuint64_t)d.NC * d.Hv * 64};
     const cuuint64_t sai[1] = {128};
     const cuuint32_t bai[2] = {64, 64};
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_bf16_map(&m.q, a.q, 3, dqk, sqk, b3, SW) || !make_bf16_map(&m.k, a.k, 3, dqk, sqk, b3, SW) ||
         !make_bf16_map(&m.v, a.v, 3, dvv, svv, b3, SW) || !make_bf16_map(&m.d_o, a.d_o, 3, dvv, svv, b3, SW) ||
-        !make_bf16_map(&m.delta, delta16, 3, dvv, svv, b3, SW) ||
         !make_bf16_map(&m.ddelta, ddelta16, 3, dvv, svv, b3, SW) ||
-        !make_bf16_map(&m.h, h_chunks16, 2, dst, sst, bst, SW) || !make_bf16_map(&m.dh, dh_chunks16, 2, dst, sst, bst, SW) ||
         !make_bf16_map(&m.ainv, a.ainv, 2, dai, sai, bai, SW) ||
         !make_bf16_map(&m.dq, a.dq, 3, dqk, sqk, b3, SW) || !make_bf16_map(&m.dk, a.dk, 3, dqk, sqk, b3, SW) ||
         !make_bf16_map(&m.dv, a.dv, 3, dvv, svv, b3, SW))
         return cudaErrorInvalidValue;
     GradParams p;
     p.d = d;
+    p.delta = (const __nv_bfloat16 *)delta16;
+    p.h = (const __nv_bfloat16 *)h_chunks16;
+    p.dh = (const __nv_bfloat16 *)dh_chunks16;
     p.gamma = a.gamma;
     p.beta = a.beta;
     p.dq = (__nv_bfloat16 *)a.dq;

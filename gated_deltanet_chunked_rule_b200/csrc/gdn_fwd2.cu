@@ -2,14 +2,14 @@
 // the sequential state chain on warp-level tensor-core MMAs, the output on
 // tcgen05. Everything that does not depend on the state (w, u and the
 // decay-masked P = M o Q K^T of every chunk) comes ready-made from the
-// chunk-prep kernel (gdn_prep3.cu) through a TMA ring.
+// chunk-prep kernel (gdn_prep3.cu) through TMA rings.
 //
 // One CTA per (sequence or segment, value head, 32-column slice of V). Per
 // 64-token chunk (h the chunk-entry state, h = S^T, notation of gdn_internal.cuh):
 //
 //   chain (mma.sync, fp32 state in registers):
 //     Delta = u - w h,     h <- e^{gamma_C} h + K^T (e^{gamma_C - gamma} o Delta)
-//   output (tcgen05, TMEM accumulators, one chunk behind the chain):
+//   output (tcgen05, TMEM accumulators, behind the chain):
 //     DQ = Q h,  DP = P Delta,   o = scale (e^gamma o DQ + DP)
 //
 // Why this split (measured on B200): a tcgen05 MMA takes ~450 cycles from
@@ -17,24 +17,39 @@
 // chunk, whereas a dependent mma.sync costs ~20 cycles; the output products do
 // not feed the chain, so they run on tcgen05 off the critical path. Shared
 // memory bandwidth (128 B/clk/SM) is the next limit, which is why every
-// state-independent product is hoisted into the prep kernel.
+// state-independent product is hoisted into the prep kernel, and why each
+// chain warp owns whole rows: the w and K^T fragments are read once per chunk.
 //
-// Warp roles (416 threads):
-//   warps 0-7   chain: h (128 x 32 fp32) in mma fragments, warp w holding
-//               state rows 32 (w % 4) .. +31 and columns 16 (w / 4) .. +15.
-//   warps 8-11  epilogue: o from the double-buffered DQ/DP accumulators;
-//               warp 8 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15).
-//   warp 12     issuer: 3-deep TMA ring (q, k, w, u, P per chunk) and the
-//               DQ/DP MMAs.
+// Warp roles (320 threads):
+//   warps 0-3   chain: h (128 x 32 fp32) in mma fragments, warp p holding
+//               state rows 32p .. +31 (all 32 columns). The w and K^T
+//               fragments and the u values of chunk j+1 are loaded into
+//               registers while chunk j updates the state, so a chunk's
+//               critical path only reads h and e^{gamma_C - gamma} Delta from
+//               shared memory. Two barriers per chunk.
+//   warps 4-7   epilogue: o from the double-buffered DQ/DP accumulators;
+//               warp 4 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15).
+//   warp 8      output issuer: the DQ/DP MMAs, the (q, P) TMA ring, and the
+//               bulk copies of the chunk states and Delta to global memory.
+//   warp 9      chain producer: the (k, w, u) TMA ring, refilled as soon as the
+//               chain has a stage in registers.
 // Roles hand over through monotonically increasing shared-memory counters
-// (release/acquire), which cannot alias the way mbarrier parities can when a
-// producer runs ahead; mbarriers only where the hardware signals (TMA
-// completion, tcgen05.commit). Every wait is bounded in time; a wait that
-// expires records GDN_ERR_TIMEOUT and winds the CTA down.
+// (release/acquire; one thread polls, a barrier passes it on), which cannot
+// alias the way mbarrier parities can when a producer runs ahead; mbarriers
+// only where the hardware signals (TMA completion, tcgen05.commit). Every
+// wait is bounded in time; a wait that expires records GDN_ERR_TIMEOUT and
+// winds the CTA down.
 //
 // Modes: whole sequences from h0; the recompute for the backward (no output,
 // stores every chunk's entry state and Delta in bf16); and the two passes of
 // the sequence split (see Fwd2Mode).
+//
+// Saved states and Delta are kept in the shared-memory tile layout, one
+// contiguous block per (chunk, value head, 32-column slice), so that each is
+// one bulk copy: entry state h [NC][Hv][V/32][4][128][8] (block of 8 columns
+// n/8, state row k, 8 columns), Delta [NC][Hv][V/32][4][64][8] (token rows; rows
+// past a ragged chunk's end are zero). These blocks are K-major operand tiles
+// without swizzle for the backward's products.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -47,8 +62,8 @@ namespace {
 using namespace sm100;
 using namespace warp;
 
-constexpr int kThreads = 416;  // 8 chain + 4 epilogue + 1 issuer warps
-constexpr int kRole = 256;     // chain threads
+constexpr int kThreads = 320;  // 4 chain + 4 epilogue + output issuer + chain producer
+constexpr int kRole = 128;     // chain threads
 constexpr int kEpi = 128;      // epilogue threads
 constexpr int kBV = 32;
 constexpr int kStages = 3;
@@ -57,27 +72,32 @@ constexpr int kStages = 3;
 constexpr int kHb = 0;          // 2 x 8192   h (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16 (k = state row)
 constexpr int kDb = 16384;      // 2 x 4096   Delta (bf16), same layout with k = token (B of DP)
 constexpr int kDt = 24576;      // 4096       e^{gamma_C - gamma} Delta, chain only
-constexpr int kStage0 = 28672;  // TMA ring
-// per stage: q [64][128] bf16 and k, w likewise (two 64-column halves, 128-byte
-// swizzle), u [64][32] fp32 (128-byte swizzle), P [64][64] bf16 (128-byte swizzle)
-constexpr int kQ = 0, kK = 16384, kW = 32768, kU = 49152, kP = 57344, kStageBytes = 65536;
-constexpr int kTxFull = 65536;                  // q, k, w, u, P
-constexpr int kTxChain = 16384 + 16384 + 8192;  // k, w, u (no output)
-constexpr int kSmall = kStage0 + kStages * kStageBytes;
+constexpr int kC0 = 28672;      // chain ring: k, w [64][128] bf16 (two 64-column halves,
+                                // 128-byte swizzle), u [64][32] fp32 (128-byte swizzle)
+constexpr int kK = 0, kW = 16384, kU = 32768, kCStageBytes = 40960;
+constexpr int kO0 = kC0 + kStages * kCStageBytes;  // output ring: q [64][128] bf16, P [64][64] bf16
+constexpr int kQ = 0, kP = 16384, kOStageBytes = 24576;
+constexpr int kSmall = kO0 + kStages * kOStageBytes;
 constexpr int kSmemBytes = kSmall + 2048 + 1024;
-static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory layout");
+static_assert(kC0 % 1024 == 0 && kO0 % 1024 == 0 && kCStageBytes % 1024 == 0 && kOStageBytes % 1024 == 0 &&
+                  kSmemBytes <= 232448,
+              "shared memory layout");
 
 // DQ, DP double-buffered in tensor memory: buffer b at columns 64 b.
 constexpr uint32_t kColQ = 0, kColP = 32, kOBuf = 64, kTmemCols = 128;
 
 // Hand-over counters (the number of chunks, or states, the producer has finished).
-enum Ctr { kH, kDelta, kStage, kODone, kTmemO, kStored, kNumCtr };
+// kChain, one release store per chunk: 1 once h_0 is in kHb and chunk 0's stage is
+// in registers, then j + 2 after chunk j (Delta_j in kDb, h_{j+1} in kHb, chunk
+// j+1's stage in registers). kODone chunks whose DQ/DP are complete, kTmemO chunks
+// whose accumulators are read, kStored chunks whose state copies have read kHb / kDb.
+enum Ctr { kChain, kODone, kTmemO, kStored, kNumCtr };
 
 struct Small {
-    uint64_t full[kStages];
+    uint64_t cfull[kStages], ofull[kStages];
     uint64_t mmaO[2];
     uint32_t ctr[kNumCtr];
-    int loads_issued, loads_landed, mma_issued, mma_seen;
+    int cl_issued, cl_landed, ol_issued, ol_landed, mma_issued, mma_seen;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -99,8 +119,8 @@ struct Fwd2Params {
     const float *h0;      // [N, Hv, K, V] or null
     __nv_bfloat16 *o;     // [T_total, Hv, V], or null: no output (the backward's recompute)
     float *final_state;   // [N, Hv, K, V] or null
-    __nv_bfloat16 *h_chunks;  // [NC, Hv, K, V] entry state of every chunk (bf16, as the products read it) or null
-    __nv_bfloat16 *delta;     // [T_total, Hv, V] Delta (bf16) or null
+    __nv_bfloat16 *h_chunks;  // entry state of every chunk (bf16, as the products read it; blocked) or null
+    __nv_bfloat16 *delta;     // Delta of every chunk (bf16; blocked) or null
     // Sequence split: blockIdx.x = sequence * nseg + segment; a segment is a
     // contiguous run of ceil(chunks / nseg) chunks of its sequence.
     int nseg;
@@ -114,8 +134,7 @@ struct Fwd2Params {
 __global__ void __launch_bounds__(kThreads, 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
-            const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_hs,
-            const __grid_constant__ CUtensorMap tm_ds, const Fwd2Params prm) {
+            const __grid_constant__ CUtensorMap tm_p, const Fwd2Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -129,7 +148,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int K = 128, V = 128;
     const bool want_o = prm.o != nullptr;
-    // chunk entry states and Delta go to global memory by TMA stores from kHb / kDb
+    // chunk entry states and Delta go to global memory by bulk copies from kHb / kDb
     const bool states = prm.h_chunks != nullptr;
     // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
     const SeqRange seq = seq_range(d, n);
@@ -144,15 +163,18 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const size_t seg_idx = (size_t)n * nseg + sseg;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm->full[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm->cfull[s], 1);
+            mbar_init(&sm->ofull[s], 1);
+        }
         mbar_init(&sm->mmaO[0], 1);
         mbar_init(&sm->mmaO[1], 1);
         for (int c = 0; c < kNumCtr; ++c) sm->ctr[c] = 0;
-        sm->loads_issued = sm->loads_landed = sm->mma_issued = sm->mma_seen = 0;
+        sm->cl_issued = sm->cl_landed = sm->ol_issued = sm->ol_landed = sm->mma_issued = sm->mma_seen = 0;
         sm->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 12) {
+    if (warp == 8) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -168,11 +190,11 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         return prm.gamma[(size_t)(sr.start + j * kChunk + min(r, len - 1)) * d.Hv + h];
     };
 
-    if (warp < 8) {
+    if (warp < 4) {
         // =========================================================== chain
-        const int p = warp & 3, cb = (warp >> 2) * 2;  // state rows 32p.., n-tiles cb, cb+1 (16 columns)
-        const int g = lane >> 2, c4 = lane & 3;
-        float hf[2][2][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8(cb+nt)+2c4(+1)
+        const int p = warp;  // state rows 32p.., tokens 16p.. of the w h product
+        const int g = lane >> 2, c4 = lane & 3, mi = lane >> 3;
+        float hf[2][4][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8nt+2c4(+1)
         {
             const float *src = prm.mode == kWhole ? (prm.h0 ? prm.h0 + ((size_t)n * d.Hv + h) * K * V : nullptr)
                                : prm.mode == kSegOut ? prm.seg_h0 + (seg_idx * d.Hv + h) * K * V
@@ -181,11 +203,11 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int dim = 32 * p + 16 * mt + g + ((q >> 1) << 3);
-                        const int col = 8 * (cb + nt) + 2 * c4 + (q & 1);
+                        const int col = 8 * nt + 2 * c4 + (q & 1);
                         hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : (ident && dim == c0 - V + col ? 1.f : 0.f);
                     }
         }
@@ -197,80 +219,97 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int half = 0; half < 2; ++half) {
                     const int dim = 32 * p + 16 * mt + g + half * 8;
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        st_shared_b32(base + (cb + nt) * 2048 + (dim >> 3) * 128 + (dim & 7) * 16,
+                    for (int nt = 0; nt < 4; ++nt)
+                        st_shared_b32(base + nt * 2048 + (dim >> 3) * 128 + (dim & 7) * 16,
                                       pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]));
+                }
+        };
+        // Registers of the coming chunk: w fragments (A of w h: tokens 16p.., all
+        // 128 state rows), K^T fragments (A of the update: state rows 32p.., 64
+        // tokens), u at this thread's (token, column) pairs.
+        uint32_t wa[8][4], ka[4][2][4];
+        float2 uu[2][4];
+        auto load_chunk_regs = [&](int j) {
+            const uint32_t st = sb + kC0 + (j % kStages) * kCStageBytes;
+            const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const int d0 = 16 * ks + (lane >> 4) * 8;
+                ldsm_x4(wa[ks], st + kW + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
+            }
+            // u tile: 32 fp32 per row, 16-byte chunks XOR (row % 8)
+            const float *ut = reinterpret_cast<const float *>(smem + kC0 + (j % kStages) * kCStageBytes + kU);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int tok = 16 * p + g + half * 8;
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int col = 8 * nt + 2 * c4;
+                    uu[half][nt] = *reinterpret_cast<const float2 *>(ut + tok * 32 + (((col >> 2) ^ (tok & 7)) << 2) + (col & 3));
+                }
+            }
+        };
+        auto load_chunk_ka = [&](int j) {
+            // K^T rows (state rows) 32p+16mt.., cols (tokens) 16ks..: 8x8 blocks of the
+            // token-major, 128-byte-swizzled k tile read transposed
+            const uint32_t kt = sb + kC0 + (j % kStages) * kCStageBytes + kK;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
+                    const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
+                    ldsm_x4_t(ka[ks][mt], kt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
                 }
         };
         write_hb(0);
         fence_proxy_async();
-        bool ok = chain_sync(true);
-        if (tid == 0) publish(&ctr[kH], 1);  // h_0
-        // gates of the current chunk, prefetched one chunk ahead
+        bool ok = true;
+        if (nch > 0) {
+            ok = wait_bar(&sm->cfull[0], 0, abort_flag);
+            if (ok) {
+                load_chunk_regs(0);
+                load_chunk_ka(0);
+            }
+        }
+        ok = chain_sync(ok);
+        if (tid == 0) {
+            sm->cl_landed = nch > 0 ? 1 : 0;
+            publish(&ctr[kChain], 1);  // h_0; chunk 0's stage is in registers
+        }
+        // gates of the current chunk and of the next, prefetched ahead
         float gl = 0.f, gt0 = 0.f, gt1 = 0.f;
         if (nch > 0) gl = gamma_at(0, 63), gt0 = gamma_at(0, 16 * p + g), gt1 = gamma_at(0, 16 * p + g + 8);
 
         for (int j = 0; j < nch && ok; ++j) {
             const int len = min(kChunk, sr.len - j * kChunk);
-            const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
-            ok = chain_sync(wait_bar(&sm->full[j % kStages], (j / kStages) & 1, abort_flag));
-            if (!ok) break;
-            if (tid == 0) sm->loads_landed = j + 1;
             const float gC = gl, gtok[2] = {gt0, gt1};
             if (j + 1 < nch) gl = gamma_at(j + 1, 63), gt0 = gamma_at(j + 1, 16 * p + g), gt1 = gamma_at(j + 1, 16 * p + g + 8);
-            // ---- w h : tokens 16p..16p+15, columns of n-tiles cb, cb+1 (A = w tile, B = h)
-            float acc[2][4] = {};
+            // ---- w h : tokens 16p..16p+15, all 32 columns (A = w fragments, B = h from kHb)
+            float acc[4][4] = {};
             {
-                // all of this warp's w fragments up front (they do not depend on h),
-                // the h fragments streamed three k-steps ahead
-                const uint32_t wt = st + kW;
                 const uint32_t hb = sb + kHb + (j & 1) * 8192;
-                const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int mi = lane >> 3;
-                uint32_t a[8][4], b[4][4];
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int d0 = 16 * ks + (lane >> 4) * 8;
-                    ldsm_x4(a[ks], wt + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
-                }
+                uint32_t b[3][2][4];
                 auto load_b = [&](int ks) {
-                    ldsm_x4_t(b[ks & 3], hb + (cb + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
+#pragma unroll
+                    for (int np = 0; np < 2; ++np)
+                        ldsm_x4_t(b[ks % 3][np], hb + (2 * np + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
                 };
                 load_b(0);
                 load_b(1);
-                load_b(2);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    if (ks + 3 < 8) load_b(ks + 3);
-                    hmma(acc[0], a[ks], b[ks & 3][0], b[ks & 3][1]);
-                    hmma(acc[1], a[ks], b[ks & 3][2], b[ks & 3][3]);
+                    if (ks + 2 < 8) load_b(ks + 2);
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        hmma(acc[2 * np], wa[ks], b[ks % 3][np][0], b[ks % 3][np][1]);
+                        hmma(acc[2 * np + 1], wa[ks], b[ks % 3][np][2], b[ks % 3][np][3]);
+                    }
                 }
             }
-            // K^T fragments of the state update (independent of the chain): issued now so that
-            // their latency overlaps the Delta step. A = K^T rows (state rows) 32p+16mt..,
-            // cols (tokens) 16ks..: 8x8 blocks of the token-major, 128-byte-swizzled k tile
-            // read transposed.
-            uint32_t ka[4][2][4];
-            {
-                const uint32_t kt = st + kK;
-                const int mi = lane >> 3;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
-                        const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
-                        ldsm_x4_t(ka[ks][mt], kt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
-                    }
-            }
-            // ---- Delta = u - w h -> Db[j%2] (read by DP) ; e^{gamma_C - gamma} Delta -> Dt
-            // DP and the state store of chunk j-2 read Db[j%2]
-            ok = chain_sync(j < 2 || ((!want_o || wait_ge(&ctr[kODone], j - 1, abort_flag)) &&
-                                      (!states || wait_ge(&ctr[kStored], j - 1, abort_flag))));
-            if (!ok) break;
+            // ---- Delta = u - w h -> Db[j%2] (read by DP and the state store) ; e^{gamma_C - gamma} Delta -> Dt
             {
                 const uint32_t db = sb + kDb + (j & 1) * 4096 + c4 * 4, dt = sb + kDt + c4 * 4;
-                const float *ut = reinterpret_cast<const float *>(smem + kStage0 + (j % kStages) * kStageBytes + kU);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int tok = 16 * p + g + half * 8;
@@ -278,57 +317,55 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     const float sc = __expf(gC - gtok[half]);
                     const uint32_t off = (tok >> 3) * 128 + (tok & 7) * 16;
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int col = 8 * (cb + nt) + 2 * c4;  // u tile: 32 fp32 per row, 16-B chunks XOR (row % 8)
-                        const float2 uu = *reinterpret_cast<const float2 *>(
-                            ut + tok * 32 + ((((col >> 2) ^ (tok & 7))) << 2) + (col & 3));
-                        const float x0 = live ? uu.x - acc[nt][2 * half] : 0.f;
-                        const float x1 = live ? uu.y - acc[nt][2 * half + 1] : 0.f;
-                        st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(x0, x1));
-                        st_shared_b32(dt + (cb + nt) * 1024 + off, pack_bf16(sc * x0, sc * x1));
-                        if (states && len < kChunk && live)  // ragged last chunk: no TMA store past its end
-                            *reinterpret_cast<uint32_t *>(prm.delta + ((size_t)(sr.start + j * kChunk + tok) * d.Hv + h) * V +
-                                                          c0 + col) = pack_bf16(x0, x1);
+                    for (int nt = 0; nt < 4; ++nt) {
+                        const float x0 = live ? uu[half][nt].x - acc[nt][2 * half] : 0.f;
+                        const float x1 = live ? uu[half][nt].y - acc[nt][2 * half + 1] : 0.f;
+                        st_shared_b32(db + nt * 1024 + off, pack_bf16(x0, x1));
+                        st_shared_b32(dt + nt * 1024 + off, pack_bf16(sc * x0, sc * x1));
                     }
                 }
             }
-            chain_sync(true);  // every warp reads all 64 tokens of Dt below
-            // ---- h <- e^{gamma_C} h + K^T Dt : rows 32p..32p+31, 16 columns, K = 64 tokens
+            // every warp reads all 64 tokens of Dt below; the stage of chunk j+1 has landed;
+            // kHb[(j+1)%2] (written below) and kDb[(j+1)%2] (written in chunk j+1) are free once
+            // the outputs and state stores of chunk j-1 are done
+            ok = chain_sync((j + 1 >= nch || wait_bar(&sm->cfull[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort_flag)) &&
+                            (tid != 0 || ((!want_o || wait_ge(&ctr[kODone], j, abort_flag)) &&
+                                          (!states || wait_ge(&ctr[kStored], j, abort_flag)))));
+            if (!ok) break;
+            // ---- h <- e^{gamma_C} h + K^T Dt : rows 32p..32p+31, 32 columns, K = 64 tokens
             {
+                uint32_t bt[4][2][4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                    for (int np = 0; np < 2; ++np)
+                        ldsm_x4_t(bt[ks][np], sb + kDt + (2 * np + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
+                if (j + 1 < nch) load_chunk_regs(j + 1);  // w, u of the next chunk (w fragments are dead)
                 const float eC = __expf(gC);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                         for (int q = 0; q < 4; ++q) hf[mt][nt][q] *= eC;
-                const int mi = lane >> 3;
-                uint32_t b[4][4];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    ldsm_x4_t(b[ks], sb + kDt + (cb + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        hmma(hf[mt][0], ka[ks][mt], b[ks][0], b[ks][1]);
-                        hmma(hf[mt][1], ka[ks][mt], b[ks][2], b[ks][3]);
-                    }
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int np = 0; np < 2; ++np) {
+                            hmma(hf[mt][2 * np], ka[ks][mt], bt[ks][np][0], bt[ks][np][1]);
+                            hmma(hf[mt][2 * np + 1], ka[ks][mt], bt[ks][np][2], bt[ks][np][3]);
+                        }
+                if (j + 1 < nch) load_chunk_ka(j + 1);  // after the products that read these registers
             }
-            chain_sync(true);
-            if (tid == 0) publish(&ctr[kStage], j + 1);
-            // ---- h_{j+1} -> Hb[(j+1)%2] once DQ of chunk j-1 (which read it) is done; then
-            //      Delta_j and h_{j+1} go to the output MMAs behind one proxy fence
-            // DQ and the state store of chunk j-1 read Hb[(j+1)%2]
-            ok = chain_sync(j < 1 || ((!want_o || wait_ge(&ctr[kODone], j, abort_flag)) &&
-                                      (!states || wait_ge(&ctr[kStored], j, abort_flag))));
-            if (!ok) break;
+            // ---- h_{j+1} -> Hb[(j+1)%2]; Delta_j and h_{j+1} go to the output MMAs behind one proxy fence
             write_hb((j + 1) & 1);
             fence_proxy_async();
             chain_sync(true);
             if (tid == 0) {
-                publish(&ctr[kDelta], j + 1);
-                publish(&ctr[kH], j + 2);
+                sm->cl_landed = j + 2 < nch ? j + 2 : nch;
+                publish(&ctr[kChain], j + 2);
             }
         }
         if (!ok) {
@@ -349,16 +386,16 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
                             const int dim = 32 * p + 16 * mt + g + half * 8;
-                            *reinterpret_cast<float2 *>(dst + (size_t)dim * ld + 8 * (cb + nt) + 2 * c4) =
+                            *reinterpret_cast<float2 *>(dst + (size_t)dim * ld + 8 * nt + 2 * c4) =
                                 make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
                         }
             }
         }
-    } else if (warp < 12) {
+    } else if (warp < 8) {
         // ======================================================== epilogue
         if (want_o) {
             const int et = tid - kRole, q = warp & 3;  // TMEM lanes 32q.. = rows 16q..16q+15
@@ -404,72 +441,66 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 *abort_flag = 1;
             }
         }
-    } else {
-        // ========================================================== issuer
-        if (lane == 0) {
+    } else if (warp == 8) {
+        // =================================================== output issuer
+        if (lane == 0 && (want_o || states)) {
             bool ok = true;
-            auto issue_loads = [&](int j) {
+            auto issue_out_loads = [&](int j) {
                 const int s = j % kStages;
-                uint8_t *stg = smem + kStage0 + s * kStageBytes;
+                uint8_t *stg = smem + kO0 + s * kOStageBytes;
                 const int t0 = sr.start + j * kChunk;
                 const int cg = sr.chunk0 + j;
-                mbar_arrive_expect_tx(&sm->full[s], want_o ? kTxFull : kTxChain);
-                atomicAdd(&sm->loads_issued, 1);
-                if (want_o) {
-                    tma_load_3d(stg + kQ, &tm_q, &sm->full[s], 0, hq, t0);
-                    tma_load_3d(stg + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
-                    tma_load_2d(stg + kP, &tm_p, &sm->full[s], 0, (cg * d.Hv + h) * kChunk);
-                }
-                tma_load_3d(stg + kK, &tm_k, &sm->full[s], 0, hq, t0);
-                tma_load_3d(stg + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
-                tma_load_3d(stg + kW, &tm_w, &sm->full[s], 0, h, t0);
-                tma_load_3d(stg + kW + 8192, &tm_w, &sm->full[s], 64, h, t0);
-                tma_load_3d(stg + kU, &tm_u, &sm->full[s], c0, h, t0);  // out of range (zero) for operator columns
+                mbar_arrive_expect_tx(&sm->ofull[s], kOStageBytes);
+                ++sm->ol_issued;
+                tma_load_3d(stg + kQ, &tm_q, &sm->ofull[s], 0, hq, t0);
+                tma_load_3d(stg + kQ + 8192, &tm_q, &sm->ofull[s], 64, hq, t0);
+                tma_load_2d(stg + kP, &tm_p, &sm->ofull[s], 0, (cg * d.Hv + h) * kChunk);
             };
-            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
+            if (want_o)
+                for (int c = 0; c < kStages && c < nch; ++c) issue_out_loads(c);
             const uint32_t id_O = idesc_bf16(64, 32, false, true);
             for (int j = 0; j < nch && ok; ++j) {
-                // refill the stage of chunk j-1 with chunk j+2 once the chain and DQ/DP are done with it
-                if (j >= 1 && j + 2 < nch) {
-                    ok = wait_ge(&ctr[kStage], j, abort_flag) && (!want_o || wait_ge(&ctr[kODone], j, abort_flag));
-                    if (!ok) break;
-                    issue_loads(j + 2);
-                }
-                if (!want_o && !states) continue;
                 // h_j and Delta_j are in kHb[j%2], kDb[j%2]
-                ok = wait_ge(&ctr[kH], j + 1, abort_flag) && wait_ge(&ctr[kDelta], j + 1, abort_flag);
+                ok = wait_ge(&ctr[kChain], j + 2, abort_flag);
                 if (!ok) break;
+                const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
+                if (want_o) {
+                    // DQ = Q h_j, DP = P Delta_j into buffer j%2 once q, P have landed and the
+                    // epilogue has read chunk j-2's accumulators
+                    ok = wait_bar(&sm->ofull[j % kStages], (j / kStages) & 1, abort_flag) &&
+                         wait_ge(&ctr[kTmemO], j >= 1 ? j - 1 : 0, abort_flag);
+                    if (!ok) break;
+                    sm->ol_landed = j + 1;
+                    tc_fence_after();
+                    const uint32_t st = sb + kO0 + (j % kStages) * kOStageBytes;
+                    const uint32_t tb = tmem + (j & 1) * kOBuf;
+                    const uint64_t qd = smem_desc(st + kQ, 16, 1024, kSw128), hd = smem_desc(hb, 128, 2048, kSwNone);
+                    const uint64_t pd = smem_desc(st + kP, 16, 1024, kSw128), dd = smem_desc(db, 128, 1024, kSwNone);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(tb + kColQ, qd + (uint64_t)((((ks >> 2) * 8192 + (ks & 3) * 32)) >> 4),
+                                 hd + (uint64_t)(ks * 256 >> 4), id_O, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tb + kColP, pd + (uint64_t)(ks * 32 >> 4), dd + (uint64_t)(ks * 256 >> 4), id_O, ks > 0);
+                    mma_commit(&sm->mmaO[j & 1]);
+                    sm->mma_issued = j + 1;
+                }
                 if (states) {
-                    // entry state (four 8-column boxes of 128 rows) and, for a full chunk, Delta
-                    const int len = min(kChunk, sr.len - j * kChunk);
-                    const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
-                    const int row = ((sr.chunk0 + j) * d.Hv + h) * K;
-                    for (int nb = 0; nb < 4; ++nb) {
-                        tma_store_2d(&tm_hs, hb + nb * 2048, c0 + 8 * nb, row);
-                        if (len == kChunk) tma_store_3d(&tm_ds, db + nb * 1024, c0 + 8 * nb, h, sr.start + j * kChunk);
-                    }
+                    // entry state and Delta: one block each per (chunk, head, column slice)
+                    const size_t blk = ((size_t)(sr.chunk0 + j) * d.Hv + h) * (V / kBV) + blockIdx.z;
+                    bulk_store(prm.h_chunks + blk * (K * kBV), hb, K * kBV * 2);
+                    bulk_store(prm.delta + blk * (kChunk * kBV), db, kChunk * kBV * 2);
                     bulk_commit();
                     bulk_wait_read<0>();
                     publish(&ctr[kStored], j + 1);
                 }
-                if (!want_o) continue;
-                // DQ = Q h_j, DP = P Delta_j into buffer j%2 once the epilogue has read chunk j-2's
-                ok = wait_ge(&ctr[kTmemO], j >= 1 ? j - 1 : 0, abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t st = sb + kStage0 + (j % kStages) * kStageBytes;
-                const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
-                const uint32_t tb = tmem + (j & 1) * kOBuf;
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t aoff = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_bf16(tb + kColQ, smem_desc(st + kQ + aoff, 16, 1024, kSw128),
-                             smem_desc(hb + ks * 256, 128, 2048, kSwNone), id_O, ks > 0);
+                // the (q, P) stage of chunk j-1 is free once its products are complete: chunk j+2
+                if (want_o && j >= 1 && j + 2 < nch) {
+                    ok = wait_ge(&ctr[kODone], j, abort_flag);
+                    if (!ok) break;
+                    issue_out_loads(j + 2);
                 }
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tb + kColP, smem_desc(st + kP + ks * 32, 16, 1024, kSw128),
-                             smem_desc(db + ks * 256, 128, 1024, kSwNone), id_O, ks > 0);
-                mma_commit(&sm->mmaO[j & 1]);
-                sm->mma_issued = j + 1;
             }
             if (!ok) {
                 set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -478,22 +509,52 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             bulk_wait_all();  // state stores complete before the CTA's shared memory goes away
         }
         __syncwarp();
+    } else {
+        // =================================================== chain producer
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                // stage c%3 held chunk c-3, which the chain has in registers once kChain >= c-2
+                if (c >= kStages) {
+                    ok = wait_ge(&ctr[kChain], c - kStages + 1, abort_flag);
+                    if (!ok) break;
+                }
+                const int s = c % kStages;
+                uint8_t *stg = smem + kC0 + s * kCStageBytes;
+                const int t0 = sr.start + c * kChunk;
+                mbar_arrive_expect_tx(&sm->cfull[s], kCStageBytes);
+                ++sm->cl_issued;
+                tma_load_3d(stg + kK, &tm_k, &sm->cfull[s], 0, hq, t0);
+                tma_load_3d(stg + kK + 8192, &tm_k, &sm->cfull[s], 64, hq, t0);
+                tma_load_3d(stg + kW, &tm_w, &sm->cfull[s], 0, h, t0);
+                tma_load_3d(stg + kW + 8192, &tm_w, &sm->cfull[s], 64, h, t0);
+                tma_load_3d(stg + kU, &tm_u, &sm->cfull[s], c0, h, t0);  // out of range (zero) for operator columns
+            }
+            if (!ok) {
+                set_status(prm.status, GDN_ERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+        }
+        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) {
-        // let every TMA load still in flight land (bounded) before the CTA exits
+        // let every TMA load and output MMA still in flight finish (bounded) before the CTA exits
         const uint64_t t0 = globaltimer();
-        for (int c = sm->loads_landed; c < sm->loads_issued; ++c)
-            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
+        for (int c = sm->cl_landed; c < sm->cl_issued; ++c)
+            while (!mbar_try_wait(smem_u32(&sm->cfull[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
             }
-        for (int c = sm->mma_seen; c < sm->mma_issued; ++c)  // and every output MMA
+        for (int c = sm->ol_landed; c < sm->ol_issued; ++c)
+            while (!mbar_try_wait(smem_u32(&sm->ofull[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
+            }
+        for (int c = sm->mma_seen; c < sm->mma_issued; ++c)
             while (!mbar_try_wait(smem_u32(&sm->mmaO[c & 1]), (c >> 1) & 1) && globaltimer() - t0 < kWaitNs) {
             }
     }
     __syncthreads();
-    if (warp == 12) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -515,7 +576,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || (a.o && !a.p16)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mw, mu, mp, mhs, mds;
+    CUtensorMap mq, mk, mw, mu, mp;
     const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
     const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
@@ -533,18 +594,8 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
         !make_map(&mw, BF, a.w16, 3, dw, sw, b64) || !make_map(&mu, F32, a.u32, 3, du, su, bu) ||
         !make_map(&mp, BF, a.p16 ? a.p16 : a.w16, 2, dp, sp, bp))
         return cudaErrorInvalidValue;
-    // state stores: entry states as [NC * Hv * K rows][V], Delta as [T][Hv][V]; 16-byte boxes
-    const bool st = a.h_chunks16 != nullptr;
-    if (st != (a.delta16 != nullptr)) return cudaErrorInvalidValue;
-    const cuuint64_t dhs[2] = {(cuuint64_t)d.V, (cuuint64_t)(d.NC > 0 ? d.NC : 1) * d.Hv * d.K};
-    const cuuint64_t shs[1] = {(cuuint64_t)d.V * 2};
-    const cuuint32_t bhs[2] = {8, 128};
-    const cuuint64_t dds[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
-    const cuuint64_t sds[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
-    const cuuint32_t bds[3] = {8, 1, 64};
-    if (!make_map(&mhs, BF, st ? a.h_chunks16 : a.w16, 2, dhs, shs, bhs, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mds, BF, st ? a.delta16 : a.w16, 3, dds, sds, bds, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    // chunk entry states and Delta: both or neither
+    if ((a.h_chunks16 != nullptr) != (a.delta16 != nullptr)) return cudaErrorInvalidValue;
     Fwd2Params p;
     p.d = d;
     p.gamma = a.gamma;
@@ -566,7 +617,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
     dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
-    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, mhs, mds, p);
+    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, p);
     return cudaGetLastError();
 }
 

@@ -53,6 +53,8 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *ctr) {
 }
 
 // Bounded wait until *ctr >= need; false if it expired or the CTA is aborting.
+// Within a warp role one thread polls, and a named barrier passes the result on
+// (role_sync_and): every poll is a shared-memory load.
 __device__ __forceinline__ bool wait_ge(const uint32_t *ctr, uint32_t need, volatile int *abort_flag) {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {

@@ -96,10 +96,13 @@ size_t gdn_bwd_workspace_size(const gdn_problem *p);
  * tensor-core backward needs from the forward: w = Ainv diag(beta e^gamma) K
  * (bf16 [B*T, Hv, K]), u = Ainv diag(beta) V (fp32 [B*T, Hv, V]), the
  * decay-masked P = M o Q K^T of every chunk (bf16 [num_chunks, Hv, 64, 64]),
- * and every chunk's entry state (bf16 [num_chunks, Hv, K, V]) and Delta (bf16
- * [B*T, Hv, V]) -- the per-chunk states h that page 1's low-level forward also
- * returns -- so that a backward given `saved` runs neither the chunk prep nor
- * a recompute of the states. Each part 256-byte aligned. */
+ * and every chunk's entry state (bf16, num_chunks * Hv * K * V elements) and
+ * Delta (bf16, num_chunks * 64 * Hv * V elements) -- the per-chunk states h
+ * that page 1's low-level forward also returns -- so that a backward given
+ * `saved` runs neither the chunk prep nor a recompute of the states. The
+ * states and Delta are stored in a blocked layout private to this library
+ * (one block per chunk, value head and 32-column slice). Each part 256-byte
+ * aligned. */
 size_t gdn_saved_size(const gdn_problem *p);
 
 /* Forward. h0 may be NULL (zero initial state); final_state may be NULL (not

@@ -52,9 +52,10 @@ def prob(B_=1, T=256, Hq=2, Hv=4, K=128, V=128, ns=0, cu=None, dtype=1, scale=0.
 
 
 def saved_bf16_k128(ntok, nc, Hv=4, K=128, V=128):
-    # gamma | Ainv | w | u | P | chunk entry states | Delta (include/gdn.h)
+    # gamma | Ainv | w | u | P | chunk entry states | Delta, the last two per chunk
+    # (include/gdn.h)
     return (ntok * Hv * 4 + nc * Hv * 64 * 64 * 2 + ntok * Hv * K * 2 + ntok * Hv * V * 4
-            + nc * Hv * 64 * 64 * 2 + nc * Hv * K * V * 2 + ntok * Hv * V * 2)
+            + nc * Hv * 64 * 64 * 2 + nc * Hv * K * V * 2 + nc * 64 * Hv * V * 2)
 
 
 def test_workspace_sizes(L):
