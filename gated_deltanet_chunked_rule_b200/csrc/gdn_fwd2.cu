@@ -29,10 +29,12 @@
 //               shared memory. Two barriers per chunk.
 //   warps 4-7   epilogue: o from the double-buffered DQ/DP accumulators;
 //               warp 4 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15).
-//   warp 8      output issuer: the DQ/DP MMAs, the (q, P) TMA ring, and the
-//               bulk copies of the chunk states and Delta to global memory.
+//   warp 8      output issuer: the DQ/DP MMAs and the (q, P) TMA ring.
 //   warp 9      chain producer: the (k, w, u) TMA ring, refilled as soon as the
-//               chain has a stage in registers.
+//               chain has a stage in registers, and the bulk copies of the
+//               chunk states and Delta to global memory (in parallel with the
+//               output products, since the chain reuses kHb / kDb once both
+//               are done).
 // Roles hand over through monotonically increasing shared-memory counters
 // (release/acquire; one thread polls, a barrier passes it on), which cannot
 // alias the way mbarrier parities can when a producer runs ahead; mbarriers
@@ -443,7 +445,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
     } else if (warp == 8) {
         // =================================================== output issuer
-        if (lane == 0 && (want_o || states)) {
+        if (lane == 0 && want_o) {
             bool ok = true;
             auto issue_out_loads = [&](int j) {
                 const int s = j % kStages;
@@ -464,7 +466,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 ok = wait_ge(&ctr[kChain], j + 2, abort_flag);
                 if (!ok) break;
                 const uint32_t hb = sb + kHb + (j & 1) * 8192, db = sb + kDb + (j & 1) * 4096;
-                if (want_o) {
+                {
                     // DQ = Q h_j, DP = P Delta_j into buffer j%2 once q, P have landed and the
                     // epilogue has read chunk j-2's accumulators
                     ok = wait_bar(&sm->ofull[j % kStages], (j / kStages) & 1, abort_flag) &&
@@ -486,15 +488,6 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     mma_commit(&sm->mmaO[j & 1]);
                     sm->mma_issued = j + 1;
                 }
-                if (states) {
-                    // entry state and Delta: one block each per (chunk, head, column slice)
-                    const size_t blk = ((size_t)(sr.chunk0 + j) * d.Hv + h) * (V / kBV) + blockIdx.z;
-                    bulk_store(prm.h_chunks + blk * (K * kBV), hb, K * kBV * 2);
-                    bulk_store(prm.delta + blk * (kChunk * kBV), db, kChunk * kBV * 2);
-                    bulk_commit();
-                    bulk_wait_read<0>();
-                    publish(&ctr[kStored], j + 1);
-                }
                 // the (q, P) stage of chunk j-1 is free once its products are complete: chunk j+2
                 if (want_o && j >= 1 && j + 2 < nch) {
                     ok = wait_ge(&ctr[kODone], j, abort_flag);
@@ -506,19 +499,13 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 set_status(prm.status, GDN_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
-            bulk_wait_all();  // state stores complete before the CTA's shared memory goes away
         }
         __syncwarp();
     } else {
         // =================================================== chain producer
         if (lane == 0) {
             bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
-                // stage c%3 held chunk c-3, which the chain has in registers once kChain >= c-2
-                if (c >= kStages) {
-                    ok = wait_ge(&ctr[kChain], c - kStages + 1, abort_flag);
-                    if (!ok) break;
-                }
+            auto issue_chain_loads = [&](int c) {
                 const int s = c % kStages;
                 uint8_t *stg = smem + kC0 + s * kCStageBytes;
                 const int t0 = sr.start + c * kChunk;
@@ -529,11 +516,34 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 tma_load_3d(stg + kW, &tm_w, &sm->cfull[s], 0, h, t0);
                 tma_load_3d(stg + kW + 8192, &tm_w, &sm->cfull[s], 64, h, t0);
                 tma_load_3d(stg + kU, &tm_u, &sm->cfull[s], c0, h, t0);  // out of range (zero) for operator columns
+            };
+            for (int c = 0; c < kStages && c < nch; ++c) issue_chain_loads(c);
+            // chunk 3 into stage 0 once the chain has chunk 0 in registers (kChain >= 1)
+            if (kStages < nch) {
+                ok = wait_ge(&ctr[kChain], 1, abort_flag);
+                if (ok) issue_chain_loads(kStages);
+            }
+            for (int j = 0; j < nch && ok; ++j) {
+                // chunk j done (kChain >= j+2): its entry state and Delta out of kHb[j%2], kDb[j%2];
+                // chunk j+1's stage is in registers, so stage (j+1)%3 takes chunk j+4
+                ok = wait_ge(&ctr[kChain], j + 2, abort_flag);
+                if (!ok) break;
+                if (j + 1 + kStages < nch) issue_chain_loads(j + 1 + kStages);
+                if (states) {
+                    // one block each per (chunk, head, column slice)
+                    const size_t blk = ((size_t)(sr.chunk0 + j) * d.Hv + h) * (V / kBV) + blockIdx.z;
+                    bulk_store(prm.h_chunks + blk * (K * kBV), sb + kHb + (j & 1) * 8192, K * kBV * 2);
+                    bulk_store(prm.delta + blk * (kChunk * kBV), sb + kDb + (j & 1) * 4096, kChunk * kBV * 2);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                    publish(&ctr[kStored], j + 1);
+                }
             }
             if (!ok) {
                 set_status(prm.status, GDN_ERR_TIMEOUT);
                 *abort_flag = 1;
             }
+            bulk_wait_all();  // state copies complete before the CTA's shared memory goes away
         }
         __syncwarp();
     }

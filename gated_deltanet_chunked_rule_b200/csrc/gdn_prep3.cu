@@ -14,7 +14,9 @@
 //   Ainv  (bf16 [NC, Hv, 64, 64], for the backward; optional)
 //
 // (the WY form of the chunk: Delta = u - w h, o = scale (diag(e^gamma) Q h + P Delta).)
-// The four bulk products (S, G, u, w) run on tcgen05 from TMA-loaded,
+// P, u and w of a full chunk are written by TMA stores from swizzled staging
+// tiles (row by row for a ragged one, whose tile would spill into the next
+// sequence). The four bulk products (S, G, u, w) run on tcgen05 from TMA-loaded,
 // 128-byte-swizzled tiles, so their operands never pass through the
 // load/store unit, which the warp-level version of this kernel saturated.
 // The unit lower-triangular inverse is taken block-wise on 16 x 16 blocks in
@@ -49,7 +51,14 @@ constexpr int kX = kA + 64 * kLd * 4;
 constexpr int kT = kX + 64 * kLd * 4;      // float [3][16][17]: one 16 x 16 block product per warp
 constexpr int kVec = kT + 3 * 16 * 17 * 4;
 constexpr int kBar = kVec + 1024;
-constexpr int kSmemBytes = kBar + 64 + 1024;
+constexpr int kPs = 89088;      // P staging for its TMA store: [64][64] bf16, 128-byte swizzle
+constexpr int kSmemBytes = kPs + 8192 + 1024;
+static_assert(kBar + 64 <= kPs && kPs % 1024 == 0, "shared memory layout");
+// u and w of a full chunk leave through TMA stores from 128-byte-swizzled staging
+// tiles over buffers that are free once the u, w products are complete: u (fp32,
+// four [64][32] tiles) over A and X, w (bf16, two [64][64] halves) over Au, Aw.
+constexpr int kUs = kA, kWs = kAu;
+static_assert(kUs % 1024 == 0 && kUs + 32768 <= kT && kWs + 16384 <= kA, "staging layout");
 static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
 
 // tensor memory: S | G (64 columns each), later u | w (128 columns each)
@@ -90,7 +99,9 @@ struct Prep3Params {
 
 __global__ void __launch_bounds__(kThreads, 2)
 prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const Prep3Params prm) {
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_uo,
+             const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_po,
+             const Prep3Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -212,11 +223,11 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             egam[tid] = __expf(gl);
             if (tid < len) prm.gamma_out[(size_t)(t0 + tid) * d.Hv + h] = gl;
         }
+        if (tid == 0) bulk_wait_read<0>();  // the previous head's P, u, w stores have read their staging
         __syncthreads();
         // ---- A (strictly lower), X = 0, and P = M o S -> global
         {
             const float gr[2] = {gam[r0], gam[r1]}, br[2] = {bet[r0], bet[r1]};
-            __nv_bfloat16 *pout = prm.p_out + ((size_t)cg * d.Hv + h) * C * C;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int s = 32 * wn + 8 * j + 2 * c4;
@@ -230,12 +241,17 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                         make_float2(s < r ? br[hi] * e0 * gacc[j][2 * hi] : 0.f, s + 1 < r ? br[hi] * e1 * gacc[j][2 * hi + 1] : 0.f);
                     *reinterpret_cast<float2 *>(&X[r][s]) = make_float2(0.f, 0.f);
                     const bool live = r < len;
-                    *reinterpret_cast<uint32_t *>(pout + r * C + s) =
-                        pack_bf16(live ? e0 * sacc[j][2 * hi] : 0.f, live ? e1 * sacc[j][2 * hi + 1] : 0.f);
+                    st_shared_b32(sb + kPs + r * 128 + (((s >> 3) ^ (r & 7)) << 4) + (s & 7) * 2,
+                                  pack_bf16(live ? e0 * sacc[j][2 * hi] : 0.f, live ? e1 * sacc[j][2 * hi + 1] : 0.f));
                 }
             }
         }
+        fence_proxy_async();  // P -> its TMA store
         __syncthreads();
+        if (tid == 0) {
+            tma_store_2d(&tm_po, sb + kPs, 0, (cg * d.Hv + h) * C);
+            bulk_commit();
+        }
         // ---- diagonal 16 x 16 blocks: thread t -> block t / 16, column t % 16
         if (tid < 64) {
             const int b = tid >> 4, cc = tid & 15, o = b * 16;
@@ -337,6 +353,7 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (ok) ++mma_phase, mma_pending = false;
         tc_fence_after();
         if (ok && tid == 0 && gi + 1 < G) load_v(h + 1);  // the v tile is free again
+        const bool full = len == C;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // columns 64 wn + 32 part .. +31, 16 values at a time
             float v[16];
@@ -345,27 +362,40 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int col = cb + 8 * i + 2 * c4;
-                if (r0 < len)
-                    *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r0) * d.Hv + h) * V + col) =
-                        make_float2(v[4 * i], v[4 * i + 1]);
-                if (r1 < len)
-                    *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r1) * d.Hv + h) * V + col) =
-                        make_float2(v[4 * i + 2], v[4 * i + 3]);
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = hi ? r1 : r0;
+                    const float2 x = make_float2(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
+                    if (full)  // [64][32] fp32 tile per 32 columns: 16-byte chunks XOR (row % 8)
+                        st_shared_v2f(sb + kUs + (col >> 5) * 8192 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) + (col & 3) * 4, x.x, x.y);
+                    else if (r < len)
+                        *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r) * d.Hv + h) * V + col) = x;
+                }
             }
             tmem_ld16x256_x4(tmem + lane_base + kColW + cb, v);  // w
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int col = cb + 8 * i + 2 * c4;
-                if (r0 < len)
-                    *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r0) * d.Hv + h) * K + col) =
-                        pack_bf16(v[4 * i], v[4 * i + 1]);
-                if (r1 < len)
-                    *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r1) * d.Hv + h) * K + col) =
-                        pack_bf16(v[4 * i + 2], v[4 * i + 3]);
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = hi ? r1 : r0;
+                    const uint32_t x = pack_bf16(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
+                    if (full)
+                        st_shared_b32(sb + kWs + (col >> 6) * 8192 + r * 128 + ((((col & 63) >> 3) ^ (r & 7)) << 4) + (col & 7) * 2, x);
+                    else if (r < len)
+                        *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r) * d.Hv + h) * K + col) = x;
+                }
             }
         }
+        fence_proxy_async();  // u, w -> their TMA stores
         tc_fence_before();
-        __syncthreads();  // u, w columns, Au, Aw, A, X free for the next value head
+        __syncthreads();  // u, w columns free for the next value head (Au, Aw, A, X once the stores have read them)
+        if (full && tid == 0) {
+            for (int c = 0; c < 4; ++c) tma_store_3d(&tm_uo, sb + kUs + c * 8192, 32 * c, h, t0);
+            tma_store_3d(&tm_wo, sb + kWs, 0, h, t0);
+            tma_store_3d(&tm_wo, sb + kWs + 8192, 64, h, t0);
+            bulk_commit();
+        }
     }
     if (!ok) {
         if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -378,6 +408,7 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
         }
     }
+    if (tid == 0) bulk_wait_all();  // the stores read shared memory until they complete
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -393,16 +424,31 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.NC == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || !a.p16 || !a.gamma) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, muo, mwo, mpo;
     const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
     const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
     const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
     const cuuint64_t sv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
     const cuuint32_t box[3] = {64, 1, 64};
-    if (!make_bf16_map(&mq, a.q, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    // stores: u fp32 [T, Hv, V] in 32-column boxes, w bf16 [T, Hv, K], P bf16 [NC * Hv * 64 rows][64]
+    const cuuint64_t du[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
+    const cuuint64_t su[2] = {(cuuint64_t)d.V * 4, (cuuint64_t)d.Hv * d.V * 4};
+    const cuuint32_t bu[3] = {32, 1, 64};
+    const cuuint64_t dw[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sw[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hv * d.K * 2};
+    const cuuint64_t dp[2] = {64, (cuuint64_t)d.NC * d.Hv * 64};
+    const cuuint64_t sp[1] = {128};
+    const cuuint32_t bp[2] = {64, 64};
+    auto enc = tensor_map_encoder();
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (!enc || !make_bf16_map(&mq, a.q, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_bf16_map(&mk, a.k, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_bf16_map(&mv, a.v, 3, dv, sv, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_bf16_map(&mv, a.v, 3, dv, sv, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        enc(&muo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.u32, du, su, bu, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        !make_bf16_map(&mwo, a.w16, 3, dw, sw, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_bf16_map(&mpo, a.p16, 2, dp, sp, bp, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     Prep3Params p;
     p.d = d;
@@ -416,7 +462,7 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(prep3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    prep3_kernel<<<dim3(d.NC, d.Hq), kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, p);
+    prep3_kernel<<<dim3(d.NC, d.Hq), kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, muo, mwo, mpo, p);
     return cudaGetLastError();
 }
 
