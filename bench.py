@@ -80,12 +80,14 @@ def kernel_bytes(name, w, saved=False):
       prep3            2K*e/G (q, k) + V*e (v) + 3*4 (g, beta, gamma) + K*2 (w) + V*4 (u) + C*2 (P)
                        [+ C*e Ainv when saved]
       fwd_hybrid       2K*e/G (q, k) + K*2 (w) + V*4 (u) + C*2 (P) + 4 (gamma) + V*e (o)
+                       [+ K*V*e/C (entry states) + V*e (Delta) when saved]
       bwd_recompute    K*e/G (k) + K*2 + V*4 + 4 + K*V*e/C (entry states) + V*e (Delta)
       bwd_dh           2K*e/G (q, k) + K*2 (w) + C*2 (P) + V*e (dO) + 4 + K*V*e/C (dh') + V*e (dDelta)
       bwd_grad         2K*e/G + 2V*e (v, dO) + 8 (gamma, beta) + C*e (Ainv) + 2K*V*e/C (h, dh')
-                       + 2V*e (Delta, dDelta) + 2K*4 (dq, dk partials) + V*e (dv) + 8 (dg, dbeta)
-      bwd_final        2K*4 (partials) + 2K*e/G (dq, dk)
+                       + 2V*e (Delta, dDelta) + 2K*e/G (dq, dk, summed over the group on chip)
+                       + V*e (dv) + 8 (dg, dbeta)
     plus the per-sequence states (h0, final, dht, dh0: K*V*4 each) where a kernel touches them.
+    Entry states and Delta are stored per chunk (64 rows, ragged ones padded).
     """
     C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
     ntok = w.B * w.T
@@ -99,8 +101,8 @@ def kernel_bytes(name, w, saved=False):
     st = N * Hv * K * V * 4
     h0 = st if w.h0_std is not None else 0
     hc = nc * Hv * K * V * 2
-    d16 = ntok * Hv * V * 2
-    part = ntok * Hv * K * 4
+    d16 = ntok * Hv * V * 2     # dDelta
+    dsb = nc * C * Hv * V * 2   # Delta, per chunk
     wb = ntok * Hv * K * 2      # w (bf16)
     ub = ntok * Hv * V * 4      # u (fp32)
     pb = nc * Hv * C * C * 2    # P (bf16)
@@ -111,12 +113,12 @@ def kernel_bytes(name, w, saved=False):
         "prep3": prep3 + (ainv if saved else 0),                # q,k,v,g,beta -> gamma,w,u,P[,Ainv]
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
         "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
-        "fwd_hybrid": 2 * qk1 + wb + ub + pb + gam + h0 + v1 + st,  # q,k,w,u,P,gamma,h0 -> o,final
+        # q,k,w,u,P,gamma,h0 -> o,final[,entry states,Delta]
+        "fwd_hybrid": 2 * qk1 + wb + ub + pb + gam + h0 + v1 + st + ((hc + dsb) if saved else 0),
         "bwd_prep3": prep3 + (0 if saved else ainv),
-        "bwd_recompute": qk1 + wb + ub + gam + h0 + hc + d16,
+        "bwd_recompute": qk1 + wb + ub + gam + h0 + hc + dsb,
         "bwd_dh": 2 * qk1 + wb + pb + v1 + gam + st + hc + d16 + st,
-        "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + 2 * d16 + 2 * part + v1 + 2 * gam,
-        "bwd_final": 2 * part + 2 * qk1,
+        "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + dsb + d16 + 2 * qk1 + v1 + 2 * gam,
     }
     return table.get(name)
 
@@ -126,18 +128,18 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=645888256 + 307320576,
-                     sources=["gdn_bwd_grad.cu"],
-                     sha256="7f74d3569aa5c14ce7c2e7a3f9055bc055fc8ae4206c046e9c8382433567aeb8"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072320 + 167649792,
-                   sources=["gdn_bwd_dh.cu"],
-                   sha256="dffa02f93180ece98e9e3ec45634479026cc213ef9376735daccfff066b3a7f8"),
-    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd", bytes=303084544 + 57421312,
-                       sources=["gdn_fwd2.cu"],
-                       sha256="ab1104a6ecb3bdf74902b31d96f0c64569529bf335816f6523efb0a37159c919"),
-    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd", bytes=138035200 + 187329280,
-                  sources=["gdn_prep3.cu"],
-                  sha256="c40c7df4f99dbc4efa75743e164771cbd04d313a0c62cb0c1ae93d5875554097"),
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639929856 + 120504832,
+               sources=["gdn_bwd_grad.cu"],
+               sha256="922fdf75f61c27e9dab6e1ea7008f872b557bf28f8a8c700706be7d3b5e9c12d"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238069760 + 167706112,
+               sources=["gdn_bwd_dh.cu"],
+               sha256="6b2bd9615693f6bca2bbd0362ec471e9fd7ed1e21451937dfa3c78da1b767843"),
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303091968 + 230028544,
+               sources=["gdn_fwd2.cu"],
+               sha256="129476ecaf0a7544e2532b67fd91152615ad381a1c0fe3c83fa7955aac1244ee"),
+    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=138346240 + 213746944,
+               sources=["gdn_prep3.cu"],
+               sha256="b5dd7e87c61c371614b692c11337e75c054daa97a1882d85b439c6cbf85f0945"),
 }
 TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
 
