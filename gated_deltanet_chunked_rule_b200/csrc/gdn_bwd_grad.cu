@@ -28,10 +28,10 @@
 //   1. S = QK^T, G = KK^T, P1 = dO Delta^T, dU = Ainv^T dDelta
 //   2. dAkk, T1 K, T1^T Q (onto dk), dO h^T
 //   3. dU h^T, Delta dh'^T, and dG K + dG^T K onto dk
-// The 8 warps read the accumulators back with the 16x256b TMEM load, whose
+// The 16 warps read the accumulators back with the 16x256b TMEM load, whose
 // register layout is the warp-MMA fragment layout (warp w: rows 16 (w % 4)..+15,
-// column half w / 4), and do the elementwise terms and the row and column sums
-// in a fixed order.
+// column quarter w / 4), and do the elementwise terms and the row and column sums
+// in a fixed order. Four warps per scheduler hide the latency of these epilogues.
 //
 // Delta, h and dh' arrive in the blocked layout the chain kernels keep them in
 // (per 32-column slice: 8-column blocks of 16-byte rows), which is the K-major
@@ -59,8 +59,10 @@ namespace {
 using namespace sm100;
 using namespace warp;
 
-constexpr int kThreads = 256;
-constexpr int kWN = 2;  // column groups: warp w owns column half w / 4
+constexpr int kThreads = 512;
+constexpr int kWN = 4;              // column groups: warp w owns column quarter w / 4
+constexpr int kJJ = 64 / kWN / 8;   // 8-column tiles of a C x C accumulator per warp
+constexpr int kParts = 128 / kWN / 32;  // 32-column loads of a C x K accumulator per warp
 constexpr int C = 64, K = 128, V = 128;
 constexpr int kStoreTid = 32;  // issues the TMA stores and the loads of the buffers they read
 // The products of a round are issued by two threads (thread 0 and kStoreTid), each
@@ -87,8 +89,8 @@ static_assert(kdG == kT1 + 8192 && kSmemBytes <= 232448, "shared memory layout")
 
 // tensor memory columns: round 1  S, G, P1, dU;  round 2  dAkk, T1 K, dk (T1^T Q), dO h^T;
 // round 3  dU h^T, Delta dh'^T, dk (+ dG K + dG^T K). dk lives at kCDK for the whole
-// item; dq is parked at kCPark between the heads of an item (lanes 16..31 of each
-// sub-partition hold the second column half).
+// item; dq is parked at kCPark between the heads of an item (column quarter w / 4 at
+// lanes 16 ((w / 4) % 2).. of the warp's sub-partition, columns 32 ((w / 4) / 2)..).
 constexpr uint32_t kCS = 0, kCG = 64, kCP1 = 128, kCU = 320;
 constexpr uint32_t kCAkk = 0, kCTK = 64, kCDK = 192, kCQ1 = 320;
 constexpr uint32_t kCKb = 0, kCK2 = 320, kCPark = 448;
@@ -99,7 +101,7 @@ enum Bar { kBarQ, kBarK, kBarD0, kBarD1, kBarDO, kBarA, kBarV, kBarSt, kBarMma, 
 
 struct Vecs {
     float gam[64], egam[64], bet[64];
-    float rowdg[kWN][64], rowdb[kWN][64];  // per column-half partial row sums
+    float rowdg[kWN][64], rowdb[kWN][64];  // per column-group partial row sums
     float coldg[4][64];                    // per row-quarter partial column sums
     float scal[kThreads / 32];             // per-warp partial of the chunk-level dgamma_C term
 };
@@ -110,6 +112,10 @@ static_assert(sizeof(Vecs) <= 4096, "vector area");
 __device__ __forceinline__ uint32_t sw_off(int r, int c, int half_bytes) {
     return (c >> 6) * half_bytes + (r >> 3) * 1024 + (r & 7) * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
 }
+
+// This warp's kJJ 8-column tiles of a C x C accumulator (16 rows): v[4 jj + q].
+static_assert(kJJ == 2, "16 columns of a C x C accumulator per warp");
+__device__ __forceinline__ void ld_cc(uint32_t taddr, float (&v)[4 * kJJ]) { tmem_ld16x256_x2(taddr, v); }
 
 __device__ __forceinline__ float2 ld_pair_sw(uint32_t base, int r, int c) {
     uint32_t u;
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = (uint32_t)(wm * 32) << 16;
-    const uint32_t park = tmem + ((uint32_t)(wm * 32 + wn * 16) << 16) + kCPark;
+    const uint32_t park = tmem + ((uint32_t)(wm * 32 + (wn & 1) * 16) << 16) + kCPark + 32 * (wn >> 1);
     uint32_t phase = 0;  // bit b: parity of the next completion of barrier b (same in every thread)
     uint32_t pend = 0;   // issuing threads: barriers with a completion not yet waited for
 
@@ -345,28 +351,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         const float er[2] = {vec.egam[r0], vec.egam[r1]};
         const float br[2] = {vec.bet[r0], vec.bet[r1]};
         const bool lr[2] = {r0 < len, r1 < len};
-        float rdg[2] = {0.f, 0.f}, rdb[2] = {0.f, 0.f}, cdg[8] = {}, sdg = 0.f;
-        const int cc0 = 32 * wn, ck0 = 64 * wn;  // this warp's first column (C x C, C x K)
+        float rdg[2] = {0.f, 0.f}, rdb[2] = {0.f, 0.f}, cdg[2 * kJJ] = {}, sdg = 0.f;
+        const int cc0 = (64 / kWN) * wn, ck0 = (128 / kWN) * wn;  // this warp's first column (C x C, C x K)
         ok = wait_bar(kBarMma);
         tc_fence_after();
         if (ok && tid == 0 && nxt.valid) load_a(nxt);  // Ainv and dDelta are consumed
         ok = ok && wait_bar(kBarV);
 
-        float sacc[4][4], gacc[4][4];  // S -> strictly lower E, G: kept for round 2
+        float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for round 2
         if (ok) {
-            float v[16], pacc[4][4];
-            tmem_ld16x256_x4(tmem + lane_base + kCS + cc0, v);
+            float v[16], pacc[kJJ][4];
+            {
+                float c[4 * kJJ];
+                ld_cc(tmem + lane_base + kCS + cc0, c);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sacc[i >> 2][i & 3] = v[i];
-            tmem_ld16x256_x4(tmem + lane_base + kCG + cc0, v);
+                for (int i = 0; i < 4 * kJJ; ++i) sacc[i >> 2][i & 3] = c[i];
+                ld_cc(tmem + lane_base + kCG + cc0, c);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) gacc[i >> 2][i & 3] = v[i];
-            tmem_ld16x256_x4(tmem + lane_base + kCP1 + cc0, v);
+                for (int i = 0; i < 4 * kJJ; ++i) gacc[i >> 2][i & 3] = c[i];
+                ld_cc(tmem + lane_base + kCP1 + cc0, c);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pacc[i >> 2][i & 3] = v[i];
+                for (int i = 0; i < 4 * kJJ; ++i) pacc[i >> 2][i & 3] = c[i];
+            }
             // T1 = scale M o P1, Z = T1 o S (row and column sums)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
+            for (int jj = 0; jj < kJJ; ++jj)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int hi = q >> 1, s = cc0 + 8 * jj + 2 * c4 + (q & 1), r = hi ? r1 : r0;
@@ -380,14 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
                     sacc[jj][q] = s < r ? E : 0.f;  // strictly lower part of E for the A terms
                 }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < kJJ; ++jj) {
                 const int s = cc0 + 8 * jj + 2 * c4;
                 st_shared_b32(sb + kT1 + sw_off(r0, s, 8192), pack_bf16(pacc[jj][0], pacc[jj][1]));
                 st_shared_b32(sb + kT1 + sw_off(r1, s, 8192), pack_bf16(pacc[jj][2], pacc[jj][3]));
             }
             // dU: dv = beta dU (in place of v for a full chunk), dbeta += dU.v, dU -> shared memory
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < kParts; ++part) {
                 const int cb = ck0 + 32 * part;
                 tmem_ld16x256_x4(tmem + lane_base + kCU + cb, v);
 #pragma unroll
@@ -449,10 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (ok && tid == 0 && nxt.valid) load_do(nxt);  // dO is consumed
         if (ok) {
             // dAkk = -dU Delta^T (s < r): dbeta, Zr, dG -> shared memory
-            float v[16];
-            tmem_ld16x256_x4(tmem + lane_base + kCAkk + cc0, v);
+            float v[4 * kJJ];
+            ld_cc(tmem + lane_base + kCAkk + cc0, v);
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < kJJ; ++jj) {
                 float dgv[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -473,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
             // dq = scale diag(e^gamma) dO h^T + T1 K (+ the group's earlier heads);
             // dgamma += scale e^gamma q.(dO h^T)
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < kParts; ++part) {
                 const int cb = ck0 + 32 * part;
                 float a[16], b[16], x[16];
                 tmem_ld16x256_x4(tmem + lane_base + kCQ1 + cb, a);
@@ -562,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (!ok) break;
         if (tid == 0 && nxt.valid) load_st(nxt);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+        for (int part = 0; part < kParts; ++part) {
             const int cb = ck0 + 32 * part;
             float kb[16], k2[16], x[16];
             tmem_ld16x256_x4(tmem + lane_base + kCKb + cb, kb);  // dU h^T = -dKb
@@ -610,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
             rdb[hi] += __shfl_xor_sync(0xffffffffu, rdb[hi], 2);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 2 * kJJ; ++i) {
             cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 4);
             cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 8);
             cdg[i] += __shfl_xor_sync(0xffffffffu, cdg[i], 16);
@@ -625,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         }
         if (g == 0) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < kJJ; ++jj) {
                 vec.coldg[wm][cc0 + 8 * jj + 2 * c4] = cdg[2 * jj];
                 vec.coldg[wm][cc0 + 8 * jj + 2 * c4 + 1] = cdg[2 * jj + 1];
             }
