@@ -243,9 +243,10 @@ BwdLayout bwd_layout(const Plan &P) {
 
 // Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv,
 // scaled inverses (when no `saved`) |
-// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta.
+// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta |
+// sequence-split scratch (r, Q, end gradients of every segment).
 struct TcBwdLayout {
-    size_t seq, saved, hc, dhc, delta, ddelta, total;
+    size_t seq, saved, hc, dhc, delta, ddelta, seg, total;
 };
 
 TcBwdLayout tc_bwd_layout(const Plan &P) {
@@ -260,7 +261,8 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dlb;
-    L.total = L.ddelta + dl;
+    L.seg = L.ddelta + dl;
+    L.total = L.seg + P.seg_bytes;
     return L;
 }
 
@@ -563,7 +565,31 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
         b.dq = dq; b.dk = dk; b.dv = dv; b.dg = dg; b.dbeta = dbeta; b.dh0 = dh0;
         b.status = status;
         b.stream = st;
-        {
+        if (P.nseg > 1) {
+            // sequence split of the reverse scan: segment pass (r, Q) -> composition of the
+            // segments' end gradients from dht -> output pass
+            float *seg = (float *)(ws + T.seg);
+            const size_t per = (size_t)P.d.N * P.nseg * P.d.Hv * P.d.K;
+            BwdSplit sp;
+            sp.nseg = P.nseg;
+            sp.seg_r = seg;
+            sp.seg_Q = seg + per * P.d.V;
+            sp.seg_dh = seg + per * (P.d.V + P.d.K);
+            sp.mode = 1;
+            {
+                TimedLaunch t("bwd_split_seg", st);
+                if (launch_bwd_dh_tc(b, f.w16, f.p16, ws + T.dhc, ws + T.ddelta, sp) != cudaSuccess) return GDN_ERR_CUDA;
+            }
+            {
+                TimedLaunch t("bwd_split_compose", st);
+                if (launch_split_compose_bwd(P.d, P.nseg, dht, sp.seg_r, sp.seg_Q, seg + per * (P.d.V + P.d.K), st) !=
+                    cudaSuccess)
+                    return GDN_ERR_CUDA;
+            }
+            sp.mode = 2;
+            TimedLaunch t("bwd_dh", st);
+            if (launch_bwd_dh_tc(b, f.w16, f.p16, ws + T.dhc, ws + T.ddelta, sp) != cudaSuccess) return GDN_ERR_CUDA;
+        } else {
             TimedLaunch t("bwd_dh", st);
             if (launch_bwd_dh_tc(b, f.w16, f.p16, ws + T.dhc, ws + T.ddelta) != cudaSuccess) return GDN_ERR_CUDA;
         }

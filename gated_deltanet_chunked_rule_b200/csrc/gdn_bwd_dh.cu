@@ -29,6 +29,15 @@
 // Y and X do not depend on the chain, so they are ready one or two chunks
 // ahead of it. Hand-over by release/acquire counters and mbarriers; every wait
 // is bounded.
+//
+// Sequence split (long sequences, few heads): a chunk maps its exit-state
+// gradient dh' to dh = A dh' + b with A = e^{gamma_C} I - w^T diag(e^{gamma_C -
+// gamma}) K, the transpose of the forward chunk's transition operator, so a
+// segment of chunks maps the gradient at its end to Q dh_end + r. The segment
+// pass runs the scan on [r | Q]: r from zero with the real dO, Q from the identity
+// on K more columns whose dO tile is read out of range (zero), so Y = X = 0
+// there. A composition walks the segments backwards from dht (gdn_split.cu), and
+// the output pass reruns every segment from its composed dh_end.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -89,8 +98,17 @@ struct BwdDhParams {
     __nv_bfloat16 *ddelta;       // [T_total, Hv, V]
     float *dh0;                  // [N, Hv, K, V] or null
     float scale;
+    // Sequence split: blockIdx.x = sequence * nseg + segment, a segment being a
+    // contiguous run of ceil(chunks / nseg) chunks of its sequence.
+    int nseg;
+    int mode;                    // BwdDhMode
+    const float *seg_dh;         // kBSegOut: [N * nseg, Hv, K, V] gradient at every segment's end
+    float *seg_r;                // kBSegPass: [N * nseg, Hv, K, V] gradient at the start from a zero end
+    float *seg_Q;                // kBSegPass: [N * nseg, Hv, K, K] the segment's operator
     unsigned *status;
 };
+
+enum BwdDhMode { kBWhole = 0, kBSegPass = 1, kBSegOut = 2 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -103,11 +121,22 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t sb = smem_u32(smem);
 
     const Dims &d = prm.d;
-    const int n = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * kBV;
+    const int nseg = prm.nseg;
+    const int n = blockIdx.x / nseg, sseg = blockIdx.x % nseg, h = blockIdx.y, c0 = blockIdx.z * kBV;
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const SeqRange sr = seq_range(d, n);
-    const int nch = (sr.len + kChunk - 1) / kChunk;
+    // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
+    const SeqRange seq = seq_range(d, n);
+    const int nch_seq = (seq.len + kChunk - 1) / kChunk;
+    const int per_seg = (nch_seq + nseg - 1) / nseg;
+    const int j0 = min(sseg * per_seg, nch_seq), j1 = min(j0 + per_seg, nch_seq);
+    SeqRange sr;
+    sr.start = seq.start + j0 * kChunk;
+    sr.chunk0 = seq.chunk0 + j0;
+    sr.len = j1 > j0 ? min(seq.len - j0 * kChunk, (j1 - j0) * kChunk) : 0;
+    const int nch = j1 - j0;
+    const size_t seg_idx = (size_t)n * nseg + sseg;
+    const bool outputs = prm.mode != kBSegPass;  // dh' and dDelta of every chunk
     constexpr int K = 128, V = 128;
 
     if (tid == 0) {
@@ -144,7 +173,10 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float scl = prm.scale;
         float hf[2][2][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8(cb+nt)+2c4(+1)
         {
-            const float *src = prm.dht ? prm.dht + ((size_t)n * d.Hv + h) * K * V : nullptr;
+            const float *src = prm.mode == kBWhole ? (prm.dht ? prm.dht + ((size_t)n * d.Hv + h) * K * V : nullptr)
+                               : prm.mode == kBSegOut ? prm.seg_dh + (seg_idx * d.Hv + h) * K * V
+                                                      : nullptr;
+            const bool ident = prm.mode == kBSegPass && c0 >= V;  // operator columns start as I
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -153,7 +185,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int q = 0; q < 4; ++q) {
                         const int dim = 32 * p + 16 * mt + g + ((q >> 1) << 3);
                         const int col = 8 * (cb + nt) + 2 * c4 + (q & 1);
-                        hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : 0.f;
+                        hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : (ident && dim == c0 - V + col ? 1.f : 0.f);
                     }
         }
         auto write_hb = [&]() {
@@ -288,18 +320,29 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (!ok) {
             if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
             *abort_flag = 1;
-        } else if (prm.dh0) {
-            float *dst = prm.dh0 + ((size_t)n * d.Hv + h) * K * V + c0;
+        } else {
+            // end state: dh0 (from the CTA holding the sequence's first chunk), or the
+            // segment's r / Q columns
+            float *dst = nullptr;
+            int ld = V;
+            if (prm.mode == kBSegPass) {
+                if (c0 < V) dst = prm.seg_r + (seg_idx * d.Hv + h) * K * V + c0;
+                else dst = prm.seg_Q + (seg_idx * d.Hv + h) * K * K + (c0 - V), ld = K;
+            } else if (prm.dh0 && sseg == 0) {
+                dst = prm.dh0 + ((size_t)n * d.Hv + h) * K * V + c0;
+            }
+            if (dst) {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int dim = 32 * p + 16 * mt + g + half * 8;
-                        *reinterpret_cast<float2 *>(dst + (size_t)dim * V + 8 * (cb + nt) + 2 * c4) =
-                            make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
-                    }
+                        for (int half = 0; half < 2; ++half) {
+                            const int dim = 32 * p + 16 * mt + g + half * 8;
+                            *reinterpret_cast<float2 *>(dst + (size_t)dim * ld + 8 * (cb + nt) + 2 * c4) =
+                                make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
+                        }
+            }
         }
     } else if (warp < 12) {
         // ============================================================= aux
@@ -358,7 +401,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             {
                 __nv_bfloat16 *hc = prm.dh_chunks + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + blockIdx.z) * (K * kBV);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 4 && outputs; ++i) {
                     const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 128 + k
                     *reinterpret_cast<uint4 *>(hc + 8 * e) = ld_shared_v4(sb + kHb + e * 16);
                 }
@@ -371,7 +414,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const int e = atid + kAux * i, t = e & 63, nb = e >> 6;
-                if (t < len) {
+                if (t < len && outputs) {
                     uint4 v4 = ld_shared_v4(sb + kDb + nb * 1024 + t * 16);
                     v4.x ^= 0x80008000u, v4.y ^= 0x80008000u, v4.z ^= 0x80008000u, v4.w ^= 0x80008000u;
                     *reinterpret_cast<uint4 *>(prm.ddelta + ((size_t)(t0 + t) * d.Hv + h) * V + c0 + 8 * nb) = v4;
@@ -469,7 +512,8 @@ bool tc_bwd_supported(const Dims &d, int dtype) {
     return dtype == GDN_DTYPE_BF16 && d.K == 128 && d.V == 128;
 }
 
-cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16) {
+cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16,
+                             const BwdSplit &split) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
     CUtensorMap mq, mk, mw, mp, mdo;
@@ -499,10 +543,20 @@ cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16,
     p.ddelta = (__nv_bfloat16 *)ddelta16;
     p.dh0 = a.dh0;
     p.scale = d.scale;
+    p.nseg = split.nseg > 0 ? split.nseg : 1;
+    p.mode = split.mode;
+    p.seg_dh = split.seg_dh;
+    p.seg_r = split.seg_r;
+    p.seg_Q = split.seg_Q;
+    if ((p.mode == kBSegPass && (!p.seg_r || !p.seg_Q)) || (p.mode == kBSegOut && !p.seg_dh) || p.mode < 0 ||
+        p.mode > kBSegOut)
+        return cudaErrorInvalidValue;
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(bwd_dh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    bwd_dh_kernel<<<dim3(d.N, d.Hv, d.V / kBV), kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mp, mdo, p);
+    // the segment pass also carries the K operator columns
+    const dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kBSegPass ? d.K : 0)) / kBV);
+    bwd_dh_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mp, mdo, p);
     return cudaGetLastError();
 }
 

@@ -155,7 +155,19 @@ cudaError_t launch_split_compose(const FwdArgs &a);
 // Tensor-core backward (bf16, K = V = 128): reverse dh scan, then the per-chunk
 // gradients, which sum dq and dk over each qk head's group of value heads.
 bool tc_bwd_supported(const Dims &d, int dtype);
-cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16);
+// Sequence split of the reverse scan (mode 0: whole sequences; 1: segment pass
+// writing each segment's r, Q; 2: output pass from each segment's composed
+// end gradient seg_dh).
+struct BwdSplit {
+    int nseg = 1, mode = 0;
+    const float *seg_dh = nullptr;
+    float *seg_r = nullptr, *seg_Q = nullptr;
+};
+cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16, void *dh_chunks16, void *ddelta16,
+                             const BwdSplit &sp = BwdSplit());
+// Composition of the backward split: seg_dh[nseg-1] = dht, seg_dh[s-1] = Q_s seg_dh[s] + r_s.
+cudaError_t launch_split_compose_bwd(const Dims &d, int nseg, const float *dht, const float *seg_r,
+                                     const float *seg_Q, float *seg_dh, cudaStream_t stream);
 cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const void *dh_chunks16,
                                const void *delta16, const void *ddelta16);
 

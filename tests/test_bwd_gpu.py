@@ -161,3 +161,56 @@ def test_backward_from_states_saved_by_a_split_forward(oracle_mod, monkeypatch):
     g = gpu_bwd(x, use_saved=True)
     monkeypatch.delenv("GDN_NSEG")
     check(oracle_mod, x, g, "bwd from split-forward states")
+
+
+def _split_inputs(seed):
+    # packed batch: an empty sequence, one shorter than the segment count (empty
+    # segments), a long one and a ragged tail; per-sequence h0 and dht
+    w = Workload("bwd_split", B=1, T=1500, Hq=2, Hv=4, K=128, V=128, grads=True, seed=seed)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 0, 100, 1037, 1500], dtype=torch.int32)
+    gen = torch.Generator().manual_seed(seed + 1)
+    x["h0"] = 0.02 * torch.randn((4, 4, 128, 128), generator=gen)
+    x["dht"] = 0.01 * torch.randn((4, 4, 128, 128), generator=gen)
+    return x
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 7])
+def test_backward_sequence_split_matches_oracle_and_unsplit(oracle_mod, monkeypatch, nseg):
+    # Sequence split of the reverse scan: each segment maps the gradient at its end
+    # to Q dh + r (Q the transposed product of its chunks' operators); the segments'
+    # end gradients are composed backwards from dht, then every segment reruns
+    # from its own. The forward runs unsplit, so only the backward differs.
+    x = _split_inputs(23)
+    monkeypatch.setenv("GDN_NSEG", "1")
+    _, _, saved = gpu_fwd(x, save_for_backward=True)
+    import gated_deltanet_chunked_rule_b200 as gdn
+    d = to_dev(x)
+
+    def bwd():
+        out = gdn.chunk_gated_delta_rule_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], saved, d["do"], d["dht"],
+                                             d["scale"], d["h0"], d["cu_seqlens"], x["cu_seqlens"])
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0
+        return dict(zip(NAMES, out))
+
+    g1 = bwd()
+    monkeypatch.setenv("GDN_NSEG", str(nseg))
+    g2 = bwd()
+    monkeypatch.delenv("GDN_NSEG")
+    check(oracle_mod, x, g2, f"bwd split{nseg}")
+    for n in NAMES:
+        assert rel_fro(f64(g2[n]), f64(g1[n])) <= TOL_GRAD_REL, n
+    torch.testing.assert_close(g2["dh0"][0].cpu(), x["dht"][0], rtol=0, atol=0)  # empty sequence
+
+
+def test_backward_sequence_split_slow_decay(oracle_mod, monkeypatch):
+    # nearly-undecayed gates: dht reaches dh0 through every segment boundary
+    w = Workload("bwd_split_slow", B=1, T=1024, Hq=1, Hv=2, K=128, V=128, h0_std=0.05, grads=True, seed=24)
+    x = make_inputs(w)
+    x["g"] = x["g"] * 0.01
+    x["dht"] = 0.01 * torch.randn((1, 2, 128, 128), generator=torch.Generator().manual_seed(3))
+    monkeypatch.setenv("GDN_NSEG", "4")
+    g = gpu_bwd(x)
+    monkeypatch.delenv("GDN_NSEG")
+    check(oracle_mod, x, g, "bwd split slow decay")
