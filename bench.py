@@ -290,6 +290,58 @@ def cpu_baseline(args, w):
                       f"{sample_T} tokens, all {w.Hv} heads ({dt:.2f} s wall)"}
 
 
+def run_decode(args):
+    """Token-by-token (decode) step through gdn_recurrent_fwd: one token for each of
+    B sequences and Hv heads per step, state updated in place. The state (B*Hv*K*V
+    fp32, 512 MB here) is larger than L2, so every step moves it from and to HBM;
+    the roofline is that traffic against the measured copy bandwidth."""
+    import torch
+    import gated_deltanet_chunked_rule_b200 as gdn
+    gdn.lib()  # fail loudly if the extension is missing
+    B, Hq, Hv, K, V = 256, 16, 32, 128, 128
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev).manual_seed(0)
+    nrm = torch.nn.functional.normalize
+    q = nrm(torch.randn(B, 1, Hq, K, device=dev, generator=gen), dim=-1).bfloat16()
+    k = nrm(torch.randn(B, 1, Hq, K, device=dev, generator=gen), dim=-1).bfloat16()
+    v = torch.randn(B, 1, Hv, V, device=dev, generator=gen).bfloat16()
+    g = -torch.nn.functional.softplus(torch.randn(B, 1, Hv, device=dev, generator=gen))
+    beta = torch.sigmoid(torch.randn(B, 1, Hv, device=dev, generator=gen))
+    state = 0.02 * torch.randn(B, Hv, K, V, device=dev, generator=gen)
+    o = torch.empty(B, 1, Hv, V, device=dev, dtype=torch.bfloat16)
+
+    def step():
+        gdn.recurrent_gated_delta_rule(q, k, v, g, beta, None, state, out=o, final_state=state)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(0) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    if gdn.device_status() != 0:
+        raise SystemExit("decode step reported a device error")
+    ms = e0.elapsed_time(e1) / args.steps
+    traffic = 2 * B * Hv * K * V * 4 + B * (2 * Hq * K + 2 * Hv * V) * 2 + 2 * B * Hv * 4
+    pk, pk_kind = peaks()
+    achieved = traffic / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "GDN decode step Mtokens/s (one token per sequence, state in HBM)",
+        "value": B / (ms * 1e3), "unit": "Mtokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode_b256_hv32", "B": B, "T": 1, "Hq": Hq, "Hv": Hv, "K": K, "V": V,
+                   "step": "decode", "l2": "state 512 MB > L2, updated in place every step"},
+        "roofline": {"kernel": "recurrent", "bound": "hbm", "unit": "GB/s", "achieved": achieved,
+                     "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)", "traffic": None,
+                     "algorithmic_bytes": traffic, "frac": achieved / pk["hbm_gbs"]},
+        "gpu_launches": args.steps, "clocks": clk.summary()}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -300,8 +352,11 @@ def main():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true", help="time the token-by-token step instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.decode:
+        return run_decode(args)
 
     from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, make_inputs, scaled
     w = WORKLOADS[args.workload]

@@ -9,5 +9,6 @@ from .api import (  # noqa: F401
     chunk_gated_delta_rule_bwd,
     chunk_gated_delta_rule_fwd,
     device_status,
+    recurrent_gated_delta_rule,
 )
 from ._binding import GdnError, lib  # noqa: F401

@@ -38,6 +38,7 @@ EXPORTS = (
     "gdn_timing_enable",
     "gdn_timing_report",
     "gdn_chunk_fwd_noalloc",
+    "gdn_recurrent_fwd",
 )
 
 # Size of the static scratch array behind gdn_chunk_fwd_noalloc.
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_bwd.restype = i
             L.gdn_chunk_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             L.gdn_chunk_fwd_noalloc.restype = i
+            L.gdn_recurrent_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            L.gdn_recurrent_fwd.restype = i
             L.gdn_get_device_status.argtypes = [vp]
             L.gdn_get_device_status.restype = i
             L.gdn_status_string.argtypes = [i]

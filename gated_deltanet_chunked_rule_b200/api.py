@@ -132,6 +132,26 @@ def chunk_gated_delta_rule_bwd(q, k, v, g, beta, saved, do, dht=None, scale=None
     return dq, dk, dv, dbeta, dg, dh0
 
 
+def recurrent_gated_delta_rule(q, k, v, g, beta, scale=None, initial_state=None, cu_seqlens=None,
+                               cu_seqlens_host=None, out=None, final_state=None):
+    """Token-by-token (decode) step: the same recurrence as the chunked forward, one
+    token after another, for a few tokens per sequence (gdn_recurrent_fwd). Returns
+    (o, final_state); `final_state` may be `initial_state` itself (updated in place)."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    q, k, v, g, beta, h0 = map(_c, (q, k, v, g, beta, initial_state))
+    P = Problem(q, v, scale, cu_seqlens, cu_seqlens_host)
+    B, T, Hq, Hv, K, V = P.shape
+    dev = q.device
+    o = out if out is not None else torch.empty((B, T, Hv, V), dtype=q.dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty((P.N, Hv, K, V), dtype=torch.float32, device=dev)
+    rc = _b.lib().gdn_recurrent_fwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                    _ptr(o), _ptr(final_state), _stream(dev))
+    _b.check("gdn_recurrent_fwd", rc)
+    return o, final_state
+
+
 class _ChunkGDN(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, g, beta, scale, h0, output_final_state, cu_seqlens, cu_host):

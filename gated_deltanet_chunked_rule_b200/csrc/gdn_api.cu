@@ -682,6 +682,31 @@ int gdn_chunk_fwd_noalloc(const gdn_problem *p, const void *q, const void *k, co
                          GDN_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+int gdn_recurrent_fwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                      const float *g, const float *beta, const float *h0, void *o,
+                      float *final_state, void *stream) {
+    Plan P;
+    int rc = make_plan(p, &P);
+    if (rc != GDN_OK) return rc;
+    if (P.d.T_total > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, h0, o, final_state};
+    for (const void *x : ptrs)
+        if (x && !aligned16(x)) return GDN_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    RecurrentArgs a;
+    memset(&a, 0, sizeof(a));
+    a.d = P.d;
+    a.dtype = P.dtype;
+    a.cu = p->num_seqs > 0 ? p->cu_seqlens : nullptr;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.h0 = h0;
+    a.o = o; a.final_state = final_state;
+    a.status = status;
+    a.stream = (cudaStream_t)stream;
+    TimedLaunch t("recurrent", a.stream);
+    return launch_recurrent(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 int gdn_get_device_status(void *stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GDN_ERR_CUDA;
     unsigned v = 0, zero = 0;

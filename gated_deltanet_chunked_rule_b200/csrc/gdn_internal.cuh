@@ -122,6 +122,22 @@ struct FwdArgs {
     float *seg_c, *seg_P;    // [N * nseg, Hv, K, V] / [.., K, K] segment end state from zero, operator
 };
 
+// Token-by-token (decode) step: q, k [T, Hq, K], v, o [T, Hv, V] (T = B*T or the
+// packed length), g, beta [T, Hv], h0 / final_state [N, Hv, K, V] fp32 (may alias).
+// cu: the device copy of cu_seqlens, or null for B sequences of T tokens.
+struct RecurrentArgs {
+    Dims d;
+    int dtype;
+    const int *cu;
+    const void *q, *k, *v;
+    const float *g, *beta, *h0;
+    void *o;
+    float *final_state;
+    unsigned *status;
+    cudaStream_t stream;
+};
+cudaError_t launch_recurrent(const RecurrentArgs &a);
+
 struct BwdArgs {
     Dims d;
     int dtype;

@@ -150,6 +150,24 @@ int gdn_chunk_fwd_noalloc(const gdn_problem *p, const void *q, const void *k, co
                           const float *g, const float *beta, const float *h0, void *o,
                           float *final_state, void *stream /* cudaStream_t */);
 
+/* Token-by-token (decode) step of the same recurrence, for a few tokens per
+ * sequence: o_t = scale S_t q_t with S_t = exp(g_t) S_{t-1} (I - beta_t k_t
+ * k_t^T) + beta_t v_t k_t^T, taken one token after another from h0 (NULL:
+ * zero) to final_state (NULL: not written). The state of every (sequence,
+ * value head) is read once and written once per call, so a decode loop calls
+ * this once per generated token. Same problem description, layouts, sizes and
+ * dtypes as gdn_chunk_fwd; no workspace. final_state may be the same buffer as
+ * h0 (the update is in place). Each sequence's tokens are read from the device
+ * copy of cu_seqlens; an inconsistent one is recorded as GDN_ERR_DEVICE_ARG in
+ * the status word and that sequence is left untouched. The chunked forward is
+ * the faster choice once a call covers more than a few dozen tokens per
+ * sequence. This is the gated delta rule exactly as the pages state it for
+ * the GDN layers (page 1, "什么是 FlashQLA"), taken without chunks: the pages'
+ * kernels are the prefill of this recurrence and give no decode kernel. */
+int gdn_recurrent_fwd(const gdn_problem *p, const void *q, const void *k, const void *v,
+                      const float *g, const float *beta, const float *h0, void *o,
+                      float *final_state, void *stream /* cudaStream_t */);
+
 /* Synchronises `stream`, then returns and clears the current device's status
  * word (GDN_OK if no kernel recorded a problem since the last call). */
 int gdn_get_device_status(void *stream /* cudaStream_t */);
