@@ -353,6 +353,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode", action="store_true", help="time the token-by-token step instead")
+    ap.add_argument("--heads", default=None, help="HQ,HV: override the workload's head counts (sweeps)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.decode:
@@ -360,6 +361,10 @@ def main():
 
     from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, make_inputs, scaled
     w = WORKLOADS[args.workload]
+    if args.heads:
+        from dataclasses import replace
+        hq, hv = (int(x) for x in args.heads.split(","))
+        w = replace(w, name=f"{w.name}_hq{hq}_hv{hv}", Hq=hq, Hv=hv)
     if args.impl == "reference":
         return run_reference(args, w)
 

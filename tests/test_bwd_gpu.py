@@ -214,3 +214,14 @@ def test_backward_sequence_split_slow_decay(oracle_mod, monkeypatch):
     g = gpu_bwd(x)
     monkeypatch.delenv("GDN_NSEG")
     check(oracle_mod, x, g, "bwd split slow decay")
+
+
+@pytest.mark.parametrize("Hq,Hv", [(2, 6), (1, 4), (4, 12)])
+def test_larger_head_groups(oracle_mod, Hq, Hv):
+    # groups of 3 and 4 value heads per qk head: the per-chunk gradient kernel sums
+    # dq and dk over every head of the group on chip (dk accumulated in TMEM by
+    # each next head's products, dq parked between heads)
+    w = Workload(f"bwd_g{Hv // Hq}", B=1, T=333, Hq=Hq, Hv=Hv, K=128, V=128, h0_std=0.02, grads=True,
+                 seed=40 + Hv)
+    x = make_inputs(w)
+    check(oracle_mod, x, gpu_bwd(x), w.name)

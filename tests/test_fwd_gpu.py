@@ -179,3 +179,13 @@ def test_sequence_split_with_fast_decay_and_slow_decay(oracle_mod, monkeypatch):
     monkeypatch.delenv("GDN_NSEG")
     e = check_fwd(oracle_mod, x, o, f, "split_slow")
     print(f"[split slow decay] o err {e[0]:.3e} final err {e[1]:.3e}")
+
+
+@pytest.mark.parametrize("Hq,Hv", [(8, 24), (16, 48), (2, 6)])
+def test_non_power_of_two_head_counts(oracle_mod, Hq, Hv):
+    # the pages' head grid includes 48 and 24 value heads (groups of 3)
+    w = Workload(f"fwd_h{Hv}", B=1, T=200, Hq=Hq, Hv=Hv, K=128, V=128, h0_std=0.02, seed=50 + Hv)
+    x = make_inputs(w)
+    o, f, _ = gpu_fwd(x)
+    e = check_fwd(oracle_mod, x, o, f, w.name)
+    print(f"[heads {Hq}/{Hv}] o err {e[0]:.3e} final err {e[1]:.3e}")
