@@ -80,7 +80,8 @@ constexpr int kK = 0, kW = 16384, kU = 32768, kCStageBytes = 40960;
 constexpr int kO0 = kC0 + kStages * kCStageBytes;  // output ring: q [64][128] bf16, P [64][64] bf16
 constexpr int kQ = 0, kP = 16384, kOStageBytes = 24576;
 constexpr int kSmall = kO0 + kStages * kOStageBytes;
-constexpr int kSmemBytes = kSmall + 2048 + 1024;
+constexpr int kOs = kSmall + 2048;  // o of a full chunk, staged for its TMA store: [64][32] bf16
+constexpr int kSmemBytes = kOs + 4096 + 1024;
 static_assert(kC0 % 1024 == 0 && kO0 % 1024 == 0 && kCStageBytes % 1024 == 0 && kOStageBytes % 1024 == 0 &&
                   kSmemBytes <= 232448,
               "shared memory layout");
@@ -136,7 +137,8 @@ struct Fwd2Params {
 __global__ void __launch_bounds__(kThreads, 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
-            const __grid_constant__ CUtensorMap tm_p, const Fwd2Params prm) {
+            const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_o,
+            const Fwd2Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -421,23 +423,36 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 tmem_ld16x256_x4(tb + kColQ, dq);
                 tmem_ld16x256_x4(tb + kColP, dp);
                 tc_fence_before();
+                if (et == 0) bulk_wait_read<0>();  // the previous chunk's o has left the staging tile
                 epi_sync(true);
                 if (et == 0) publish(&ctr[kTmemO], j + 1);
                 const float er[2] = {__expf(g0), __expf(g1)};
                 const int t0 = sr.start + j * kChunk;
+                const bool full = len == kChunk;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    if (rr[half] < len) {
-                        __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + rr[half]) * d.Hv + h) * V + c0 + 2 * ec;
+                    __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + rr[half]) * d.Hv + h) * V + c0 + 2 * ec;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int k = 4 * i + 2 * half;
-                            *reinterpret_cast<uint32_t *>(dst + 8 * i) =
-                                pack_bf16(scl * fmaf(er[half], dq[k], dp[k]), scl * fmaf(er[half], dq[k + 1], dp[k + 1]));
-                        }
+                    for (int i = 0; i < 4; ++i) {
+                        const int k = 4 * i + 2 * half;
+                        const uint32_t x =
+                            pack_bf16(scl * fmaf(er[half], dq[k], dp[k]), scl * fmaf(er[half], dq[k + 1], dp[k + 1]));
+                        if (full)  // a ragged chunk's tile would spill into the next sequence
+                            st_shared_b32(sb + kOs + rr[half] * 64 + (8 * i + 2 * ec) * 2, x);
+                        else if (rr[half] < len)
+                            *reinterpret_cast<uint32_t *>(dst + 8 * i) = x;
+                    }
+                }
+                if (full) {
+                    fence_proxy_async();
+                    epi_sync(true);
+                    if (et == 0) {
+                        tma_store_3d(&tm_o, sb + kOs, c0, h, t0);
+                        bulk_commit();
                     }
                 }
             }
+            if (et == 0) bulk_wait_all();  // the o stores read shared memory until they complete
             if (!ok) {
                 if (et == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
                 *abort_flag = 1;
@@ -586,7 +601,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.N == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || (a.o && !a.p16)) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mw, mu, mp;
+    CUtensorMap mq, mk, mw, mu, mp, mo;
     const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
     const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
@@ -604,6 +619,11 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
         !make_map(&mw, BF, a.w16, 3, dw, sw, b64) || !make_map(&mu, F32, a.u32, 3, du, su, bu) ||
         !make_map(&mp, BF, a.p16 ? a.p16 : a.w16, 2, dp, sp, bp))
         return cudaErrorInvalidValue;
+    // o [T, Hv, V] bf16 in 32-column, 64-row boxes (stores of full chunks)
+    const cuuint64_t dov[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
+    const cuuint64_t sov[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
+    const cuuint32_t bov[3] = {kBV, 1, 64};
+    if (!make_map(&mo, BF, a.o ? a.o : a.w16, 3, dov, sov, bov, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorInvalidValue;
     // chunk entry states and Delta: both or neither
     if ((a.h_chunks16 != nullptr) != (a.delta16 != nullptr)) return cudaErrorInvalidValue;
     Fwd2Params p;
@@ -627,7 +647,7 @@ cudaError_t launch_fwd2(const FwdArgs &a) {
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
     dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
-    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, p);
+    fwd2_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, mo, p);
     return cudaGetLastError();
 }
 
