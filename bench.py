@@ -128,15 +128,18 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639929856 + 120504832,
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639905536 + 119271680,
                sources=["gdn_bwd_grad.cu"],
-               sha256="922fdf75f61c27e9dab6e1ea7008f872b557bf28f8a8c700706be7d3b5e9c12d"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238069760 + 167706112,
+               sha256="9c445f906f00d11b8b9a477e3088567f1a89c86c4e970f0a174b9f8557a5a85e"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 167724544,
                sources=["gdn_bwd_dh.cu"],
-               sha256="6b2bd9615693f6bca2bbd0362ec471e9fd7ed1e21451937dfa3c78da1b767843"),
-    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303091968 + 230028544,
+               sha256="7b3bee60d740f4a86890b88a113f9935853013967a03f843e91efbff6e9b84c8"),
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303088896 + 230655744,
                sources=["gdn_fwd2.cu"],
-               sha256="129476ecaf0a7544e2532b67fd91152615ad381a1c0fe3c83fa7955aac1244ee"),
+               sha256="bc5af0eeb7db80640505b8f0a1593de1399503b8526b8dee7019091daa9fd905"),
+    "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549451520 + 481462272,
+               sources=["gdn_recurrent.cu"],
+               sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),
     "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=138346240 + 213746944,
                sources=["gdn_prep3.cu"],
                sha256="b5dd7e87c61c371614b692c11337e75c054daa97a1882d85b439c6cbf85f0945"),
@@ -337,7 +340,8 @@ def run_decode(args):
         "config": {"workload": "decode_b256_hv32", "B": B, "T": 1, "Hq": Hq, "Hv": Hv, "K": K, "V": V,
                    "step": "decode", "l2": "state 512 MB > L2, updated in place every step"},
         "roofline": {"kernel": "recurrent", "bound": "hbm", "unit": "GB/s", "achieved": achieved,
-                     "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)", "traffic": None,
+                     "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)",
+                     "traffic": measured_traffic("recurrent", "decode_b256_hv32", "decode"),
                      "algorithmic_bytes": traffic, "frac": achieved / pk["hbm_gbs"]},
         "gpu_launches": args.steps, "clocks": clk.summary()}))
 
