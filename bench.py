@@ -87,7 +87,7 @@ def kernel_bytes(name, w, saved=False):
                        + 2V*e (Delta, dDelta) + 2K*e/G (dq, dk, summed over the group on chip)
                        + V*e (dv) + 8 (dg, dbeta)
     plus the per-sequence states (h0, final, dht, dh0: K*V*4 each) where a kernel touches them.
-    Entry states and Delta are stored per chunk (64 rows, ragged ones padded).
+    Entry states, Delta and dDelta are stored per chunk (64 rows, ragged ones padded).
     """
     C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
     ntok = w.B * w.T
@@ -101,8 +101,7 @@ def kernel_bytes(name, w, saved=False):
     st = N * Hv * K * V * 4
     h0 = st if w.h0_std is not None else 0
     hc = nc * Hv * K * V * 2
-    d16 = ntok * Hv * V * 2     # dDelta
-    dsb = nc * C * Hv * V * 2   # Delta, per chunk
+    dsb = nc * C * Hv * V * 2   # Delta and dDelta, per chunk
     wb = ntok * Hv * K * 2      # w (bf16)
     ub = ntok * Hv * V * 4      # u (fp32)
     pb = nc * Hv * C * C * 2    # P (bf16)
@@ -117,8 +116,8 @@ def kernel_bytes(name, w, saved=False):
         "fwd_hybrid": 2 * qk1 + wb + ub + pb + gam + h0 + v1 + st + ((hc + dsb) if saved else 0),
         "bwd_prep3": prep3 + (0 if saved else ainv),
         "bwd_recompute": qk1 + wb + ub + gam + h0 + hc + dsb,
-        "bwd_dh": 2 * qk1 + wb + pb + v1 + gam + st + hc + d16 + st,
-        "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + dsb + d16 + 2 * qk1 + v1 + 2 * gam,
+        "bwd_dh": 2 * qk1 + wb + pb + v1 + gam + st + hc + dsb + st,
+        "bwd_grad": 2 * qk1 + 2 * v1 + 2 * gam + ainv + 2 * hc + 2 * dsb + 2 * qk1 + v1 + 2 * gam,
     }
     return table.get(name)
 

@@ -243,7 +243,7 @@ BwdLayout bwd_layout(const Plan &P) {
 
 // Tensor-core backward (bf16, K = V = 128) workspace: sequence table | gamma, Ainv,
 // scaled inverses (when no `saved`) |
-// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta |
+// bf16 per-chunk entry states and exit-state gradients | bf16 Delta and dDelta (blocked) |
 // sequence-split scratch (r, Q, end gradients of every segment).
 struct TcBwdLayout {
     size_t seq, saved, hc, dhc, delta, ddelta, seg, total;
@@ -254,14 +254,13 @@ TcBwdLayout tc_bwd_layout(const Plan &P) {
     TcBwdLayout L;
     const size_t hc = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * d.Hv * d.K * d.V);
     const size_t dlb = align_up(sizeof(__nv_bfloat16) * (size_t)d.NC * kChunk * d.Hv * d.V);  // blocked per chunk
-    const size_t dl = align_up(sizeof(__nv_bfloat16) * (size_t)d.T_total * d.Hv * d.V);
     L.seq = 0;
     L.saved = L.seq + P.seq_info_bytes;
     L.hc = L.saved + P.core_bytes;
     L.dhc = L.hc + hc;
     L.delta = L.dhc + hc;
     L.ddelta = L.delta + dlb;
-    L.seg = L.ddelta + dl;
+    L.seg = L.ddelta + dlb;
     L.total = L.seg + P.seg_bytes;
     return L;
 }

@@ -95,7 +95,7 @@ struct BwdDhParams {
     const float *dht;            // [N, Hv, K, V] or null
     __nv_bfloat16 *dh_chunks;    // gradient w.r.t. each chunk's exit state, blocked: per (chunk, head)
                                  // V/32 slices of [4][128][8] (the tile layout of kHb)
-    __nv_bfloat16 *ddelta;       // [T_total, Hv, V]
+    __nv_bfloat16 *ddelta;       // dDelta, blocked: per (chunk, head) V/32 slices of [4][64][8]
     float *dh0;                  // [N, Hv, K, V] or null
     float scale;
     // Sequence split: blockIdx.x = sequence * nseg + segment, a segment being a
@@ -388,8 +388,6 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (nch > 0) ok = make_do(0);
         for (int it = 0; it < nch && ok; ++it) {
             const int ci = chunk_of(it);
-            const int len = min(kChunk, sr.len - ci * kChunk);
-            const int t0 = sr.start + ci * kChunk;
             if (it + 1 < nch) {
                 ok = make_do(it + 1);  // one iteration ahead of the chain
                 if (!ok) break;
@@ -408,16 +406,19 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             aux_sync(true);
             if (atid == 0) publish(&ctr[kHbRead], it + 1);
-            // dDelta of this iteration: kDb holds -dDelta -> ddelta (live tokens), sign restored
+            // dDelta of this iteration: kDb holds -dDelta -> ddelta, one contiguous block per
+            // (chunk, head, column slice) in the tile layout (rows past a ragged chunk's end
+            // are zero), sign restored
             ok = aux_sync(atid != 0 || wait_ge(&ctr[kDbFull], it + 1, abort_flag));
             if (!ok) break;
+            {
+                __nv_bfloat16 *dc = prm.ddelta + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + blockIdx.z) * (kChunk * kBV);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int e = atid + kAux * i, t = e & 63, nb = e >> 6;
-                if (t < len && outputs) {
-                    uint4 v4 = ld_shared_v4(sb + kDb + nb * 1024 + t * 16);
+                for (int i = 0; i < 2 && outputs; ++i) {
+                    const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 64 + t
+                    uint4 v4 = ld_shared_v4(sb + kDb + e * 16);
                     v4.x ^= 0x80008000u, v4.y ^= 0x80008000u, v4.z ^= 0x80008000u, v4.w ^= 0x80008000u;
-                    *reinterpret_cast<uint4 *>(prm.ddelta + ((size_t)(t0 + t) * d.Hv + h) * V + c0 + 8 * nb) = v4;
+                    *reinterpret_cast<uint4 *>(dc + 8 * e) = v4;
                 }
             }
             aux_sync(true);

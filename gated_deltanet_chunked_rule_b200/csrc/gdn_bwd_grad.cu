@@ -74,7 +74,7 @@ constexpr int kStoreTid = 32;  // issues the TMA stores and the loads of the buf
 constexpr int kQ = 0, kKt = 16384;  // per item; dq goes out through the q tile
 constexpr int kdO = 32768;
 constexpr int kD = 49152;           // Delta, two buffers (step parity): (v/8)*1024 + t*16
-constexpr int kdD = 81920;
+constexpr int kdD = 81920;          // dDelta, blocked: (v/8)*1024 + t*16
 constexpr int kVt = 98304;          // v; dv goes out through it
 constexpr int kA = 114688;          // Ainv [64 s][64 r]
 constexpr int kT1 = 122880;         // T1 [64 r][64 s]   } dk goes out through these two:
@@ -142,7 +142,7 @@ __device__ __forceinline__ constexpr uint64_t bstep(int ks, int kblk) { return (
 
 struct GradParams {
     Dims d;
-    const __nv_bfloat16 *delta, *h, *dh;  // blocked: per (chunk, head) 4 slices of [4][64][8] / [4][128][8]
+    const __nv_bfloat16 *delta, *ddelta, *h, *dh;  // blocked: per (chunk, head) 4 slices of [4][64][8] / [4][128][8]
     const float *gamma, *beta;
     __nv_bfloat16 *dq, *dk;  // [T, Hq, K]
     __nv_bfloat16 *dv;       // [T, Hv, V]
@@ -152,7 +152,7 @@ struct GradParams {
 };
 
 struct GradMaps {
-    CUtensorMap q, k, v, d_o, ddelta, ainv;  // loads
+    CUtensorMap q, k, v, d_o, ainv;  // loads
     CUtensorMap dq, dk, dv;                 // stores
 };
 
@@ -259,8 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
     };
     auto load_a = [&](const Step &s) {  // dDelta and Ainv
         expect(kBarA, 16384 + 8192);
-        tma_load_3d(smem + kdD, &tm.ddelta, &bars[kBarA], 0, head(s), s.t0);
-        tma_load_3d(smem + kdD + 8192, &tm.ddelta, &bars[kBarA], 64, head(s), s.t0);
+        bulk_load(smem + kdD, prm.ddelta + ((size_t)s.cg * d.Hv + head(s)) * (C * V), 16384, &bars[kBarA]);
         tma_load_2d(smem + kA, &tm.ainv, &bars[kBarA], 0, (s.cg * d.Hv + head(s)) * C);
     };
     auto load_v = [&](const Step &s) {
@@ -335,11 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         } else if (ok && tid == kStoreTid) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false), idU = idesc_bf16(64, 128, true, true);
-            const uint64_t o = kbase(sb + kdO), dl = bbase(sD, 1024), ai = mbase(sb + kA), dd = mbase(sb + kdD);
+            const uint64_t o = kbase(sb + kdO), dl = bbase(sD, 1024), ai = mbase(sb + kA);
+            // dDelta as the MN-major B of dU = Ainv^T dDelta, without swizzle: core matrices of
+            // 8 tokens x 8 columns, 128 bytes apart along K (tokens), 1024 along N
+            const uint64_t dd = smem_desc(sb + kdD, 128, 1024, kSwNone);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) mma_bf16(tmem + kCP1, o + kstep(ks, 8192), dl + bstep(ks, 1024), idCC, ks > 0);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCU, ai + mstep(ks), dd + mstep(ks), idU, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + kCU, ai + mstep(ks), dd + (uint64_t)(ks * 256 >> 4), idU, ks > 0);
             commit_mma();
         }
         if (tid == kStoreTid) bulk_wait_read<0>();  // the previous dk store has read T1 | dG
@@ -732,7 +734,7 @@ cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const v
     const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_bf16_map(&m.q, a.q, 3, dqk, sqk, b3, SW) || !make_bf16_map(&m.k, a.k, 3, dqk, sqk, b3, SW) ||
         !make_bf16_map(&m.v, a.v, 3, dvv, svv, b3, SW) || !make_bf16_map(&m.d_o, a.d_o, 3, dvv, svv, b3, SW) ||
-        !make_bf16_map(&m.ddelta, ddelta16, 3, dvv, svv, b3, SW) ||
+
         !make_bf16_map(&m.ainv, a.ainv, 2, dai, sai, bai, SW) ||
         !make_bf16_map(&m.dq, a.dq, 3, dqk, sqk, b3, SW) || !make_bf16_map(&m.dk, a.dk, 3, dqk, sqk, b3, SW) ||
         !make_bf16_map(&m.dv, a.dv, 3, dvv, svv, b3, SW))
@@ -740,6 +742,7 @@ cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const v
     GradParams p;
     p.d = d;
     p.delta = (const __nv_bfloat16 *)delta16;
+    p.ddelta = (const __nv_bfloat16 *)ddelta16;
     p.h = (const __nv_bfloat16 *)h_chunks16;
     p.dh = (const __nv_bfloat16 *)dh_chunks16;
     p.gamma = a.gamma;
