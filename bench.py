@@ -272,7 +272,7 @@ def run_reference(args, w):
 
 
 def cpu_baseline(args, w):
-    """The oracle, as it stands, on the GPU machine's host cores (bounded sample)."""
+    """The oracle, as it stands, on this host's CPU cores (bounded sample)."""
     import oracle
     from gated_deltanet_chunked_rule_b200.inputs import make_inputs, scaled
     oracle.build()

@@ -24,7 +24,7 @@
 // on chip and written once, in bf16: dk stays in tensor memory (the next
 // head's T1^T Q product accumulates onto it), dq is parked in spare columns.
 // All twelve products of a step run on tcgen05 from 128-byte-swizzled
-// shared-memory tiles, in three rounds:
+// shared-memory tiles, in three product rounds:
 //   1. S = QK^T, G = KK^T, P1 = dO Delta^T, dU = Ainv^T dDelta
 //   2. dAkk, T1 K, T1^T Q (onto dk), dO h^T
 //   3. dU h^T, Delta dh'^T, and dG K + dG^T K onto dk
@@ -37,8 +37,8 @@
 // (per 32-column slice: 8-column blocks of 16-byte rows), which is the K-major
 // operand layout without swizzle; each is one contiguous bulk copy per step.
 // Each input tile of the next step is loaded by TMA as soon as the current
-// step is done with its buffer (Ainv and dDelta after round 1, dO after round
-// 2, h and dh' after round 3; Delta has two buffers), so that only a new
+// step is done with its buffer (Ainv and dDelta after product round 1, dO after
+// product round 2, h and dh' after product round 3; Delta has two buffers), so that only a new
 // item's k tile waits on memory. dv, dq and dk of a full chunk are written by
 // TMA stores from shared memory: dv in place of v, dq in place of q, dk in
 // the T1 | dG tiles; a ragged chunk is written row by row.
@@ -87,8 +87,9 @@ constexpr int kBar = kVec + 4096;
 constexpr int kSmemBytes = kBar + 128 + 1024;
 static_assert(kdG == kT1 + 8192 && kSmemBytes <= 232448, "shared memory layout");
 
-// tensor memory columns: round 1  S, G, P1, dU;  round 2  dAkk, T1 K, dk (T1^T Q), dO h^T;
-// round 3  dU h^T, Delta dh'^T, dk (+ dG K + dG^T K). dk lives at kCDK for the whole
+// tensor memory columns: product round 1  S, G, P1, dU;
+// product round 2  dAkk, T1 K, dk (T1^T Q), dO h^T;
+// product round 3  dU h^T, Delta dh'^T, dk (+ dG K + dG^T K). dk lives at kCDK for the whole
 // item; dq is parked at kCPark between the heads of an item (column quarter w / 4 at
 // lanes 16 ((w / 4) % 2).. of the warp's sub-partition, columns 32 ((w / 4) / 2)..).
 constexpr uint32_t kCS = 0, kCG = 64, kCP1 = 128, kCU = 320;
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         const bool first = cur.g == 0, last = cur.g == G - 1, full = len == C;
         const uint32_t sD = sb + kD + db * 16384;
 
-        // Delta of the next step into the other buffer (its last reader, round 3 of the
+        // Delta of the next step into the other buffer (its last reader, product round 3 of the
         // previous step, has completed)
         if (tid == 0 && nxt.valid) load_delta(nxt, db ^ 1);
         if (tid < C) {
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         ok = ok && (!first || (wait_bar(kBarQ) && wait_bar(kBarK))) && wait_bar(kBarD0 + db) &&
              wait_bar(kBarDO) && wait_bar(kBarA);
 
-        // ---- round 1: S, G, P1 (64 x 64) and dU (64 x 128)
+        // ---- product round 1: S, G, P1 (64 x 64) and dU (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false);
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (ok && tid == 0 && nxt.valid) load_a(nxt);  // Ainv and dDelta are consumed
         ok = ok && wait_bar(kBarV);
 
-        float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for round 2
+        float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for product round 2
         if (ok) {
             float v[16], pacc[kJJ][4];
             {
@@ -431,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         }
         ok = wait_bar(kBarSt);
 
-        // ---- round 2: dAkk (64 x 64), T1 K, T1^T Q onto dk, dO h^T (64 x 128)
+        // ---- product round 2: dAkk (64 x 64), T1 K, T1^T Q onto dk, dO h^T (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false), idKM = idesc_bf16(64, 128, false, true);
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         ok = __syncthreads_and(ok);
         if (!ok) break;
 
-        // ---- round 3: dU h^T, Delta dh'^T; dG K + dG^T K onto dk
+        // ---- product round 3: dU h^T, Delta dh'^T; dG K + dG^T K onto dk
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idKK = idesc_bf16(64, 128, false, false);
