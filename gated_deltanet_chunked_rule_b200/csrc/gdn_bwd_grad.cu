@@ -33,9 +33,10 @@
 // column quarter w / 4), and do the elementwise terms and the row and column sums
 // in a fixed order. Four warps per scheduler hide the latency of these epilogues.
 //
-// Delta, h and dh' arrive in the blocked layout the chain kernels keep them in
-// (per 32-column slice: 8-column blocks of 16-byte rows), which is the K-major
-// operand layout without swizzle; each is one contiguous bulk copy per step.
+// Delta, dDelta, h and dh' arrive in the blocked layout the chain kernels keep
+// them in (per 32-column slice: 8-column blocks of 16-byte rows), each one
+// contiguous bulk copy per step; h, dh' and Delta are read as K-major operands
+// without swizzle, dDelta as an MN-major one.
 // Each input tile of the next step is loaded by TMA as soon as the current
 // step is done with its buffer (Ainv and dDelta after product round 1, dO after
 // product round 2, h and dh' after product round 3; Delta has two buffers), so that only a new
