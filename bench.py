@@ -127,12 +127,12 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639905536 + 119271680,
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639742464 + 119971328,
                sources=["gdn_bwd_grad.cu"],
-               sha256="9c445f906f00d11b8b9a477e3088567f1a89c86c4e970f0a174b9f8557a5a85e"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 167724544,
+               sha256="e20c7c69f537e473cda690e7d19391ff9b29cb235fb9747b1424ccc8358afef3"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 170267136,
                sources=["gdn_bwd_dh.cu"],
-               sha256="7b3bee60d740f4a86890b88a113f9935853013967a03f843e91efbff6e9b84c8"),
+               sha256="50e3d6d340b3e3f019b4e41e0f12a896b571cc3ec4935feb264aded684b8130c"),
     "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303088896 + 230655744,
                sources=["gdn_fwd2.cu"],
                sha256="bc5af0eeb7db80640505b8f0a1593de1399503b8526b8dee7019091daa9fd905"),
