@@ -217,6 +217,28 @@ class Clocks:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+def rank_workload(w, rank):
+    """Each rank runs its own independent batch (weak scaling, no collective on the
+    data path): the workload's shape, its seed offset by the rank."""
+    from gated_deltanet_chunked_rule_b200.inputs import scaled
+    return scaled(w, seed=w.seed + rank, grads=True)
+
+
+def slowest_ms(total_ms, dist=None, device="cpu"):
+    """The job's time: the slowest rank's device time (max over ranks)."""
+    if dist is None:
+        return total_ms
+    import torch
+    t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_mtokens_s(tokens_per_rank, world, steps, total_ms):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms * 1e-3) / 1e6
+
+
 def dist_setup():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -388,7 +410,7 @@ def main():
                                 device_id=dev)
     gdn.lib()  # fail loudly if the extension is missing
 
-    wr = scaled(w, seed=w.seed + rank, grads=True)
+    wr = rank_workload(w, rank)
     xh = make_inputs(wr)
     x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in xh.items()}
     cu_host = xh["cu_seqlens"]
@@ -447,15 +469,11 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms = sum(ms_list)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = slowest_ms(sum(ms_list), dist, dev)
     alg = algorithmic(w)
     tokens = alg["tokens"]
     ms_step = total_ms / args.steps
-    value = tokens * world * args.steps / (total_ms * 1e-3) / 1e6
+    value = job_mtokens_s(tokens, world, args.steps, total_ms)
 
     # Per-kernel device times: a second pass of the same steps with the library's
     # event timing on (events on the launch stream around every launch).
@@ -521,13 +539,9 @@ def main():
         e2e_step()
     torch.cuda.synchronize()
     e2e_ms = timed_steps(args.steps, e2e_step)
-    e2e_total = sum(e2e_ms)
-    if dist:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = slowest_ms(sum(e2e_ms), dist, dev)
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e = {"value": tokens * world * args.steps / (e2e_total * 1e-3) / 1e6, "unit": "Mtokens/s",
+    e2e = {"value": job_mtokens_s(tokens, world, args.steps, e2e_total), "unit": "Mtokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     status = gdn.device_status()
