@@ -103,6 +103,19 @@ def test_invalid_problems_rejected_before_any_launch(L, kw, code):
     assert rc == code
     assert L.gdn_chunk_fwd(None, dummy, dummy, dummy, dummy, dummy, None, dummy, None, None,
                            dummy, 0, None) == B.GDN_ERR_INVALID_ARG
+    # the decode step validates the same problem description
+    assert L.gdn_recurrent_fwd(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy, None, dummy, None,
+                               None) == code
+
+
+def test_decode_step_null_and_misaligned_pointers_rejected(L):
+    p = prob()
+    d = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    assert L.gdn_recurrent_fwd(None, d, d, d, d, d, None, d, None, None) == B.GDN_ERR_INVALID_ARG
+    assert L.gdn_recurrent_fwd(ctypes.byref(p), d, d, d, d, d, None, None, None, None) == B.GDN_ERR_INVALID_ARG  # o
+    assert L.gdn_recurrent_fwd(ctypes.byref(p), bad, d, d, d, d, None, d, None, None) == B.GDN_ERR_INVALID_ARG
+    assert L.gdn_recurrent_fwd(ctypes.byref(p), d, d, d, d, d, bad, d, None, None) == B.GDN_ERR_INVALID_ARG  # h0
 
 
 def test_null_and_misaligned_pointers_rejected(L):
