@@ -282,8 +282,10 @@ def run_reference(args, w):
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": sample_T, "Hq": w.Hq, "Hv": w.Hv,
-                   "K": w.K, "V": w.V, "step": "fwd" if args.fwd_only else "fwd+bwd"},
+        # the same workload as the CUDA arm's line; each step times a bounded sample of
+        # it (cpu_baseline.sample), and the value is the sample's tokens over its time
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hv": w.Hv,
+                   "K": w.K, "V": w.V, "chunk": CHUNK, "step": "fwd" if args.fwd_only else "fwd+bwd"},
         "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
