@@ -132,7 +132,7 @@ NCU_TRAFFIC = {
                sha256="e20c7c69f537e473cda690e7d19391ff9b29cb235fb9747b1424ccc8358afef3"),
     "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 170267136,
                sources=["gdn_bwd_dh.cu"],
-               sha256="50e3d6d340b3e3f019b4e41e0f12a896b571cc3ec4935feb264aded684b8130c"),
+               sha256="ca66ab3574fc215bf4fee7b29431bcb20e89949c8d939b5fe71680a0560c0f0a"),
     "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303088896 + 230655744,
                sources=["gdn_fwd2.cu"],
                sha256="bc5af0eeb7db80640505b8f0a1593de1399503b8526b8dee7019091daa9fd905"),

@@ -9,8 +9,10 @@
 //
 // (the adjoint of Delta = u - w h, o = scale (diag(e^gamma) Q h + (M o Q K^T) Delta),
 // h' = e^{gamma_C} h + K^T diag(e^{gamma_C - gamma}) Delta). Every chunk's dh'
-// (bf16, [NC, Hv, K, V]) and dDelta (bf16, [T, Hv, V]) are stored for the
-// per-chunk gradient kernel; dh0 (fp32) is the gradient at the sequence start.
+// and dDelta (bf16) are stored for the per-chunk gradient kernel in the blocked
+// tile layout, one contiguous block per (chunk, value head, 32-column slice):
+// dh' [NC][Hv][V/32][4][128][8], dDelta [NC][Hv][V/32][4][64][8]; dh0 (fp32) is
+// the gradient at the sequence start.
 //
 // Same organisation as the forward kernel (gdn_fwd2.cu): one CTA per
 // (sequence, value head, 32-column slice of V), w and P = M o Q K^T of every
