@@ -141,7 +141,7 @@ NCU_TRAFFIC = {
                sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),
     "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=138346240 + 213746944,
                sources=["gdn_prep3.cu"],
-               sha256="b5dd7e87c61c371614b692c11337e75c054daa97a1882d85b439c6cbf85f0945"),
+               sha256="d5112d7d5b5bdabaae238225b67aafbcc81991cccfd568afff397ea44998cf48"),
 }
 TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
 
