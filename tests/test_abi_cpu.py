@@ -134,3 +134,26 @@ def test_null_and_misaligned_pointers_rejected(L):
                            None) == B.GDN_ERR_WORKSPACE
     assert L.gdn_chunk_fwd(ctypes.byref(p), d, d, d, d, d, None, d, None, None,
                            ctypes.c_void_p((1 << 20) + 16), ws, None) == B.GDN_ERR_WORKSPACE
+
+
+def test_sequence_split_scratch_in_both_workspaces(L, monkeypatch):
+    # With S segments the forward and the backward's reverse scan each need the split scratch:
+    # per segment and value head, c or r (K x V), the K x K operator and the
+    # composed start / end state (K x V), fp32, 256-byte aligned.
+    p = prob(T=1024)  # 16 chunks per sequence
+    monkeypatch.setenv("GDN_NSEG", "1")
+    f1, b1 = L.gdn_fwd_workspace_size(ctypes.byref(p)), L.gdn_bwd_workspace_size(ctypes.byref(p))
+    monkeypatch.setenv("GDN_NSEG", "4")
+    f4, b4 = L.gdn_fwd_workspace_size(ctypes.byref(p)), L.gdn_bwd_workspace_size(ctypes.byref(p))
+    monkeypatch.delenv("GDN_NSEG")
+    scratch = 4 * 1 * 4 * 128 * (2 * 128 + 128) * 4  # nseg * N * Hv * K * (2V + K) floats
+    scratch = (scratch + 255) // 256 * 256
+    assert f4 - f1 == scratch
+    # the backward's size is the larger of the CUDA-core and tensor-core layouts (either
+    # path may run); the split scratch is part of the tensor-core one, so it never shrinks
+    assert b4 >= b1 and b4 >= scratch
+    # the saved buffer does not depend on the split
+    monkeypatch.setenv("GDN_NSEG", "4")
+    s4 = L.gdn_saved_size(ctypes.byref(p))
+    monkeypatch.delenv("GDN_NSEG")
+    assert s4 == L.gdn_saved_size(ctypes.byref(p))
