@@ -129,7 +129,7 @@ def kernel_bytes(name, w, saved=False):
 NCU_TRAFFIC = {
     "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639742464 + 119971328,
                sources=["gdn_bwd_grad.cu"],
-               sha256="e20c7c69f537e473cda690e7d19391ff9b29cb235fb9747b1424ccc8358afef3"),
+               sha256="d950affb8ccbca052df0113665b5b83ac2259302e965a6acd032a926380a5a35"),
     "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 170267136,
                sources=["gdn_bwd_dh.cu"],
                sha256="ca66ab3574fc215bf4fee7b29431bcb20e89949c8d939b5fe71680a0560c0f0a"),

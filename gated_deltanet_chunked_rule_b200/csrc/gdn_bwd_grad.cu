@@ -24,7 +24,7 @@
 // on chip and written once, in bf16: dk stays in tensor memory (the next
 // head's T1^T Q product accumulates onto it), dq is parked in spare columns.
 // All twelve products of a step run on tcgen05 from 128-byte-swizzled
-// shared-memory tiles, in three product rounds:
+// shared-memory tiles, in three product batches:
 //   1. S = QK^T, G = KK^T, P1 = dO Delta^T, dU = Ainv^T dDelta
 //   2. dAkk, T1 K, T1^T Q (onto dk), dO h^T
 //   3. dU h^T, Delta dh'^T, and dG K + dG^T K onto dk
@@ -38,8 +38,8 @@
 // contiguous bulk copy per step; h, dh' and Delta are read as K-major operands
 // without swizzle, dDelta as an MN-major one.
 // Each input tile of the next step is loaded by TMA as soon as the current
-// step is done with its buffer (Ainv and dDelta after product round 1, dO after
-// product round 2, h and dh' after product round 3; Delta has two buffers), so that only a new
+// step is done with its buffer (Ainv and dDelta after product batch 1, dO after
+// product batch 2, h and dh' after product batch 3; Delta has two buffers), so that only a new
 // item's k tile waits on memory. dv, dq and dk of a full chunk are written by
 // TMA stores from shared memory: dv in place of v, dq in place of q, dk in
 // the T1 | dG tiles; a ragged chunk is written row by row.
@@ -66,8 +66,8 @@ constexpr int kJJ = 64 / kWN / 8;   // 8-column tiles of a C x C accumulator per
 constexpr int kParts = 128 / kWN / 32;  // 32-column loads of a C x K accumulator per warp
 constexpr int C = 64, K = 128, V = 128;
 constexpr int kStoreTid = 32;  // issues the TMA stores and the loads of the buffers they read
-// The products of a round are issued by two threads (thread 0 and kStoreTid), each
-// committing to the round's mbarrier (two arrivals): a single issuing thread spends
+// The products of a batch are issued by two threads (thread 0 and kStoreTid), each
+// committing to the batch's mbarrier (two arrivals): a single issuing thread spends
 // about 70 cycles per tcgen05.mma.
 
 // ---- shared memory (bytes from a 1024-aligned base); [64][128] tiles are two
@@ -88,9 +88,9 @@ constexpr int kBar = kVec + 4096;
 constexpr int kSmemBytes = kBar + 128 + 1024;
 static_assert(kdG == kT1 + 8192 && kSmemBytes <= 232448, "shared memory layout");
 
-// tensor memory columns: product round 1  S, G, P1, dU;
-// product round 2  dAkk, T1 K, dk (T1^T Q), dO h^T;
-// product round 3  dU h^T, Delta dh'^T, dk (+ dG K + dG^T K). dk lives at kCDK for the whole
+// tensor memory columns: product batch 1  S, G, P1, dU;
+// product batch 2  dAkk, T1 K, dk (T1^T Q), dO h^T;
+// product batch 3  dU h^T, Delta dh'^T, dk (+ dG K + dG^T K). dk lives at kCDK for the whole
 // item; dq is parked at kCPark between the heads of an item (column quarter w / 4 at
 // lanes 16 ((w / 4) % 2).. of the warp's sub-partition, columns 32 ((w / 4) / 2)..).
 constexpr uint32_t kCS = 0, kCG = 64, kCP1 = 128, kCU = 320;
@@ -98,7 +98,7 @@ constexpr uint32_t kCAkk = 0, kCTK = 64, kCDK = 192, kCQ1 = 320;
 constexpr uint32_t kCKb = 0, kCK2 = 320, kCPark = 448;
 constexpr uint32_t kTmemCols = 512;
 
-// mbarriers: one per load group, and one for the rounds of MMAs
+// mbarriers: one per load group, and one for the batches of MMAs
 enum Bar { kBarQ, kBarK, kBarD0, kBarD1, kBarDO, kBarA, kBarV, kBarSt, kBarMma, kNumBar };
 
 struct Vecs {
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         const bool first = cur.g == 0, last = cur.g == G - 1, full = len == C;
         const uint32_t sD = sb + kD + db * 16384;
 
-        // Delta of the next step into the other buffer (its last reader, product round 3 of the
+        // Delta of the next step into the other buffer (its last reader, product batch 3 of the
         // previous step, has completed)
         if (tid == 0 && nxt.valid) load_delta(nxt, db ^ 1);
         if (tid < C) {
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         ok = ok && (!first || (wait_bar(kBarQ) && wait_bar(kBarK))) && wait_bar(kBarD0 + db) &&
              wait_bar(kBarDO) && wait_bar(kBarA);
 
-        // ---- product round 1: S, G, P1 (64 x 64) and dU (64 x 128)
+        // ---- product batch 1: S, G, P1 (64 x 64) and dU (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false);
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         if (ok && tid == 0 && nxt.valid) load_a(nxt);  // Ainv and dDelta are consumed
         ok = ok && wait_bar(kBarV);
 
-        float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for product round 2
+        float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for product batch 2
         if (ok) {
             float v[16], pacc[kJJ][4];
             {
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         }
         ok = wait_bar(kBarSt);
 
-        // ---- product round 2: dAkk (64 x 64), T1 K, T1^T Q onto dk, dO h^T (64 x 128)
+        // ---- product batch 2: dAkk (64 x 64), T1 K, T1^T Q onto dk, dO h^T (64 x 128)
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t idCC = idesc_bf16(64, 64, false, false), idKM = idesc_bf16(64, 128, false, true);
@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         ok = __syncthreads_and(ok);
         if (!ok) break;
 
-        // ---- product round 3: dU h^T, Delta dh'^T; dG K + dG^T K onto dk
+        // ---- product batch 3: dU h^T, Delta dh'^T; dG K + dG^T K onto dk
         if (tid == 0) {
             tc_fence_after();
             const uint32_t idKK = idesc_bf16(64, 128, false, false);
