@@ -157,3 +157,30 @@ def test_sequence_split_scratch_in_both_workspaces(L, monkeypatch):
     s4 = L.gdn_saved_size(ctypes.byref(p))
     monkeypatch.delenv("GDN_NSEG")
     assert s4 == L.gdn_saved_size(ctypes.byref(p))
+
+
+@pytest.mark.parametrize("T,Hq,Hv,expect", [
+    (8192, 16, 32, 1),   # 128 chain CTAs fill one wave of 148 SMs: no split
+    (8192, 8, 16, 1),    # 64 CTAs: splitting would need 3 waves of 64-chunk segments
+    (8192, 4, 8, 4),     # 32 CTAs: 4 segments, 2 + 1 waves of 32 chunks beat 128 steps
+    (65536, 8, 8, 4),    # 32 CTAs over 1024 chunks: 4 segments of 256
+    (1024, 1, 1, 1),     # 16 chunks: S = 2 would cost 2 x 8 + 3 = 19 steps > 16
+    (1536, 1, 1, 3),     # 24 chunks: S = 3 costs 2 x 8 + 4.5 = 20.5 < 0.9 x 24
+    (448, 1, 1, 1),      # 7 chunks: too short to split
+])
+def test_segment_count_from_wave_model(L, monkeypatch, T, Hq, Hv, expect):
+    # The automatic segment count (bf16, K = V = 128) on a 148-SM part: the estimate
+    # is ceil(CTAs / SMs) * chunks unsplit, and for S segments ceil(2 CTAs S / SMs) +
+    # ceil(CTAs S / SMs) waves of ceil(chunks / S) steps plus 1.5 steps per composed
+    # segment; a count is taken only if it beats the best so far by 10 %. The expected
+    # counts above are worked out by hand from that estimate. The count shows in the
+    # forward workspace as the split scratch it adds.
+    monkeypatch.delenv("GDN_NSEG", raising=False)
+    p = prob(T=T, Hq=Hq, Hv=Hv)
+    auto = L.gdn_fwd_workspace_size(ctypes.byref(p))
+    monkeypatch.setenv("GDN_NSEG", "1")
+    base = L.gdn_fwd_workspace_size(ctypes.byref(p))
+    monkeypatch.delenv("GDN_NSEG")
+    per_seg = Hv * 128 * (2 * 128 + 128) * 4
+    scratch = (expect * per_seg + 255) // 256 * 256 if expect > 1 else 0
+    assert auto - base == scratch
