@@ -42,10 +42,18 @@ class Problem:
     """Host-side description of one call (gdn_problem plus the cu_seqlens copies)."""
 
     def __init__(self, q, v, scale, cu_seqlens=None, cu_seqlens_host=None):
+        if q.dim() != 4 or v.dim() != 4:
+            raise ValueError(f"q and v must be [B, T, H, D], got {tuple(q.shape)} and {tuple(v.shape)}")
         B, T, Hq, K = q.shape
         Hv, V = v.shape[2], v.shape[3]
         if q.dtype not in _DTYPES:
             raise TypeError(f"unsupported dtype {q.dtype}")
+        if cu_seqlens is not None:
+            if cu_seqlens.dim() != 1 or cu_seqlens.dtype not in (torch.int32, torch.int64):
+                raise ValueError("cu_seqlens must be a 1-D integer tensor")
+            if cu_seqlens_host is not None and (cu_seqlens_host.device.type != "cpu"
+                                                or cu_seqlens_host.shape != cu_seqlens.shape):
+                raise ValueError("cu_seqlens_host must be a CPU copy of cu_seqlens")
         self.cu_dev = None
         self.cu_host = None
         num_seqs = 0
@@ -79,6 +87,46 @@ def _c(x):
     return None if x is None else x.contiguous()
 
 
+def _check(P: Problem, dev, *, q, k, v, g, beta, h0=None, out=None, final=None, do=None, dht=None,
+           saved=None, workspace=None):
+    """Every tensor the library will read or write through a raw pointer: on the
+    CUDA device of q, with the shape and dtype the C ABI expects for this problem.
+    The kernels trust these sizes, so nothing else guards against a short buffer."""
+    if dev.type != "cuda":
+        raise ValueError(f"inputs must be CUDA tensors (got {dev}); the library has no CPU path")
+    _check_tensors(P, dev, q=q, k=k, v=v, g=g, beta=beta, h0=h0, out=out, final=final, do=do, dht=dht,
+                   saved=saved, workspace=workspace)
+
+
+def _check_tensors(P: Problem, dev, *, q, k, v, g, beta, h0=None, out=None, final=None, do=None,
+                   dht=None, saved=None, workspace=None):
+    B, T, Hq, Hv, K, V = P.shape
+    state = (P.N, Hv, K, V)
+    want = {
+        "q": (q, (B, T, Hq, K), q.dtype), "k": (k, (B, T, Hq, K), q.dtype),
+        "v": (v, (B, T, Hv, V), q.dtype), "g": (g, (B, T, Hv), torch.float32),
+        "beta": (beta, (B, T, Hv), torch.float32), "initial_state": (h0, state, torch.float32),
+        "out": (out, (B, T, Hv, V), q.dtype), "final_state": (final, state, torch.float32),
+        "do": (do, (B, T, Hv, V), q.dtype), "dht": (dht, state, torch.float32),
+        "saved": (saved, None, torch.uint8), "workspace": (workspace, None, torch.uint8),
+    }
+    for name, (t, shape, dtype) in want.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+        if shape is not None and tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if shape is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if saved is not None and saved.numel() < P.saved_size():
+        raise ValueError(f"saved holds {saved.numel()} bytes, the problem needs {P.saved_size()}")
+
+
 def chunk_gated_delta_rule_fwd(q, k, v, g, beta, scale, initial_state=None,
                                output_final_state=True, cu_seqlens=None, cu_seqlens_host=None,
                                save_for_backward=False, workspace=None, out=None):
@@ -91,15 +139,17 @@ def chunk_gated_delta_rule_fwd(q, k, v, g, beta, scale, initial_state=None,
     P = Problem(q, v, scale, cu_seqlens, cu_seqlens_host)
     B, T, Hq, Hv, K, V = P.shape
     dev = q.device
+    _check(P, dev, q=q, k=k, v=v, g=g, beta=beta, h0=h0, out=out, workspace=workspace)
     o = out if out is not None else torch.empty((B, T, Hv, V), dtype=q.dtype, device=dev)
     fin = torch.empty((P.N, Hv, K, V), dtype=torch.float32, device=dev) if output_final_state else None
     saved = torch.empty(P.saved_size(), dtype=torch.uint8, device=dev) if save_for_backward else None
     ws_bytes = P.fwd_workspace_size()
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = _b.lib().gdn_chunk_fwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                _ptr(o), _ptr(fin), _ptr(saved), _ptr(workspace),
-                                workspace.numel(), _stream(dev))
+    with torch.cuda.device(dev):
+        rc = _b.lib().gdn_chunk_fwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                    _ptr(o), _ptr(fin), _ptr(saved), _ptr(workspace),
+                                    workspace.numel(), _stream(dev))
     _b.check("gdn_chunk_fwd", rc)
     return o, fin, saved
 
@@ -115,6 +165,7 @@ def chunk_gated_delta_rule_bwd(q, k, v, g, beta, saved, do, dht=None, scale=None
     P = Problem(q, v, scale, cu_seqlens, cu_seqlens_host)
     B, T, Hq, Hv, K, V = P.shape
     dev = q.device
+    _check(P, dev, q=q, k=k, v=v, g=g, beta=beta, h0=h0, do=do, dht=dht, saved=saved, workspace=workspace)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
@@ -124,10 +175,11 @@ def chunk_gated_delta_rule_bwd(q, k, v, g, beta, saved, do, dht=None, scale=None
     ws_bytes = P.bwd_workspace_size()
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = _b.lib().gdn_chunk_bwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                _ptr(saved), _ptr(do), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv),
-                                _ptr(dg), _ptr(dbeta), _ptr(dh0), _ptr(workspace),
-                                workspace.numel(), _stream(dev))
+    with torch.cuda.device(dev):
+        rc = _b.lib().gdn_chunk_bwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                    _ptr(saved), _ptr(do), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv),
+                                    _ptr(dg), _ptr(dbeta), _ptr(dh0), _ptr(workspace),
+                                    workspace.numel(), _stream(dev))
     _b.check("gdn_chunk_bwd", rc)
     return dq, dk, dv, dbeta, dg, dh0
 
@@ -143,11 +195,13 @@ def recurrent_gated_delta_rule(q, k, v, g, beta, scale=None, initial_state=None,
     P = Problem(q, v, scale, cu_seqlens, cu_seqlens_host)
     B, T, Hq, Hv, K, V = P.shape
     dev = q.device
+    _check(P, dev, q=q, k=k, v=v, g=g, beta=beta, h0=h0, out=out, final=final_state)
     o = out if out is not None else torch.empty((B, T, Hv, V), dtype=q.dtype, device=dev)
     if final_state is None:
         final_state = torch.empty((P.N, Hv, K, V), dtype=torch.float32, device=dev)
-    rc = _b.lib().gdn_recurrent_fwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                    _ptr(o), _ptr(final_state), _stream(dev))
+    with torch.cuda.device(dev):
+        rc = _b.lib().gdn_recurrent_fwd(P.ref(), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                        _ptr(o), _ptr(final_state), _stream(dev))
     _b.check("gdn_recurrent_fwd", rc)
     return o, final_state
 
