@@ -17,7 +17,9 @@
  *     dq, dk, dv, db, dg, dh0);
  *   - the automatic intra-GPU sequence split inside gdn_chunk_fwd is the
  *     "gate-driven automatic intra-card context parallelism" of page 2
- *     ("三大关键特性" table, first row), realised exactly (no truncation).
+ *     ("三大关键特性" table, first row), realised exactly (no truncation);
+ *     gdn_chunk_bwd splits its reverse state-gradient scan the same way, with
+ *     the same segment count for the same problem.
  *
  * Layouts (contiguous, row-major, device memory unless stated):
  *   q, k        [B, T, Hq, K]   dtype (GDN_DTYPE_F32 or GDN_DTYPE_BF16)
@@ -38,7 +40,10 @@
  *
  * Supported sizes: K, V in {64, 128}; Hv a multiple of Hq; T >= 0; B >= 1.
  *
- * Ownership and synchronisation: every pointer is caller-owned. The library
+ * Ownership and synchronisation: every pointer is caller-owned; the problem
+ * description and cu_seqlens_host are host memory, everything else is device
+ * memory on the current device (a host pointer there is not detected and
+ * faults the kernels, so bindings must check it). The library
  * never allocates, frees or synchronises (except gdn_get_device_status); it
  * enqueues its kernels on the caller's stream and keeps no state between
  * calls other than the device status word. Scratch memory comes from the
@@ -178,9 +183,10 @@ int gdn_get_device_status(void *stream /* cudaStream_t */);
  * JSON object {"<kernel>": [launches, total_ms], ...} covering every launch
  * since the last enable/reset, and returns the number of bytes needed
  * (excluding the terminating NUL; the output is truncated if buf_len is too
- * small), or minus a gdn_status code on failure. Enabling clears earlier records. The events come from a pool the
- * library creates on first use; it holds no device memory. Timing changes
- * nothing in the results; it adds a few microseconds per launch. */
+ * small), or minus a gdn_status code on failure. Enabling clears earlier
+ * records. The events come from a pool the library creates on first use; it
+ * holds no device memory. Timing changes nothing in the results; it adds a few
+ * microseconds per launch. */
 int gdn_timing_enable(int on);
 int gdn_timing_report(char *buf, size_t buf_len);
 
