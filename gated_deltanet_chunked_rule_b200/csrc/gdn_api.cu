@@ -287,11 +287,12 @@ void set_saved_ptrs(FwdArgs &a, char *sv, const Plan &P, bool with_states) {
     }
 }
 
-// Either backward path fits in the size reported to callers.
-size_t bwd_ws_bytes(const Plan &P) {
-    const size_t a = bwd_layout(P).total, b = P.tc_ok ? tc_bwd_layout(P).total : 0;
-    return a > b ? a : b;
-}
+// The size reported to callers is that of the path the call takes: the
+// tensor-core layout (bf16 states) for bf16 K = V = 128, the CUDA-core layout
+// (fp32 states and partials, about twice as large) otherwise or under
+// GDN_IMPL=simt. A call whose workspace is smaller than its path needs is
+// refused with GDN_ERR_WORKSPACE before anything is enqueued.
+size_t bwd_ws_bytes(const Plan &P) { return tc_bwd_path(P) ? tc_bwd_layout(P).total : bwd_layout(P).total; }
 
 // Builds the sequence table from the device copy of cu_seqlens and checks it
 // against the host plan (total tokens, total chunks). On any disagreement it

@@ -58,6 +58,30 @@ def saved_bf16_k128(ntok, nc, Hv=4, K=128, V=128):
             + nc * Hv * 64 * 64 * 2 + nc * Hv * K * V * 2 + nc * 64 * Hv * V * 2)
 
 
+def test_backward_workspace_is_the_running_paths(L, monkeypatch):
+    # bf16, K = V = 128, T = 256 (4 chunks), Hv = 4: the tensor-core backward needs the
+    # forward's core buffers (gamma | Ainv | w | u | P, for the no-saved recompute), then bf16
+    # chunk entry states and exit-state gradients, then bf16 Delta and dDelta
+    monkeypatch.delenv("GDN_IMPL", raising=False)
+    monkeypatch.delenv("GDN_NSEG", raising=False)
+    p = prob()
+    nc, Hv, K, V, T = 4, 4, 128, 128, 256
+    core = T * Hv * 4 + nc * Hv * 64 * 64 * 2 + T * Hv * K * 2 + T * Hv * V * 4 + nc * Hv * 64 * 64 * 2
+    tc = core + 2 * nc * Hv * K * V * 2 + 2 * nc * 64 * Hv * V * 2
+    assert L.gdn_bwd_workspace_size(ctypes.byref(p)) == tc
+    # the CUDA-core path (forced) keeps fp32 states, Delta, dDelta and dq, dk partials
+    monkeypatch.setenv("GDN_IMPL", "simt")
+    simt = core + 2 * nc * Hv * K * V * 4 + 2 * T * Hv * V * 4 + 2 * T * Hv * K * 4
+    assert L.gdn_bwd_workspace_size(ctypes.byref(p)) == simt
+    monkeypatch.delenv("GDN_IMPL")
+    # a workspace sized for one path is refused by the other before anything is enqueued
+    d = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 24)
+    monkeypatch.setenv("GDN_IMPL", "simt")
+    assert L.gdn_chunk_bwd(ctypes.byref(p), d, d, d, d, d, None, None, d, None, d, d, d, d, d, None,
+                           ws, ctypes.c_size_t(tc), None) == B.GDN_ERR_WORKSPACE
+
+
 def test_workspace_sizes(L):
     p = prob()
     nc = 4  # 256 tokens -> 4 chunks
@@ -149,9 +173,8 @@ def test_sequence_split_scratch_in_both_workspaces(L, monkeypatch):
     scratch = 4 * 1 * 4 * 128 * (2 * 128 + 128) * 4  # nseg * N * Hv * K * (2V + K) floats
     scratch = (scratch + 255) // 256 * 256
     assert f4 - f1 == scratch
-    # the backward's size is the larger of the CUDA-core and tensor-core layouts (either
-    # path may run); the split scratch is part of the tensor-core one, so it never shrinks
-    assert b4 >= b1 and b4 >= scratch
+    # the backward's size is that of the tensor-core path, which holds the same scratch
+    assert b4 - b1 == scratch
     # the saved buffer does not depend on the split
     monkeypatch.setenv("GDN_NSEG", "4")
     s4 = L.gdn_saved_size(ctypes.byref(p))
