@@ -17,7 +17,10 @@ or index, or a transposed operand in the oracle fails at least one of them:
 * linearity in (v, h0); varlen and batch rows equal separate calls; GQA equals
   explicitly repeated q/k heads;
 * gradients: scalar closed forms, beta=0 closed forms, central finite
-  differences of every input, random-direction adjoint identities.
+  differences of every input, random-direction adjoint identities;
+* the dense unrolling and the adjoint identity again over randomly drawn shapes
+  (hypothesis): batch or packed sequences with empty ones, T = 0, group sizes
+  1-3, any K, V in 1..5.
 """
 import json
 import math
@@ -361,6 +364,64 @@ def test_gradients_adjoint_identity_random_direction(oracle_mod):
         lp = loss(oracle_mod, xp, 0.4, d_o, dht)
         xp[name] = x[name] - eps * dx
         lm = loss(oracle_mod, xp, 0.4, d_o, dht)
+        fd = (lp - lm) / (2 * eps)
+        an = float(np.sum(r[gname] * dx))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+# ------------------------------------------------------------------ random shapes
+
+from hypothesis import HealthCheck, given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@st.composite
+def shapes(draw):
+    Hq = draw(st.integers(1, 2))
+    G = draw(st.integers(1, 3))
+    K, V = draw(st.integers(1, 5)), draw(st.integers(1, 5))
+    varlen = draw(st.booleans())
+    if varlen:
+        lens = draw(st.lists(st.integers(0, 6), min_size=1, max_size=4))
+        return dict(B=1, T=sum(lens), Hq=Hq, Hv=Hq * G, K=K, V=V,
+                    cu=np.concatenate([[0], np.cumsum(lens)]).astype(np.int32))
+    return dict(B=draw(st.integers(1, 2)), T=draw(st.integers(0, 9)), Hq=Hq, Hv=Hq * G, K=K, V=V, cu=None)
+
+
+@settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(shapes(), st.integers(0, 2**31 - 1), st.floats(0.1, 2.0))
+def test_fwd_matches_dense_unrolling_random_shapes(oracle_mod, s, seed, scale):
+    # any batch / packing, group size, K != V, empty sequences and T = 0 included
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, _ = rand_problem(rng, B=s["B"], T=s["T"], Hq=s["Hq"], Hv=s["Hv"], K=s["K"],
+                                       V=s["V"], h0=False)
+    N = s["B"] if s["cu"] is None else len(s["cu"]) - 1
+    h0 = rng.standard_normal((N, s["Hv"], s["K"], s["V"])) * 0.5
+    o, fin = oracle_mod.fwd(q, k, v, g, beta, scale, h0=h0, cu_seqlens=s["cu"])
+    o_ref, fin_ref = unrolled(q, k, v, g, beta, scale, h0=h0, cu=s["cu"])
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(fin, fin_ref, rtol=1e-10, atol=1e-11)
+
+
+@settings(max_examples=25, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(shapes(), st.integers(0, 2**31 - 1))
+def test_gradients_adjoint_identity_random_shapes(oracle_mod, s, seed):
+    # <grad L, dx> equals the central difference of L along a random dx, for every input
+    rng = np.random.default_rng(seed)
+    q, k, v, g, beta, _ = rand_problem(rng, B=s["B"], T=s["T"], Hq=s["Hq"], Hv=s["Hv"], K=s["K"],
+                                       V=s["V"], h0=False)
+    N = s["B"] if s["cu"] is None else len(s["cu"]) - 1
+    h0 = rng.standard_normal((N, s["Hv"], s["K"], s["V"])) * 0.5
+    x = dict(q=q, k=k, v=v, g=g, beta=beta, h0=h0)
+    o, fin = oracle_mod.fwd(q, k, v, g, beta, 0.6, h0=h0, cu_seqlens=s["cu"])
+    d_o, dht = rng.standard_normal(o.shape), rng.standard_normal(fin.shape)
+    r = oracle_mod.bwd(q, k, v, g, beta, 0.6, d_o, dht=dht, h0=h0, cu_seqlens=s["cu"])
+    for name, gname in dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", h0="dh0").items():
+        assert r[gname].shape == x[name].shape, gname
+        dx = rng.standard_normal(x[name].shape)
+        eps = 1e-6
+        lp = loss(oracle_mod, {**x, name: x[name] + eps * dx}, 0.6, d_o, dht, s["cu"])
+        lm = loss(oracle_mod, {**x, name: x[name] - eps * dx}, 0.6, d_o, dht, s["cu"])
         fd = (lp - lm) / (2 * eps)
         an = float(np.sum(r[gname] * dx))
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
