@@ -1,8 +1,8 @@
 """fp64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
 
 This package is the independent checker for the CUDA library. Only the tests,
-``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
-it. It shares no code with the CUDA path and must never be used to produce a
+``__graft_entry__.smoke()`` and the CPU-baseline and reference legs of
+``bench.py`` (both time this oracle on the host cores) may import it. It shares no code with the CUDA path and must never be used to produce a
 product result.
 
 The arithmetic lives in ``gdn_oracle.c`` (plain C, fp64, token by token):

@@ -3,8 +3,8 @@
  *
  * TEST INFRASTRUCTURE ONLY. This file is the independent checker that the
  * CUDA path is compared against. It shares no code, header or table with the
- * CUDA library; only tests, the smoke check and the bench's CPU-baseline leg
- * may load it.
+ * CUDA library; only tests, the smoke check and the bench's CPU-baseline and
+ * reference legs (both time this oracle on the host cores) may load it.
  *
  * What it computes (token by token, no chunking, no reordering):
  *
