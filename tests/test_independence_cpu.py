@@ -52,3 +52,17 @@ def test_importing_and_using_the_package_loads_no_oracle():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
 
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    # with libgdn.so absent every entry point raises; nothing falls back to a CPU path
+    code = ("import gated_deltanet_chunked_rule_b200 as gdn\n"
+            "from gated_deltanet_chunked_rule_b200 import _binding as B\n"
+            f"B.LIB_PATH = {str(tmp_path / 'absent' / 'libgdn.so')!r}\n"
+            "try:\n"
+            "    gdn.lib()\n"
+            "except RuntimeError as e:\n"
+            "    assert 'missing' in str(e), e\n"
+            "    print('raised')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "raised", r.stdout + r.stderr
