@@ -224,14 +224,19 @@ def rank_workload(w, rank):
     return scaled(w, seed=w.seed + rank, grads=True)
 
 
-def slowest_ms(total_ms, dist=None, device="cpu"):
-    """The job's time: the slowest rank's device time (max over ranks)."""
+def max_over_ranks(x, dist=None, device="cpu"):
+    """x on this rank -> its maximum over all ranks (x itself with one rank)."""
     if dist is None:
-        return total_ms
+        return x
     import torch
-    t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+    t = torch.tensor([x], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def slowest_ms(total_ms, dist=None, device="cpu"):
+    """The job's time: the slowest rank's device time (max over ranks)."""
+    return max_over_ranks(total_ms, dist, device)
 
 
 def job_mtokens_s(tokens_per_rank, world, steps, total_ms):
@@ -546,9 +551,13 @@ def main():
     e2e = {"value": job_mtokens_s(tokens, world, args.steps, e2e_total), "unit": "Mtokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    status = gdn.device_status()
+    # every rank takes this collective, so a device error on one rank ends all of them
+    # here rather than leaving the others waiting at the next barrier
+    status = int(max_over_ranks(gdn.device_status(), dist, dev))
     if status != 0:
-        raise SystemExit(f"device status {status} after the bench")
+        if dist:
+            dist.destroy_process_group()
+        raise SystemExit(f"device status {status} after the bench (max over ranks)")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

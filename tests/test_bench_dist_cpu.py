@@ -39,11 +39,13 @@ def _rank(rank, world, port, out_dir):
         # this rank's own (deliberately different) device time
         mine = 3.0 + 2.0 * r
         job = bench.slowest_ms(mine, dist, "cpu")
+        # a device status seen on one rank only reaches every rank
+        status = int(bench.max_over_ranks(6 if r == 1 else 0, dist, "cpu"))
         value = bench.job_mtokens_s(w.B * w.T, ws, 4, job)
         dist.barrier()
         with open(os.path.join(out_dir, f"rank{r}.json"), "w") as f:
             json.dump({"rank": r, "local": local, "seed": wr.seed, "q_sum": float(x["q"].double().sum()),
-                       "job_ms": job, "value": value}, f)
+                       "job_ms": job, "value": value, "status": status}, f)
     finally:
         dist.destroy_process_group()
 
@@ -58,6 +60,7 @@ def test_two_gloo_ranks_time_max_and_independent_batches(tmp_path):
     assert res[0]["job_ms"] == res[1]["job_ms"] == pytest.approx(5.0)
     # whole-job throughput: both ranks' tokens over that time
     assert res[0]["value"] == pytest.approx(96 * 2 * 4 / 5.0e-3 / 1e6)
+    assert res[0]["status"] == res[1]["status"] == 6
     # independent batches: different seeds, different inputs
     assert res[0]["seed"] != res[1]["seed"] and res[0]["q_sum"] != res[1]["q_sum"]
 
