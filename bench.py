@@ -376,14 +376,18 @@ def run_decode(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="qwen_prefill_t8192_hv32")
-    ap.add_argument("--fwd-only", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=1024)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs in the job (one process per GPU under torchrun; N replicas)")
+    ap.add_argument("--steps", type=int, default=20, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
+                    help="reference: time the fp64 oracle on the host cores on a bounded sample")
+    ap.add_argument("--workload", default="qwen_prefill_t8192_hv32",
+                    help="one of the named synthetic workloads (inputs.py)")
+    ap.add_argument("--fwd-only", action="store_true", help="time the forward alone")
+    ap.add_argument("--ref-tokens", type=int, default=1024,
+                    help="tokens per row in the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--decode", action="store_true", help="time the token-by-token step instead")
     ap.add_argument("--heads", default=None, help="HQ,HV: override the workload's head counts (sweeps)")
     args = ap.parse_args()
