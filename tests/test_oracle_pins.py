@@ -10,7 +10,8 @@ or index, or a transposed operand in the oracle fails at least one of them:
 
 * brute-force dense unrolling (ordered products of the per-token transition
   matrices) on tiny inputs with K != V, random h0, unnormalised k;
-* a hand-worked three-token example (tests/golden/worked_example_k2v2.json);
+* hand-worked examples: three tokens forward (tests/golden/worked_example_k2v2.json)
+  and two tokens with every gradient (tests/golden/worked_example_grad_k1v1.json);
 * closed forms: constant-input scalar recurrence (geometric series), beta=0
   pure decay of h0, g=0 and beta=0 constant state, a reset when exp(g)
   underflows to 0, beta=1 with unit-norm k giving S_t k_t = v_t;
@@ -316,6 +317,24 @@ def test_beta_zero_gradients_closed_form(oracle_mod):
     np.testing.assert_allclose(r["dh0"][0, 0], dh0_ref, rtol=1e-11)
     np.testing.assert_array_equal(r["dv"], 0.0)
     np.testing.assert_array_equal(r["dk"], 0.0)
+
+
+def test_worked_gradient_example(oracle_mod):
+    # two tokens with K = V = 1, gradients derived by hand (tests/golden)
+    ex = json.load(open(os.path.join(HERE, "golden", "worked_example_grad_k1v1.json")))
+    x, e = ex["inputs"], ex["expected"]
+    col = lambda a: np.array(a, dtype=np.float64).reshape(1, -1, 1, 1)  # noqa: E731
+    g = np.log(np.array(x["decay"])).reshape(1, -1, 1)
+    beta = np.array(x["beta"]).reshape(1, -1, 1)
+    h0 = np.full((1, 1, 1, 1), x["h0"])
+    o, fin = oracle_mod.fwd(col(x["q"]), col(x["k"]), col(x["v"]), g, beta, x["scale"], h0=h0)
+    np.testing.assert_allclose(o.ravel(), e["o"], rtol=0, atol=ex["tolerance"])
+    np.testing.assert_allclose(fin.ravel(), [e["final_state"]], rtol=0, atol=ex["tolerance"])
+    r = oracle_mod.bwd(col(x["q"]), col(x["k"]), col(x["v"]), g, beta, x["scale"], col(x["do"]),
+                       dht=np.full((1, 1, 1, 1), x["dht"]), h0=h0)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dh0"):
+        np.testing.assert_allclose(r[name].ravel(), np.ravel(e[name]), rtol=0, atol=ex["tolerance"],
+                                   err_msg=name)
 
 
 @pytest.mark.parametrize("varlen", [False, True])
