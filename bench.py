@@ -135,7 +135,7 @@ NCU_TRAFFIC = {
                sha256="ca66ab3574fc215bf4fee7b29431bcb20e89949c8d939b5fe71680a0560c0f0a"),
     "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303088896 + 230655744,
                sources=["gdn_fwd2.cu"],
-               sha256="bc5af0eeb7db80640505b8f0a1593de1399503b8526b8dee7019091daa9fd905"),
+               sha256="9577197f9cc991b68c924b4cce99cacaadd3aacef535ded4fe595f62798731a1"),
     "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549451520 + 481462272,
                sources=["gdn_recurrent.cu"],
                sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),

@@ -15,10 +15,11 @@
 // Why this split (measured on B200): a tcgen05 MMA takes ~450 cycles from
 // issue to a completed mbarrier, and the chain has two dependent products per
 // chunk, whereas a dependent mma.sync costs ~20 cycles; the output products do
-// not feed the chain, so they run on tcgen05 off the critical path. Shared
-// memory bandwidth (128 B/clk/SM) is the next limit, which is why every
-// state-independent product is hoisted into the prep kernel, and why each
-// chain warp owns whole rows: the w and K^T fragments are read once per chunk.
+// not feed the chain, so they run on tcgen05 off the critical path. A chain
+// warp's shared-memory reads are limited by its own issue rate (one
+// ldmatrix.x4 per ~8.6 cycles), which is why every state-independent product
+// is hoisted into the prep kernel, and why each chain warp owns whole rows:
+// the w and K^T fragments are read once per chunk.
 //
 // Warp roles (320 threads):
 //   warps 0-3   chain: h (128 x 32 fp32) in mma fragments, warp p holding
@@ -28,7 +29,10 @@
 //               critical path only reads h and e^{gamma_C - gamma} Delta from
 //               shared memory. Two barriers per chunk.
 //   warps 4-7   epilogue: o from the double-buffered DQ/DP accumulators;
-//               warp 4 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15).
+//               warp 4 + q reads TMEM lanes 32 q .. +31 (rows 16 q .. +15),
+//               stages its rows of o in shared memory, and one TMA store per
+//               full chunk writes them (fewer stores beside the chain warps;
+//               a ragged last chunk is stored directly, row by row).
 //   warp 8      output issuer: the DQ/DP MMAs and the (q, P) TMA ring.
 //   warp 9      chain producer: the (k, w, u) TMA ring, refilled as soon as the
 //               chain has a stage in registers, and the bulk copies of the
