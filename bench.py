@@ -71,10 +71,71 @@ def algorithmic(w, tokens_per_seq=None):
     return dict(f_fwd=f_fwd, f_bwd=f_bwd, b_fwd=b_fwd, b_bwd=b_bwd, tokens=ntok)
 
 
+def kernel_work(name, w):
+    """Algorithmic work of one launch of a named kernel, by the rows of the hot
+    path it implements: (flops of the method's dense contractions in those
+    rows, bytes of the method's own inputs and outputs the kernel reads or
+    writes). Intermediates of this design (w, u, P, gamma, Ainv, chunk states,
+    Delta, dh', dDelta) are not counted: they are design bytes (kernel_bytes).
+
+    Flops per token (C = 64), split from the chain totals of algorithmic():
+      prep3 (gamma, A, Ainv, w, u):      Hq*4CK + Hv*(2CK + 2CV)
+      fwd_hybrid (chain + output):       Hv*(6KV + 2CV)
+      bwd_dh (reverse state scan):       Hv*(2CV + 6KV)
+      bwd_grad (per-chunk gradients):    Hq*4CK + Hv*(14CK + 8CV + 12KV + 4C^2)
+    so prep3 + fwd_hybrid = the forward and bwd_dh + bwd_grad = the backward.
+    Bytes: q, k [T,Hq,K], v, o, do, dv [T,Hv,V] in the input dtype, g, beta,
+    dg, dbeta [T,Hv] fp32, states h0, final, dht, dh0 [N,Hv,K,V] fp32, each
+    counted once for every kernel that touches it.
+    Returns None for a kernel without a row of its own (split composition,
+    recompute, plan)."""
+    C, K, V, Hq, Hv = CHUNK, w.K, w.V, w.Hq, w.Hv
+    ntok = w.B * w.T
+    N = w.varlen[0] if w.varlen else w.B
+    e = 2 if w.dtype == "bf16" else 4
+    qk1 = ntok * Hq * K * e        # q or k (or dq, dk)
+    v1 = ntok * Hv * V * e         # v, o, do or dv
+    g1 = ntok * Hv * 4             # g, beta, dg or dbeta
+    st = N * Hv * K * V * 4        # one state per (sequence, value head)
+    h0 = st if w.h0_std is not None else 0
+    f_prep = ntok * (Hq * 4 * C * K + Hv * (2 * C * K + 2 * C * V))
+    f_chain = ntok * Hv * (6 * K * V + 2 * C * V)
+    f_dh = ntok * Hv * (2 * C * V + 6 * K * V)
+    f_grad = ntok * (Hq * 4 * C * K + Hv * (14 * C * K + 8 * C * V + 12 * K * V + 4 * C * C))
+    table = {
+        "prep3": (f_prep, 2 * qk1 + v1 + 2 * g1),                    # q, k, v, g, beta
+        "fwd_hybrid": (f_chain, 2 * qk1 + h0 + v1 + st),             # q, k, h0 -> o, final
+        "bwd_dh": (f_dh, 2 * qk1 + v1 + st + st),                    # q, k, do, dht -> dh0
+        "bwd_grad": (f_grad, 2 * qk1 + 2 * v1 + 2 * g1 + 2 * qk1 + v1 + 2 * g1),
+        # q, k, v, do, g, beta -> dq, dk, dv, dg, dbeta
+        "recurrent": (ntok * Hv * 8 * K * V, 2 * qk1 + v1 + 2 * g1 + h0 + v1 + st),
+    }
+    return table.get(name)
+
+
+def kernel_roofline(name, w, avg_s, pk):
+    """The roofline of one kernel on its own rows: time bound = max(F / tensor
+    peak, B / HBM peak); the binding side's achieved rate over its peak."""
+    work = kernel_work(name, w)
+    if work is None or not avg_s:
+        return None
+    F, B = work
+    t_tc = F / (pk["bf16_tflops"] * 1e12)
+    t_hbm = B / (pk["hbm_gbs"] * 1e9)
+    if t_tc >= t_hbm:
+        return {"bound": "tensor", "unit": "TFLOP/s", "achieved": F / avg_s / 1e12,
+                "peak": pk["bf16_tflops"], "frac": t_tc / avg_s, "algorithmic_flops": F,
+                "algorithmic_bytes": B}
+    return {"bound": "hbm", "unit": "GB/s", "achieved": B / avg_s / 1e9, "peak": pk["hbm_gbs"],
+            "frac": t_hbm / avg_s, "algorithmic_flops": F, "algorithmic_bytes": B}
+
+
 def kernel_bytes(name, w, saved=False):
-    """Algorithmic bytes of one launch of a named kernel: the tensors that kernel
-    must read once and write once in this design (intermediates between the
-    kernels of the chain included, since each kernel has to move them).
+    """Design bytes of one launch of a named kernel: the tensors that kernel
+    must read once and write once in this design, intermediates between the
+    kernels of the chain included (w, u, P, chunk states, ...). Their ratio to
+    the launch time is a streaming efficiency, reported as design_frac beside
+    the roofline of kernel_work().
 
     Per token and value head at K = V = 128, bf16 (e = 2), G = Hv / Hq:
       prep3            2K*e/G (q, k) + V*e (v) + 3*4 (g, beta, gamma) + K*2 (w) + V*4 (u) + C*2 (P)
@@ -111,7 +172,6 @@ def kernel_bytes(name, w, saved=False):
         "prep_tc": qk1 + 2 * gam + gam + ainv,
         "prep3": prep3 + (ainv if saved else 0),                # q,k,v,g,beta -> gamma,w,u,P[,Ainv]
         "fwd_simt": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,  # q,k,v,gamma,beta,Ainv,h0 -> o,final
-        "fwd_tc": 2 * qk1 + v1 + 2 * gam + ainv + h0 + v1 + st,
         # q,k,w,u,P,gamma,h0 -> o,final[,entry states,Delta]
         "fwd_hybrid": 2 * qk1 + wb + ub + pb + gam + h0 + v1 + st + ((hc + dsb) if saved else 0),
         "bwd_prep3": prep3 + (0 if saved else ainv),
@@ -374,52 +434,56 @@ def run_decode(args):
         "gpu_launches": args.steps, "clocks": clk.summary()}))
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1,
-                    help="GPUs in the job (one process per GPU under torchrun; N replicas)")
-    ap.add_argument("--steps", type=int, default=20, help="timed steps")
-    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
-                    help="reference: time the fp64 oracle on the host cores on a bounded sample")
-    ap.add_argument("--workload", default="qwen_prefill_t8192_hv32",
-                    help="one of the named synthetic workloads (inputs.py)")
-    ap.add_argument("--fwd-only", action="store_true", help="time the forward alone")
-    ap.add_argument("--ref-tokens", type=int, default=1024,
-                    help="tokens per row in the oracle's bounded sample")
-    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
-    ap.add_argument("--decode", action="store_true", help="time the token-by-token step instead")
-    ap.add_argument("--heads", default=None, help="HQ,HV: override the workload's head counts (sweeps)")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.decode:
-        return run_decode(args)
+def torchrun_cmd(nproc, argv, port):
+    """The command that relaunches this script with one process per GPU."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nproc}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
 
-    from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS, make_inputs, scaled
-    w = WORKLOADS[args.workload]
-    if args.heads:
-        from dataclasses import replace
-        hq, hv = (int(x) for x in args.heads.split(","))
-        w = replace(w, name=f"{w.name}_hq{hq}_hv{hv}", Hq=hq, Hv=hv)
-    if args.impl == "reference":
-        return run_reference(args, w)
 
+def relaunch(args, argv):
+    """`--gpus N` (N > 1) without a torchrun environment: start N local ranks under
+    torch.distributed.run and return their exit status. Refuses when fewer than N
+    devices are visible (the CPU self-test of the launcher needs none)."""
+    import socket
+    if not args.dist_selftest:
+        import torch
+        have = torch.cuda.device_count()
+        if have < args.gpus:
+            raise SystemExit(f"--gpus {args.gpus}: only {have} CUDA device(s) visible")
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    return subprocess.call(["timeout", "-k", "60", "1800", *torchrun_cmd(args.gpus, argv, port)], env=env)
+
+
+def run_dist_selftest(args):
+    """Host-side multi-rank path without a GPU (gloo): every rank reports a
+    different per-rank time; rank 0 prints the line with the job's max-over-ranks
+    time and all ranks' tokens. Used by the CPU test of the `--gpus N` launcher."""
+    import datetime
+    import torch.distributed as dist
+    world, rank, local = dist_setup()
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    mine = 1.0 + rank
+    total = slowest_ms(mine, dist, "cpu")
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "n_gpus": world, "selftest": True, "ms_per_step": total,
+                          "value": job_mtokens_s(1024, world, 1, total)}), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
+def measure(w, steps, warmup, dev, rank, dist=None, timing=True, infer=True):
+    """Times fwd (+bwd) steps of one workload on this rank's GPU: CUDA events on
+    the launch stream, L2 flushed between steps (outside the events), the max
+    over ranks. Returns per-step times, per-kernel times and the chain rooflines."""
     import torch
     import gated_deltanet_chunked_rule_b200 as gdn
     from gated_deltanet_chunked_rule_b200 import _binding
-
-    world, rank, local = dist_setup()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    gdn.lib()  # fail loudly if the extension is missing
+    from gated_deltanet_chunked_rule_b200.inputs import make_inputs
 
     wr = rank_workload(w, rank)
     xh = make_inputs(wr)
@@ -429,32 +493,30 @@ def main():
     ws_f = torch.empty(max(P.fwd_workspace_size(), 1), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(max(P.bwd_workspace_size(), 1), dtype=torch.uint8, device=dev)
     o = torch.empty_like(x["v"])
+    do_bwd = True
+    try:
+        _, _, sv = gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"],
+                                                  x["scale"], x["h0"], True, x["cu_seqlens"],
+                                                  cu_host, save_for_backward=True)
+        gdn.chunk_gated_delta_rule_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], sv, x["do"],
+                                       x["dht"], x["scale"], x["h0"], x["cu_seqlens"], cu_host)
+    except _binding.GdnError as e:
+        if e.code != _binding.GDN_ERR_UNSUPPORTED:
+            raise
+        do_bwd = False
 
-    do_bwd = not args.fwd_only
-    if do_bwd:
-        try:
-            _, _, sv = gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"],
-                                                      x["scale"], x["h0"], True, x["cu_seqlens"],
-                                                      cu_host, save_for_backward=True)
-            gdn.chunk_gated_delta_rule_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], sv, x["do"],
-                                           x["dht"], x["scale"], x["h0"], x["cu_seqlens"], cu_host)
-        except _binding.GdnError as e:
-            if e.code != _binding.GDN_ERR_UNSUPPORTED:
-                raise
-            do_bwd = False
-
-    def step(inp):
+    def step(inp, train=True):
+        save = do_bwd and train
         o_, fin_, sv_ = gdn.chunk_gated_delta_rule_fwd(
             inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["scale"], inp["h0"], True,
-            inp["cu_seqlens"], cu_host, save_for_backward=do_bwd, workspace=ws_f, out=o)
-        if do_bwd:
+            inp["cu_seqlens"], cu_host, save_for_backward=save, workspace=ws_f, out=o)
+        if save:
             grads = gdn.chunk_gated_delta_rule_bwd(
                 inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], sv_, inp["do"], inp["dht"],
                 inp["scale"], inp["h0"], inp["cu_seqlens"], cu_host, workspace=ws_b)
             return o_, fin_, grads
         return o_, fin_, None
 
-    # L2 flush buffer: 2x the L2 size, written between timed steps (outside the events).
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=dev)
 
@@ -469,64 +531,155 @@ def main():
         torch.cuda.synchronize()
         return [a.elapsed_time(b) for a, b in ev]
 
-    for _ in range(args.warmup):
+    def kernel_pass(fn):
+        # the same steps again with the library's event timing on (events on the
+        # launch stream around every launch)
+        _binding.timing_enable(True)
+        timed_steps(steps, fn)
+        rep = _binding.timing_report()
+        _binding.timing_enable(False)
+        return rep
+
+    for _ in range(warmup):
         step(x)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with Clocks(local) as clk:
-        ms_list = timed_steps(args.steps, lambda: step(x))
+    res = {"x": x, "xh": xh, "step": step, "timed_steps": timed_steps, "do_bwd": do_bwd}
+    res["ms_list"] = timed_steps(steps, lambda: step(x))
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms = slowest_ms(sum(ms_list), dist, dev)
+    res["total_ms"] = slowest_ms(sum(res["ms_list"]), dist, dev)
+    pk, _ = peaks()
     alg = algorithmic(w)
-    tokens = alg["tokens"]
-    ms_step = total_ms / args.steps
-    value = job_mtokens_s(tokens, world, args.steps, total_ms)
-
-    # Per-kernel device times: a second pass of the same steps with the library's
-    # event timing on (events on the launch stream around every launch).
-    _binding.timing_enable(True)
-    timed_steps(args.steps, lambda: step(x))
-    rep = _binding.timing_report()
-    _binding.timing_enable(False)
-    launches_per_step = sum(v[0] for v in rep.values()) / args.steps
-    kern_total = sum(v[1] for v in rep.values())
-    kernels = {k: {"launches": v[0], "avg_us": 1e3 * v[1] / v[0],
-                   "share": v[1] / kern_total if kern_total else None}
-               for k, v in rep.items()}
-    dom = max(rep, key=lambda k: rep[k][1])
-    pk, pk_kind = peaks()
-    dom_avg_s = rep[dom][1] / rep[dom][0] * 1e-3
-    dom_bytes = kernel_bytes(dom, w, saved=do_bwd)
-    roofline = {"kernel": dom, "bound": "hbm", "unit": "GB/s",
-                "achieved": dom_bytes / dom_avg_s / 1e9 if dom_bytes else None,
-                "peak": pk["hbm_gbs"], "peak_kind": f"{pk_kind} hbm_gbs (burst copy)",
-                "traffic": measured_traffic(dom, w.name, "fwd+bwd" if do_bwd else "fwd"),
-                "algorithmic_bytes": dom_bytes}
-    if roofline["achieved"]:
-        roofline["frac"] = roofline["achieved"] / roofline["peak"]
-
-    # Whole-chain roofline of the forward (and backward) against max(F/peak, B/peak).
-    fwd_ms = sum(v[1] for k, v in rep.items() if not k.startswith("bwd")) / args.steps
-    bwd_ms = sum(v[1] for k, v in rep.items() if k.startswith("bwd")) / args.steps
 
     def chain(F, Bt, ms):
         t_tc = F / (pk["bf16_tflops"] * 1e12)
         t_hbm = Bt / (pk["hbm_gbs"] * 1e9)
-        return {"ms": ms, "Mtokens_s": tokens / (ms * 1e-3) / 1e6 if ms else None,
+        return {"ms": ms, "Mtokens_s": alg["tokens"] / (ms * 1e-3) / 1e6 if ms else None,
                 "tflops": F / (ms * 1e-3) / 1e12 if ms else None,
                 "gbs": Bt / (ms * 1e-3) / 1e9 if ms else None,
                 "bound_us": 1e6 * max(t_tc, t_hbm), "binding": "tensor" if t_tc > t_hbm else "hbm",
                 "frac": (1e3 * max(t_tc, t_hbm)) / ms if ms else None}
 
-    fwd_chain = chain(alg["f_fwd"], alg["b_fwd"], fwd_ms)
-    bwd_chain = chain(alg["f_bwd"], alg["b_bwd"], bwd_ms) if do_bwd else None
+    if timing:
+        rep = kernel_pass(lambda: step(x))
+        res["rep"] = rep
+        fwd_ms = sum(v[1] for k, v in rep.items() if not k.startswith("bwd")) / steps
+        bwd_ms = sum(v[1] for k, v in rep.items() if k.startswith("bwd")) / steps
+        res["fwd"] = chain(alg["f_fwd"], alg["b_fwd"], fwd_ms)
+        res["bwd"] = chain(alg["f_bwd"], alg["b_bwd"], bwd_ms) if do_bwd else None
+    if infer:
+        # the plain (inference) forward: nothing saved for a backward
+        inf_ms = timed_steps(steps, lambda: step(x, train=False))
+        inf_total = slowest_ms(sum(inf_ms), dist, dev)
+        res["fwd_infer"] = chain(alg["f_fwd"], alg["b_fwd"], inf_total / steps)
+        if timing:
+            rep_i = kernel_pass(lambda: step(x, train=False))
+            res["rep_infer"] = rep_i
+            res["fwd_infer"]["kernels_us"] = {k: 1e3 * v[1] / v[0] for k, v in rep_i.items()}
+    res["alg"] = alg
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs in the job: N replicas, one process per GPU (relaunched under "
+                         "torch.distributed.run when not already started by it)")
+    ap.add_argument("--steps", type=int, default=20, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
+                    help="reference: time the fp64 oracle on the host cores on a bounded sample")
+    ap.add_argument("--workload", default="qwen_prefill_t8192_hv32",
+                    help="one of the named synthetic workloads (inputs.py)")
+    ap.add_argument("--fwd-only", action="store_true", help="time the forward alone")
+    ap.add_argument("--ref-tokens", type=int, default=1024,
+                    help="tokens per row in the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the long-sequence and packed-batch workloads of the headline run")
+    ap.add_argument("--decode", action="store_true", help="time the token-by-token step instead")
+    ap.add_argument("--heads", default=None, help="HQ,HV: override the workload's head counts (sweeps)")
+    ap.add_argument("--dist-selftest", action="store_true", help=argparse.SUPPRESS)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args, sys.argv[1:])
+    if "WORLD_SIZE" in os.environ and world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.dist_selftest:
+        return run_dist_selftest(args)
+    if args.decode:
+        return run_decode(args)
+
+    from gated_deltanet_chunked_rule_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.heads:
+        from dataclasses import replace
+        hq, hv = (int(x) for x in args.heads.split(","))
+        w = replace(w, name=f"{w.name}_hq{hq}_hv{hv}", Hq=hq, Hv=hv)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import gated_deltanet_chunked_rule_b200 as gdn
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    gdn.lib()  # fail loudly if the extension is missing
+
+    with Clocks(local) as clk:
+        r = measure(w, args.steps, args.warmup, dev, rank, dist)
+    if args.fwd_only:
+        # forward-only line: the plain (inference) forward is the step
+        r["total_ms"] = r["fwd_infer"]["ms"] * args.steps
+        r["do_bwd"] = False
+        r["rep"] = r["rep_infer"]
+    do_bwd = r["do_bwd"]
+    rep, alg = r["rep"], r["alg"]
+    fwd_blocks = (None if args.fwd_only else r["fwd"], r["bwd"] if do_bwd else None, r["fwd_infer"])
+    tokens = alg["tokens"]
+    total_ms = r["total_ms"]
+    ms_step = total_ms / args.steps
+    value = job_mtokens_s(tokens, world, args.steps, total_ms)
+
+    kern_total = sum(v[1] for v in rep.values())
+    pk, pk_kind = peaks()
+    kernels = {}
+    for k, v in rep.items():
+        avg_s = v[1] / v[0] * 1e-3
+        kr = kernel_roofline(k, w, avg_s, pk)
+        kernels[k] = {"launches": v[0], "avg_us": 1e3 * v[1] / v[0],
+                      "share": v[1] / kern_total if kern_total else None,
+                      "frac": kr["frac"] if kr else None, "bound": kr["bound"] if kr else None}
+    # the roofline block: the kernel with the largest share of the step's device
+    # time among those that implement rows of the hot path, on its own rows
+    dom = max((k for k in rep if kernel_work(k, w)), key=lambda k: rep[k][1])
+    dom_avg_s = rep[dom][1] / rep[dom][0] * 1e-3
+    roofline = {"kernel": dom, **kernel_roofline(dom, w, dom_avg_s, pk)}
+    roofline["peak_kind"] = (f"{pk_kind} bf16_tflops (burst)" if roofline["bound"] == "tensor"
+                             else f"{pk_kind} hbm_gbs (burst copy)")
+    roofline["traffic"] = measured_traffic(dom, w.name, "fwd+bwd" if do_bwd else "fwd")
+    db = kernel_bytes(dom, w, saved=do_bwd)
+    if db:
+        roofline["design_bytes"] = db
+        roofline["design_frac"] = db / dom_avg_s / 1e9 / pk["hbm_gbs"]
 
     # End to end through the public API with host buffers: pinned H2D of the
     # step's inputs, the call, and D2H of its results, all inside the timing.
+    x, xh, step, timed_steps = r["x"], r["xh"], r["step"], r["timed_steps"]
     names_in = ["q", "k", "v", "g", "beta"] + (["h0"] if xh["h0"] is not None else []) + \
         (["do", "dht"] if do_bwd else [])
     host_in = {k: xh[k].pin_memory() for k in names_in}
@@ -539,7 +692,7 @@ def main():
             dev_in[k].copy_(host_in[k], non_blocking=True)
         inp = dict(x)
         inp.update(dev_in)
-        o_, fin_, grads = step(inp)
+        o_, fin_, grads = step(inp, train=do_bwd)
         outs = [o_, fin_] + (list(grads) if grads is not None else [])
         for i, t in enumerate(outs):
             if i not in host_out:
@@ -554,6 +707,19 @@ def main():
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     e2e = {"value": job_mtokens_s(tokens, world, args.steps, e2e_total), "unit": "Mtokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del r
+
+    # the long-sequence (sequence split) and packed-batch workloads, at their full
+    # sizes: per-step fwd / bwd chains and their rooflines
+    extra = {}
+    if not args.no_extra and not args.heads and w.name == "qwen_prefill_t8192_hv32":
+        for name in ("long_split_t65536_h8", "varlen_16seq_32k_h32"):
+            rr = measure(WORKLOADS[name], 5, 3, dev, rank, dist)
+            extra[name] = {"ms_per_step": rr["total_ms"] / 5,
+                           "Mtokens_s": job_mtokens_s(rr["alg"]["tokens"], world, 5, rr["total_ms"]),
+                           "fwd": rr["fwd"], "bwd": rr["bwd"], "fwd_infer": rr["fwd_infer"],
+                           "kernels_us": {k: 1e3 * v[1] / v[0] for k, v in rr["rep"].items()}}
+            del rr
 
     # every rank takes this collective, so a device error on one rank ends all of them
     # here rather than leaving the others waiting at the next barrier
@@ -577,11 +743,15 @@ def main():
                        "V": w.V, "chunk": CHUNK, "step": "fwd+bwd" if do_bwd else "fwd",
                        "l2": "flushed between steps (2x L2 write, outside the events)",
                        "parallelism": f"replicas x{world} (independent sequences per GPU)"},
-            "fwd": fwd_chain, "bwd": bwd_chain, "kernels": kernels, "roofline": roofline,
+            "fwd": None, "bwd": None, "fwd_infer": None,
+            "kernels": kernels, "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "gpu_launches": int(round(sum(v[0] for v in rep.values()))),
             "clocks": clk.summary(),
         }
+        line["fwd"], line["bwd"], line["fwd_infer"] = fwd_blocks
+        if extra:
+            line["other_workloads"] = extra
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()

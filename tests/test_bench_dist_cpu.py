@@ -71,3 +71,22 @@ def test_single_rank_needs_no_collective():
     import bench
     assert bench.slowest_ms(4.25) == 4.25
     assert bench.job_mtokens_s(8192, 1, 10, 8.0) == pytest.approx(8192 * 10 / 8e-3 / 1e6)
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun relaunches itself with two local ranks
+    (torch.distributed.run on 127.0.0.1); the host-side self-test of that path runs
+    on gloo, so the line's n_gpus and max-over-ranks time come from two processes."""
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dist-selftest"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["selftest"]
+    # rank r reports 1 + r ms: the job's time is the slower rank's
+    assert lines[0]["ms_per_step"] == pytest.approx(2.0)
