@@ -39,6 +39,7 @@ EXPORTS = (
     "gdn_timing_report",
     "gdn_chunk_fwd_noalloc",
     "gdn_recurrent_fwd",
+    "gdn_selftest_wait_timeout",
 )
 
 # Size of the static scratch array behind gdn_chunk_fwd_noalloc.
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_timing_enable.restype = i
             L.gdn_timing_report.argtypes = [ctypes.c_char_p, sz]
             L.gdn_timing_report.restype = i
+            L.gdn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, vp, vp]
+            L.gdn_selftest_wait_timeout.restype = i
             L.gdn_version.argtypes = []
             L.gdn_version.restype = ctypes.c_char_p
             _lib = L

@@ -371,6 +371,14 @@ int launch_prep(const FwdArgs &a, const char *tc_name = "prep_tc", const char *s
     return launch_prep_simt(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+// State chain + output of the tensor-core forward (transposed register chain;
+// GDN_CHAIN=v2 selects the earlier row-split chain for comparison).
+cudaError_t launch_chain(const FwdArgs &a) {
+    const char *e = getenv("GDN_CHAIN");
+    if (e && strcmp(e, "v2") == 0) return launch_fwd2(a);
+    return launch_fwd3(a);
+}
+
 int launch_plan(const gdn_problem *p, Plan &P, char *ws, unsigned *status, cudaStream_t st) {
     if (!P.varlen) return GDN_OK;
     int *info = (int *)ws;
@@ -436,9 +444,10 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
     a.status = status;
     a.stream = st;
     a.nseg = 1;
-    const char *which = getenv("GDN_FWD");
-    const bool tc = !use_simt(P.dtype) && tc_fwd_supported(a);
-    const bool hybrid = tc && !(which && strcmp(which, "v1") == 0) && P.tc_ok;
+    // bf16 with K = V = 128: the tensor-core kernels (chunk prep, then the state
+    // chain with the output); otherwise the fp32 CUDA-core kernels
+    const bool hybrid = !use_simt(P.dtype) && P.tc_ok &&
+                        (long long)P.d.NC * P.d.Hv * kChunk < (1ll << 31);
     if (hybrid) {
         if (!saved) a.ainv = nullptr;  // the hybrid forward reads w, u, P; Ainv only for `saved`
         TimedLaunch t("prep3", st);
@@ -465,7 +474,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
         s1.fwd_mode = 1;
         {
             TimedLaunch t("fwd_split_seg", st);
-            if (launch_fwd2(s1) != cudaSuccess) return GDN_ERR_CUDA;
+            if (launch_chain(s1) != cudaSuccess) return GDN_ERR_CUDA;
         }
         {
             TimedLaunch t("fwd_split_compose", st);
@@ -473,13 +482,10 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
         }
         a.fwd_mode = 2;
         TimedLaunch t("fwd_hybrid", st);
-        if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
+        if (launch_chain(a) != cudaSuccess) return GDN_ERR_CUDA;
     } else if (hybrid) {
         TimedLaunch t("fwd_hybrid", st);
-        if (launch_fwd2(a) != cudaSuccess) return GDN_ERR_CUDA;
-    } else if (tc) {
-        TimedLaunch t("fwd_tc", st);
-        if (launch_fwd_tc(a) != cudaSuccess) return GDN_ERR_CUDA;
+        if (launch_chain(a) != cudaSuccess) return GDN_ERR_CUDA;
     } else {
         TimedLaunch t("fwd_simt", st);
         if (launch_fwd_simt(a) != cudaSuccess) return GDN_ERR_CUDA;
@@ -492,7 +498,7 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
         r.nseg = 1;
         r.fwd_mode = 0;
         TimedLaunch t("fwd_states", st);
-        if (launch_fwd2(r) != cudaSuccess) return GDN_ERR_CUDA;
+        if (launch_chain(r) != cudaSuccess) return GDN_ERR_CUDA;
     }
     return GDN_OK;
 }
@@ -551,7 +557,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
             f.h_chunks16 = ws + T.hc;
             f.delta16 = ws + T.delta;
             TimedLaunch t("bwd_recompute", st);
-            if (launch_fwd2(f) != cudaSuccess) return GDN_ERR_CUDA;
+            if (launch_chain(f) != cudaSuccess) return GDN_ERR_CUDA;
         }
         char *hcs = (char *)f.h_chunks16, *dls = (char *)f.delta16;
         BwdArgs b;
@@ -714,6 +720,15 @@ int gdn_get_device_status(void *stream) {
     if (v && cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
         return GDN_ERR_CUDA;
     return (int)v;
+}
+
+int gdn_selftest_wait_timeout(unsigned long long limit_ns, unsigned long long *elapsed_ns, void *stream) {
+    if (!elapsed_ns || !aligned16(elapsed_ns)) return GDN_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return GDN_ERR_CUDA;
+    TimedLaunch t("selftest_wait", (cudaStream_t)stream);
+    return launch_wait_selftest(limit_ns, elapsed_ns, status, (cudaStream_t)stream) == cudaSuccess ? GDN_OK
+                                                                                                   : GDN_ERR_CUDA;
 }
 
 int gdn_timing_enable(int on) {

@@ -137,6 +137,9 @@ struct RecurrentArgs {
     cudaStream_t stream;
 };
 cudaError_t launch_recurrent(const RecurrentArgs &a);
+// Self-test of the bounded waits (gdn_selftest.cu).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, unsigned long long *elapsed, unsigned *status,
+                                 cudaStream_t stream);
 
 struct BwdArgs {
     Dims d;
@@ -158,11 +161,10 @@ struct BwdArgs {
 cudaError_t launch_prep_simt(const FwdArgs &a);
 cudaError_t launch_fwd_simt(const FwdArgs &a);
 cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part);
-bool tc_fwd_supported(const FwdArgs &a);
 bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
-cudaError_t launch_fwd_tc(const FwdArgs &a);
 cudaError_t launch_fwd2(const FwdArgs &a);
+cudaError_t launch_fwd3(const FwdArgs &a);
 // Chunk prep of the tensor-core path: gamma, Ainv (optional), w, u, P.
 bool prep3_supported(const FwdArgs &a);
 cudaError_t launch_prep3(const FwdArgs &a);

@@ -86,6 +86,16 @@ __device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// Zeroes rows [len, 64) of a [64][128] bf16 tile stored as two 64-column halves of
+// 128-byte rows (the swizzle permutes 16-byte chunks within a row, so whole rows
+// are zeroed regardless of it).
+__device__ __forceinline__ void zero_rows(uint32_t tile, int len, int tid) {
+    for (int i = tid; i < (C - len) * 16; i += kThreads) {
+        const int r = len + (i >> 4), c = i & 15;
+        st_shared_v4(tile + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
+    }
+}
+
 struct Prep3Params {
     Dims d;
     const float *g, *beta;
@@ -160,6 +170,14 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     ok = cta_wait(tma_bar, tma_phase & 1);
     if (ok) ++tma_phase, tma_pending = false;
+    if (len < C) {
+        // a ragged chunk: rows past its end hold the next packed sequence (or zeros); zero them so that
+        // a non-finite value there cannot reach this sequence through a product with a zero weight
+        zero_rows(sb + kQV, len, tid);
+        zero_rows(sb + kKt, len, tid);
+        fence_proxy_async();
+        __syncthreads();
+    }
     if (ok && tid == 0) {
         tc_fence_after();
         const uint32_t id_S = idesc_bf16(64, 64, false, false);
@@ -337,6 +355,11 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // ---- u = Au V, w = Aw K on tcgen05 once this head's v tile has landed
         ok = cta_wait(tma_bar, tma_phase & 1);
         if (ok) ++tma_phase, tma_pending = false;
+        if (len < C) {
+            zero_rows(sb + kQV, len, tid);  // the v tile's rows past the end, as for q and k
+            fence_proxy_async();
+            __syncthreads();
+        }
         if (ok && tid == 0) {
             tc_fence_after();
             const uint32_t id_W = idesc_bf16(64, 128, false, true);

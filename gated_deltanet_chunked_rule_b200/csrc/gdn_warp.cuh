@@ -27,8 +27,10 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
-// Bounded mbarrier wait; false if it expired or the CTA is aborting.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// Bounded mbarrier wait; false if it expired (limit_ns of globaltimer, checked
+// every 1024 polls) or the CTA is aborting.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         uint64_t limit_ns = kWaitNs) {
     const uint32_t a = smem_u32(bar);
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
@@ -37,7 +39,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
             if (*abort_flag) return false;
             const uint64_t t = globaltimer();
             if (i == 0) t0 = t;
-            else if (t - t0 > kWaitNs) return false;
+            else if (t - t0 > limit_ns) return false;
         }
     }
 }
@@ -55,7 +57,8 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *ctr) {
 // Bounded wait until *ctr >= need; false if it expired or the CTA is aborting.
 // Within a warp role one thread polls, and a named barrier passes the result on
 // (role_sync_and): every poll is a shared-memory load.
-__device__ __forceinline__ bool wait_ge(const uint32_t *ctr, uint32_t need, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_ge(const uint32_t *ctr, uint32_t need, volatile int *abort_flag,
+                                        uint64_t limit_ns = kWaitNs) {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         if (ld_acquire(ctr) >= need) return true;
@@ -63,7 +66,7 @@ __device__ __forceinline__ bool wait_ge(const uint32_t *ctr, uint32_t need, vola
             if (*abort_flag) return false;
             const uint64_t t = globaltimer();
             if (i == 0) t0 = t;
-            else if (t - t0 > kWaitNs) return false;
+            else if (t - t0 > limit_ns) return false;
         }
     }
 }
@@ -108,6 +111,11 @@ __device__ __forceinline__ void st_shared_v4f(uint32_t addr, float a, float b, f
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d));
 }
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -123,6 +131,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
+}
+
+// Stores four 8x8 bf16 matrices, each transposed: lane i of matrix q's lane
+// group (lanes 8q .. 8q+7) gives the address of memory row i, which receives
+// column i of the fragment matrix held in register r[q] (the m16n8 accumulator
+// layout: lane l holds row l/4, columns 2(l%4) and 2(l%4)+1).
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]));
+}
+
+// Named barrier over kCount threads.
+template <int kCount>
+__device__ __forceinline__ void named_sync(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kCount) : "memory");
 }
 
 // D (16 x 8, fp32) += A (16 x 16, bf16, row) * B (16 x 8, bf16, col).
@@ -169,6 +192,16 @@ __device__ __forceinline__ void wgemm(float (&c)[NT][4], const Tile &A, const Ti
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                  : "memory");
+}
+// 4-byte asynchronous copy global -> shared (completion tracked by cp.async groups or,
+// with cp_async_mbar_arrive, by an mbarrier).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+// The mbarrier's current phase also waits for every cp.async this thread issued
+// before: its pending count is raised now and lowered when those copies land.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }

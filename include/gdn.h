@@ -190,6 +190,23 @@ int gdn_get_device_status(void *stream /* cudaStream_t */);
 int gdn_timing_enable(int on);
 int gdn_timing_report(char *buf, size_t buf_len);
 
+/* Self-test of the device-side failure detection. Every wait inside this
+ * library's kernels (on a TMA or tensor-core completion, or on another warp's
+ * hand-over) is bounded: after a limit it gives up, records GDN_ERR_TIMEOUT in
+ * the status word and lets the kernel wind down instead of hanging the GPU.
+ * This entry point enqueues one small kernel whose two waits can never be
+ * satisfied -- an mbarrier phase that nothing completes and a hand-over
+ * counter that nothing publishes -- with limit_ns of wall-clock time each
+ * (0: the limit the kernels use, 2 s). Nothing else is in flight in it, so it
+ * always ends normally. elapsed_ns: device memory, 2 entries (16-byte
+ * aligned), receiving the time each wait took before giving up (all ones if
+ * a wait was, impossibly, satisfied). Afterwards gdn_get_device_status reports
+ * GDN_ERR_TIMEOUT. The FlashQLA pages have no counterpart to this entry
+ * point; it serves the failure-detection tests. Returns GDN_ERR_INVALID_ARG
+ * for a null or misaligned elapsed_ns, GDN_ERR_CUDA if the launch fails. */
+int gdn_selftest_wait_timeout(unsigned long long limit_ns, unsigned long long *elapsed_ns,
+                              void *stream /* cudaStream_t */);
+
 /* Static, human-readable name of a status code. */
 const char *gdn_status_string(int status);
 

@@ -225,3 +225,31 @@ def test_larger_head_groups(oracle_mod, Hq, Hv):
                  seed=40 + Hv)
     x = make_inputs(w)
     check(oracle_mod, x, gpu_bwd(x), w.name)
+
+
+def test_empty_batch_backward():
+    # T = 0: no token, so dq, dk, dv, dg, dbeta are empty and dh0 = dht exactly
+    import gated_deltanet_chunked_rule_b200 as gdn
+    for K, V in ((64, 64), (128, 128)):
+        w = Workload("bwd_empty", B=2, T=0, Hq=1, Hv=2, K=K, V=V, h0_std=0.02, grads=True)
+        x = to_dev(make_inputs(w))
+        _, _, saved = gdn.chunk_gated_delta_rule_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"],
+                                                     initial_state=x["h0"], save_for_backward=True)
+        out = gdn.chunk_gated_delta_rule_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], saved, x["do"],
+                                             x["dht"], x["scale"], x["h0"])
+        torch.cuda.synchronize()
+        assert gdn.device_status() == 0
+        g = dict(zip(NAMES, out))
+        for n in ("dq", "dk", "dv", "dbeta", "dg"):
+            assert g[n].numel() == 0
+        torch.testing.assert_close(g["dh0"], x["dht"], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("name", ["qwen_prefill_t8192_hv32"])
+def test_slow_decay_backward_full_size(oracle_mod, name):
+    # g x 0.01 at the headline shape: the reverse scan's bf16 operands
+    # accumulate over all 128 chunks
+    w = scaled(WORKLOADS[name], grads=True)
+    x = make_inputs(w)
+    x["g"] = x["g"] * 0.01
+    check(oracle_mod, x, gpu_bwd(x), name + "_slow")

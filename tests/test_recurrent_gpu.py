@@ -80,3 +80,15 @@ def test_decode_agrees_with_chunked_forward(oracle_mod):
     o_c, f_c, _ = gpu_fwd(x)
     check_fwd(oracle_mod, x, o_r, f_r, "dec_vs_chunk recurrent")
     assert rel_fro(f64(o_r), f64(o_c)) <= TOL_BF16_REL and rel_fro(f64(f_r), f64(f_c)) <= TOL_BF16_REL
+
+
+def test_decode_empty_batch_keeps_state():
+    # T = 0: nothing to decode, the state is returned unchanged, bit for bit
+    import gated_deltanet_chunked_rule_b200 as gdn
+    w = Workload("dec_empty", B=2, T=0, Hq=1, Hv=2, K=128, V=128, h0_std=0.02)
+    x = to_dev(make_inputs(w))
+    o, fin = gdn.recurrent_gated_delta_rule(x["q"], x["k"], x["v"], x["g"], x["beta"], x["scale"], x["h0"])
+    torch.cuda.synchronize()
+    assert gdn.device_status() == 0
+    assert o.numel() == 0
+    torch.testing.assert_close(fin, x["h0"], rtol=0, atol=0)
