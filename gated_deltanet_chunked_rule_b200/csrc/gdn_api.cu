@@ -163,7 +163,7 @@ int make_plan(const gdn_problem *p, Plan *out) {
         }
         d.N = p->num_seqs;
         d.NC = (int)nc;
-        P.seq_info_bytes = align_up(sizeof(int) * (3 * (size_t)d.N + 1));
+        P.seq_info_bytes = align_up(sizeof(int) * (4 * (size_t)d.N + 1));
     } else {
         d.N = p->B;
         d.NC = p->B * ((p->T + kChunk - 1) / kChunk);
@@ -349,8 +349,25 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *__restrict__ 
         if (carry != NC_expected) ok = 0;
     }
     __syncthreads();
+    // longest first: order[rank] = n, rank = number of sequences with more chunks
+    // (ties by index), so that chain kernels start their longest work first; a
+    // batch of more than 1024 sequences keeps its own order (the quadratic ranking
+    // would cost more than it saves)
+    for (int n = tid; n < N; n += 1024) {
+        int rank = n;
+        if (N <= 1024) {
+            const int cn = info[2 * N + n + 1] - info[2 * N + n];
+            rank = 0;
+            for (int m = 0; m < N; ++m) {
+                const int cm = info[2 * N + m + 1] - info[2 * N + m];
+                rank += (cm > cn) || (cm == cn && m < n);
+            }
+        }
+        info[3 * N + 1 + rank] = n;
+    }
+    __syncthreads();
     if (!ok) {
-        for (int e = tid; e < 3 * N + 1; e += 1024) info[e] = 0;
+        for (int e = tid; e < 4 * N + 1; e += 1024) info[e] = e >= 3 * N + 1 ? e - (3 * N + 1) : 0;
         if (tid == 0) set_status(status, GDN_ERR_DEVICE_ARG);
     }
 }

@@ -100,8 +100,8 @@ struct BwdDhParams {
     __nv_bfloat16 *ddelta;       // dDelta, blocked: per (chunk, head) V/32 slices of [4][64][8]
     float *dh0;                  // [N, Hv, K, V] or null
     float scale;
-    // Sequence split: blockIdx.x = sequence * nseg + segment, a segment being a
-    // contiguous run of ceil(chunks / nseg) chunks of its sequence.
+    // Sequence split: each sequence runs as nseg segments, contiguous runs of
+    // ceil(chunks / nseg) chunks (CTA slot = sequence rank * nseg + segment).
     int nseg;
     int mode;                    // BwdDhMode
     const float *seg_dh;         // kBSegOut: [N * nseg, Hv, K, V] gradient at every segment's end
@@ -117,14 +117,18 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
               const __grid_constant__ CUtensorMap tm_do, const BwdDhParams prm) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
     volatile int *abort_flag = &sm->abort_flag;
     const uint32_t sb = smem_u32(smem);
 
     const Dims &d = prm.d;
     const int nseg = prm.nseg;
-    const int n = blockIdx.x / nseg, sseg = blockIdx.x % nseg, h = blockIdx.y, c0 = blockIdx.z * kBV;
+    // 1-D grid, sequence-major in longest-first order (the longest scans start first)
+    const int nsl = (d.V + (prm.mode == kBSegPass ? d.K : 0)) / kBV;
+    const int slot = blockIdx.x / (d.Hv * nsl), rem = blockIdx.x % (d.Hv * nsl);
+    const int n = seq_by_length(d, slot / nseg), sseg = slot % nseg, h = rem / nsl, zs = rem % nsl;
+    const int c0 = zs * kBV;
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
@@ -399,7 +403,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             ok = aux_sync(atid != 0 || wait_ge(&ctr[kHbFull], it + 1, abort_flag));
             if (!ok) break;
             {
-                __nv_bfloat16 *hc = prm.dh_chunks + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + blockIdx.z) * (K * kBV);
+                __nv_bfloat16 *hc = prm.dh_chunks + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + zs) * (K * kBV);
 #pragma unroll
                 for (int i = 0; i < 4 && outputs; ++i) {
                     const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 128 + k
@@ -414,7 +418,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             ok = aux_sync(atid != 0 || wait_ge(&ctr[kDbFull], it + 1, abort_flag));
             if (!ok) break;
             {
-                __nv_bfloat16 *dc = prm.ddelta + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + blockIdx.z) * (kChunk * kBV);
+                __nv_bfloat16 *dc = prm.ddelta + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + zs) * (kChunk * kBV);
 #pragma unroll
                 for (int i = 0; i < 2 && outputs; ++i) {
                     const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 64 + t
@@ -558,7 +562,9 @@ cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16,
     cudaError_t e = cudaFuncSetAttribute(bwd_dh_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
-    const dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kBSegPass ? d.K : 0)) / kBV);
+    const long long nctas = (long long)d.N * p.nseg * d.Hv * ((d.V + (p.mode == kBSegPass ? d.K : 0)) / kBV);
+    if (nctas >= (1ll << 31)) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)nctas);
     bwd_dh_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mp, mdo, p);
     return cudaGetLastError();
 }

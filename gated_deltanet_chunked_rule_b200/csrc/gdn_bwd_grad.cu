@@ -196,7 +196,7 @@ __device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity) {
 __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_constant__ GradMaps tm,
                                                                const GradParams prm) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     const uint32_t sb = smem_u32(smem);
     Vecs &vec = *reinterpret_cast<Vecs *>(smem + kVec);
     const Dims &d = prm.d;

@@ -144,7 +144,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_o,
             const Fwd2Params prm) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
     volatile int *abort_flag = &sm->abort_flag;
     const uint32_t sb = smem_u32(smem);

@@ -89,6 +89,7 @@ constexpr int kHb = kO0 + kOS * kOStageBytes;  // kHB x 8192: h^T (bf16): (v/8)*
 constexpr int kDb = kHb + kHB * 8192;          // kHB x 4096: Delta (bf16): (v/8)*1024 + t*16 + (v%8)*2
 constexpr int kXb = kDb + kHB * 4096;          // 4096: Delta~ A fragments, [group][quarter][lane] x 16 bytes
 constexpr int kOs = kXb + 4096;                // 4096: o of a full chunk, staged for its TMA store
+                                               // ([64][32] bf16, 64-byte swizzle)
 constexpr int kGam = kOs + 4096;               // kCS x 64 fp32: gamma of each staged chunk
 constexpr int kSmall = kGam + 1024;
 constexpr int kSmemBytes = kSmall + 2048 + 1024;
@@ -130,8 +131,8 @@ struct Fwd3Params {
     float *final_state;   // [N, Hv, K, V] or null
     __nv_bfloat16 *h_chunks;  // entry state of every chunk (bf16, blocked) or null
     __nv_bfloat16 *delta;     // Delta of every chunk (bf16, blocked) or null
-    // Sequence split: blockIdx.x = sequence * nseg + segment; a segment is a
-    // contiguous run of ceil(chunks / nseg) chunks of its sequence.
+    // Sequence split: each sequence runs as nseg segments, contiguous runs of
+    // ceil(chunks / nseg) chunks (CTA slot = sequence rank * nseg + segment).
     int nseg;
     int mode;             // Fwd3Mode
     const float *seg_h0;  // kSegOut: [N * nseg, Hv, K, V] start state of every segment
@@ -152,7 +153,7 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_o,
             const Fwd3Params prm) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
     volatile int *abort_flag = &sm->abort_flag;
     const uint32_t sb = smem_u32(smem);
@@ -160,7 +161,12 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     const Dims &d = prm.d;
     const int nseg = prm.nseg;
-    const int n = blockIdx.x / nseg, sseg = blockIdx.x % nseg, h = blockIdx.y, c0 = blockIdx.z * kBV;
+    // 1-D grid, sequence-major in longest-first order: the CTAs of the longest
+    // sequences (all their heads and column slices) are dispatched first
+    const int nsl = (d.V + (prm.mode == kSegPass ? d.K : 0)) / kBV;
+    const int slot = blockIdx.x / (d.Hv * nsl), rem = blockIdx.x % (d.Hv * nsl);
+    const int n = seq_by_length(d, slot / nseg), sseg = slot % nseg, h = rem / nsl, zs = rem % nsl;
+    const int c0 = zs * kBV;
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int K = 128, V = 128;
@@ -465,18 +471,35 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const float er[2] = {__expf(g0), __expf(g1)};
                 const int t0 = sr.start + j * kChunk;
                 const bool full = len == kChunk;
+                // o in the m16n8 accumulator layout the 16x256b loads deliver: ov[i][half] is the
+                // 8 x 8 block (rows 16q + 8 half .., columns 8i ..), this lane holding row eg,
+                // columns 2ec, 2ec + 1
+                uint32_t ov[4][2];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + rr[half]) * d.Hv + h) * V + c0 + 2 * ec;
+                for (int half = 0; half < 2; ++half)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int k = 4 * i + 2 * half;
-                        const uint32_t xv =
-                            pack_bf16(scl * fmaf(er[half], dq[k], dp[k]), scl * fmaf(er[half], dq[k + 1], dp[k + 1]));
-                        if (full)  // a ragged chunk's tile would spill into the next sequence
-                            st_shared_b32(sb + kOs + rr[half] * 64 + (8 * i + 2 * ec) * 2, xv);
-                        else if (rr[half] < len)
-                            *reinterpret_cast<uint32_t *>(dst + 8 * i) = xv;
+                        ov[i][half] = pack_bf16(scl * fmaf(er[half], dq[k], dp[k]), scl * fmaf(er[half], dq[k + 1], dp[k + 1]));
+                    }
+                if (full) {
+                    // staging tile [64][32] bf16 with the 64-byte swizzle of its TMA store (16-byte
+                    // chunk c of row r at chunk c ^ ((r / 2) % 4)): two conflict-free stmatrix.x4
+                    const int li = lane & 7, mi = lane >> 3;
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        const int i = 2 * a + (mi >> 1), r = 16 * q + 8 * (mi & 1) + li;
+                        const uint32_t regs[4] = {ov[2 * a][0], ov[2 * a][1], ov[2 * a + 1][0], ov[2 * a + 1][1]};
+                        stsm_x4(sb + kOs + r * 64 + ((i ^ ((r >> 1) & 3)) << 4), regs);
+                    }
+                } else {
+                    // a ragged chunk's tile would spill into the next sequence: row by row
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        __nv_bfloat16 *dst = prm.o + ((size_t)(t0 + rr[half]) * d.Hv + h) * V + c0 + 2 * ec;
+                        if (rr[half] < len)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 8 * i) = ov[i][half];
                     }
                 }
                 if (full) {
@@ -604,7 +627,7 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 if (lane == 0) {
-                    const size_t blk = ((size_t)(sr.chunk0 + j) * d.Hv + h) * (V / kBV) + blockIdx.z;
+                    const size_t blk = ((size_t)(sr.chunk0 + j) * d.Hv + h) * (V / kBV) + zs;
                     bulk_store(prm.h_chunks + blk * (K * kBV), sb + kHb + (j % kHB) * 8192, K * kBV * 2);
                     bulk_store(prm.delta + blk * (kChunk * kBV), sb + kDb + (j % kHB) * 4096, kChunk * kBV * 2);
                     bulk_commit();
@@ -686,7 +709,7 @@ cudaError_t launch_fwd3(const FwdArgs &a) {
     const cuuint64_t dov[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
     const cuuint64_t sov[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
     const cuuint32_t bov[3] = {kBV, 1, 64};
-    if (!make_map(&mo, BF, a.o ? a.o : a.w16, 3, dov, sov, bov, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorInvalidValue;
+    if (!make_map(&mo, BF, a.o ? a.o : a.w16, 3, dov, sov, bov, CU_TENSOR_MAP_SWIZZLE_64B)) return cudaErrorInvalidValue;
     // chunk entry states and Delta: both or neither
     if ((a.h_chunks16 != nullptr) != (a.delta16 != nullptr)) return cudaErrorInvalidValue;
     Fwd3Params p;
@@ -709,7 +732,9 @@ cudaError_t launch_fwd3(const FwdArgs &a) {
     cudaError_t e = cudaFuncSetAttribute(fwd3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     // the segment pass also carries the K operator columns
-    dim3 grid(d.N * p.nseg, d.Hv, (d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
+    const long long nctas = (long long)d.N * p.nseg * d.Hv * ((d.V + (p.mode == kSegPass ? d.K : 0)) / kBV);
+    if (nctas >= (1ll << 31)) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)nctas);
     fwd3_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mw, mu, mp, mo, p);
     return cudaGetLastError();
 }

@@ -27,6 +27,7 @@ constexpr int kChunk = 64;
 //   info[0 .. N)        first token of sequence n
 //   info[N .. 2N)       length of sequence n
 //   info[2N .. 3N]      first global chunk of sequence n (info[3N] = total chunks)
+//   info[3N+1 .. 4N]    sequences by decreasing chunk count (ties by index)
 // With no packing the table is not built (seq_info == nullptr): sequence n is
 // batch row n, tokens [n*T, (n+1)*T), chunks [n*ceil(T/64), (n+1)*ceil(T/64)).
 struct Dims {
@@ -55,6 +56,11 @@ __device__ __forceinline__ SeqRange seq_range(const Dims &d, int n) {
         r.chunk0 = n * per;
     }
     return r;
+}
+
+// The k-th sequence in longest-first order (identity without packing).
+__device__ __forceinline__ int seq_by_length(const Dims &d, int k) {
+    return d.seq_info ? d.seq_info[3 * d.N + 1 + k] : k;
 }
 
 // Sequence that owns global chunk c (binary search in the chunk offsets); -1 if none.

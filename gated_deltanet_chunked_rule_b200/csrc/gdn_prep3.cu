@@ -25,6 +25,7 @@
 // beta = 0, so their rows of A vanish, the inverse is the identity there and
 // their columns of Ainv diag(beta) are zero: whatever the TMA reads past the
 // end (the next sequence, or zeros) never reaches an output.
+#include <algorithm>
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -77,13 +78,19 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Bounded wait on an mbarrier phase by every thread of the CTA.
+// Bounded wait on an mbarrier phase by every thread of the CTA. The result is
+// the same in every thread (a barrier ANDs it), so that the CTA's control flow,
+// and with it every later __syncthreads, stays uniform even when a wait expires.
 __device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
     const uint64_t t0 = globaltimer();
+    bool ok = true;
     while (!mbar_try_wait(a, parity))
-        if (globaltimer() - t0 > kWaitNs) return false;
-    return true;
+        if (globaltimer() - t0 > kWaitNs) {
+            ok = false;
+            break;
+        }
+    return __syncthreads_and(ok ? 1 : 0) != 0;
 }
 
 // Zeroes rows [len, 64) of a [64][128] bf16 tile stored as two 64-column halves of
@@ -113,15 +120,9 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
              const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_po,
              const Prep3Params prm) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = align_smem_1024(smem_raw);
     const uint32_t sb = smem_u32(smem);
     const Dims &d = prm.d;
-    const int cg = blockIdx.x, hq = blockIdx.y;
-    const int n = chunk_owner(d, cg);
-    if (n < 0) return;  // whole CTA, before any allocation
-    const SeqRange sr = seq_range(d, n);
-    const int ci = cg - sr.chunk0;
-    const int t0 = sr.start + ci * C, len = min(C, sr.len - ci * C);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wm = warp & 3, wn = warp >> 2, g8 = lane >> 2, c4 = lane & 3;
     const int r0 = 16 * wm + g8, r1 = r0 + 8;
@@ -153,6 +154,33 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint32_t tma_phase = 0, mma_phase = 0;  // phases consumed so far
     bool tma_pending = false, mma_pending = false;  // (thread 0) issued and not yet consumed
     bool ok = true;
+    const int n_items = d.NC * d.Hq;
+    // Persistent: items (chunk, qk head) in steps of the grid; the tiles of this CTA's next
+    // item are prefetched into L2 while it works on the current one.
+    auto prefetch_item = [&](int item) {
+        if (item >= n_items) return;
+        const int cg2 = item / d.Hq, hq2 = item % d.Hq;
+        const int n2 = chunk_owner(d, cg2);
+        if (n2 < 0) return;
+        const SeqRange s2 = seq_range(d, n2);
+        const int t2 = s2.start + (cg2 - s2.chunk0) * C;
+        tma_prefetch_3d(&tm_q, 0, hq2, t2);
+        tma_prefetch_3d(&tm_q, 64, hq2, t2);
+        tma_prefetch_3d(&tm_k, 0, hq2, t2);
+        tma_prefetch_3d(&tm_k, 64, hq2, t2);
+        for (int gi = 0; gi < G; ++gi) {
+            tma_prefetch_3d(&tm_v, 0, hq2 * G + gi, t2);
+            tma_prefetch_3d(&tm_v, 64, hq2 * G + gi, t2);
+        }
+    };
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    const int cg = item / d.Hq, hq = item % d.Hq;
+    const int n = chunk_owner(d, cg);
+    if (n < 0) continue;  // the whole CTA
+    const SeqRange sr = seq_range(d, n);
+    const int ci = cg - sr.chunk0;
+    const int t0 = sr.start + ci * C, len = min(C, sr.len - ci * C);
+    if (tid == 0) prefetch_item(item + gridDim.x);
 
     // ---- q, k tiles by TMA; S = Q K^T and G = K K^T on tcgen05
     if (tid == 0) {
@@ -396,18 +424,33 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
             tmem_ld16x256_x4(tmem + lane_base + kColW + cb, v);  // w
+            // wx[i][hi]: the 8 x 8 block (rows 16 wm + 8 hi .., columns cb + 8 i ..) in the m16n8
+            // accumulator layout (this lane: row g8, columns 2 c4, 2 c4 + 1)
+            uint32_t wx[4][2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int col = cb + 8 * i + 2 * c4;
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = hi ? r1 : r0;
-                    const uint32_t x = pack_bf16(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
-                    if (full)
-                        st_shared_b32(sb + kWs + (col >> 6) * 8192 + r * 128 + ((((col & 63) >> 3) ^ (r & 7)) << 4) + (col & 7) * 2, x);
-                    else if (r < len)
-                        *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r) * d.Hv + h) * K + col) = x;
+                for (int hi = 0; hi < 2; ++hi) wx[i][hi] = pack_bf16(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
+            if (full) {
+                // two stmatrix.x4 into the 128-byte-swizzled staging tile (conflict-free: the 8 rows
+                // of a block land in 8 distinct 16-byte chunks)
+                const int li = lane & 7, mi = lane >> 3;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const int col = cb + 8 * (2 * a + (mi >> 1)), r = 16 * wm + 8 * (mi & 1) + li;
+                    const uint32_t regs[4] = {wx[2 * a][0], wx[2 * a][1], wx[2 * a + 1][0], wx[2 * a + 1][1]};
+                    stsm_x4(sb + kWs + (col >> 6) * 8192 + r * 128 + ((((col & 63) >> 3) ^ (r & 7)) << 4), regs);
                 }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int hi = 0; hi < 2; ++hi) {
+                        const int r = hi ? r1 : r0;
+                        if (r < len)
+                            *reinterpret_cast<uint32_t *>(prm.w_out + ((size_t)(t0 + r) * d.Hv + h) * K + cb + 8 * i + 2 * c4) =
+                                wx[i][hi];
+                    }
             }
         }
         fence_proxy_async();  // u, w -> their TMA stores
@@ -420,6 +463,8 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             bulk_commit();
         }
     }
+    __syncthreads();  // every thread is done with this item's shared memory before the next one's loads
+    }  // item loop
     if (!ok) {
         if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
         // a TMA load or MMA that has not completed may still be in flight: wait (bounded) for it
@@ -485,7 +530,15 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     p.status = a.status;
     cudaError_t e = cudaFuncSetAttribute(prep3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    prep3_kernel<<<dim3(d.NC, d.Hq), kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, muo, mwo, mpo, p);
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+    }
+    const long long items = (long long)d.NC * d.Hq;
+    if (items >= (1ll << 31)) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<long long>(items, 2ll * sms);  // persistent, two CTAs per SM
+    prep3_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, muo, mwo, mpo, p);
     return cudaGetLastError();
 }
 

@@ -142,6 +142,13 @@ __device__ __forceinline__ void stsm_x4_t(uint32_t addr, const uint32_t (&r)[4])
                  "r"(r[1]), "r"(r[2]), "r"(r[3]));
 }
 
+// The same without the transpose: memory row i of matrix q receives row i of
+// the fragment matrix in r[q].
+__device__ __forceinline__ void stsm_x4(uint32_t addr, const uint32_t (&r)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3]));
+}
+
 // Named barrier over kCount threads.
 template <int kCount>
 __device__ __forceinline__ void named_sync(int id) {

@@ -26,6 +26,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory buffer rounded up to a 1024-byte boundary (what the
+// 128-byte-swizzled tiles need), computed as an offset from the __shared__ array
+// itself rather than through an integer cast, so that the compiler still knows
+// the result points into shared memory and emits shared (not generic) loads and
+// stores for every access made through it.
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *smem_raw) {
+    return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
