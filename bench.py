@@ -193,9 +193,6 @@ NCU_TRAFFIC = {
     "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 170267136,
                sources=["gdn_bwd_dh.cu"],
                sha256="ca66ab3574fc215bf4fee7b29431bcb20e89949c8d939b5fe71680a0560c0f0a"),
-    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303088896 + 230655744,
-               sources=["gdn_fwd2.cu"],
-               sha256="9577197f9cc991b68c924b4cce99cacaadd3aacef535ded4fe595f62798731a1"),
     "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549451520 + 481462272,
                sources=["gdn_recurrent.cu"],
                sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),

@@ -388,13 +388,8 @@ int launch_prep(const FwdArgs &a, const char *tc_name = "prep_tc", const char *s
     return launch_prep_simt(a) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-// State chain + output of the tensor-core forward (transposed register chain;
-// GDN_CHAIN=v2 selects the earlier row-split chain for comparison).
-cudaError_t launch_chain(const FwdArgs &a) {
-    const char *e = getenv("GDN_CHAIN");
-    if (e && strcmp(e, "v2") == 0) return launch_fwd2(a);
-    return launch_fwd3(a);
-}
+// State chain + output of the tensor-core forward.
+cudaError_t launch_chain(const FwdArgs &a) { return launch_fwd3(a); }
 
 int launch_plan(const gdn_problem *p, Plan &P, char *ws, unsigned *status, cudaStream_t st) {
     if (!P.varlen) return GDN_OK;

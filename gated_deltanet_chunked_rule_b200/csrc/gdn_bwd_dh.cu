@@ -14,7 +14,7 @@
 // dh' [NC][Hv][V/32][4][128][8], dDelta [NC][Hv][V/32][4][64][8]; dh0 (fp32) is
 // the gradient at the sequence start.
 //
-// Same organisation as the forward kernel (gdn_fwd2.cu): one CTA per
+// Organised like the forward chain kernel (gdn_fwd3.cu): one CTA per
 // (sequence, value head, 32-column slice of V), w and P = M o Q K^T of every
 // chunk from the chunk-prep kernel through a TMA ring, 416 threads:
 //   warps 0-7   chain: dh' (128 x 32 fp32) in mma.sync fragments; per chunk

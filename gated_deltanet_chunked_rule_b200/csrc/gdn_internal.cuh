@@ -169,7 +169,6 @@ cudaError_t launch_fwd_simt(const FwdArgs &a);
 cudaError_t launch_bwd_simt(const BwdArgs &a, float *dq_part, float *dk_part);
 bool prep_tc_supported(const FwdArgs &a);
 cudaError_t launch_prep_tc(const FwdArgs &a);
-cudaError_t launch_fwd2(const FwdArgs &a);
 cudaError_t launch_fwd3(const FwdArgs &a);
 // Chunk prep of the tensor-core path: gamma, Ainv (optional), w, u, P.
 bool prep3_supported(const FwdArgs &a);

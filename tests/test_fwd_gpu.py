@@ -128,12 +128,12 @@ def test_full_size_workloads(oracle_mod, name):
     run(oracle_mod, WORKLOADS[name])
 
 
-@pytest.mark.parametrize("env", [("GDN_IMPL", "simt"), ("GDN_CHAIN", "v2")])
+@pytest.mark.parametrize("env", [("GDN_IMPL", "simt")])
 def test_tensor_core_and_cuda_core_paths_agree(oracle_mod, monkeypatch, env):
     # K = V = 128 bf16 runs on the tensor-core kernels (transposed register
-    # chain + tcgen05 output) by default; GDN_CHAIN=v2 selects the row-split
-    # chain kernel and GDN_IMPL=simt the fp32 CUDA-core one. Each must meet the
-    # oracle tolerance, and they agree.
+    # chain + tcgen05 output) by default; GDN_IMPL=simt selects the fp32
+    # CUDA-core ones, an independent implementation of the same chunked form.
+    # Each must meet the oracle tolerance, and they agree.
     w = Workload("paths", B=1, T=777, Hq=2, Hv=4, K=128, V=128, h0_std=0.02, seed=8)
     x = make_inputs(w)
     o_tc, f_tc, _ = gpu_fwd(x)
