@@ -2,8 +2,9 @@
 // per-chunk quantity that does not depend on the state, so that the state
 // chains downstream only run their two state-dependent products.
 //
-// One CTA (8 warps) per (64-token chunk, qk head) serves the value heads of the
-// qk head's group. From k, q (per qk head) and v, g, beta (per value head):
+// Persistent CTAs (8 warps, two per SM) walk the (64-token chunk, qk head) items;
+// an item serves the value heads of the qk head's group. From k, q (per qk head)
+// and v, g, beta (per value head):
 //
 //   G     = K K^T,   S = Q K^T                                  (once per qk head)
 //   gamma = in-chunk cumulative sum of g
@@ -14,17 +15,21 @@
 //   Ainv  (bf16 [NC, Hv, 64, 64], for the backward; optional)
 //
 // (the WY form of the chunk: Delta = u - w h, o = scale (diag(e^gamma) Q h + P Delta).)
-// P, u and w of a full chunk are written by TMA stores from swizzled staging
+// The q and k tiles are double-buffered: the next item's load is issued as soon
+// as this item's S and G are formed, so that a whole item's work hides its
+// latency (a load issued at the start of its own item stalled the CTA for about
+// 4 us). P and w of a full chunk are written by TMA stores from swizzled staging
 // tiles (row by row for a ragged one, whose tile would spill into the next
-// sequence). The four bulk products (S, G, u, w) run on tcgen05 from TMA-loaded,
-// 128-byte-swizzled tiles, so their operands never pass through the
-// load/store unit, which the warp-level version of this kernel saturated.
-// The unit lower-triangular inverse is taken block-wise on 16 x 16 blocks in
-// fp32: diagonal blocks by forward substitution, off-diagonal blocks one block
-// diagonal at a time on tf32 MMAs. Rows past the end of a sequence have
-// beta = 0, so their rows of A vanish, the inverse is the identity there and
-// their columns of Ainv diag(beta) are zero: whatever the TMA reads past the
-// end (the next sequence, or zeros) never reaches an output.
+// sequence); u goes out straight from the accumulator registers, four lanes per
+// 32-byte sector. The four bulk products (S, G, u, w) run on tcgen05 from
+// TMA-loaded, 128-byte-swizzled tiles. The unit lower-triangular inverse is
+// taken block-wise on 16 x 16 blocks in fp32, in one work matrix that holds the
+// inverse on and below the diagonal and A transposed above it: diagonal blocks by
+// forward substitution, off-diagonal blocks one block diagonal at a time on tf32
+// MMAs. Rows past the end of a sequence have beta = 0, and a ragged chunk's rows
+// past its end are zeroed in the q, k and v tiles before any product, so that
+// whatever the TMA reads there (the next sequence, or zeros) never reaches an
+// output.
 #include <algorithm>
 #include <cstddef>
 
@@ -43,23 +48,23 @@ constexpr int C = 64, K = 128, V = 128;
 constexpr int kLd = 68;  // row pitch (floats) of the fp32 work matrices
 
 // ---- shared memory (bytes from a 1024-aligned base)
-constexpr int kQV = 0;          // q tile, then the current value head's v tile: [64][128] bf16, 128-byte swizzle, two halves
-constexpr int kKt = 16384;      // k tile, same layout
-constexpr int kAu = 32768;      // Ainv diag(beta): [64][64] bf16, 128-byte swizzle (K-major A operand)
-constexpr int kAw = 40960;      // Ainv diag(beta e^gamma)
-constexpr int kA = 49152;       // float [64][kLd]
-constexpr int kX = kA + 64 * kLd * 4;
-constexpr int kT = kX + 64 * kLd * 4;      // float [3][16][17]: one 16 x 16 block product per warp
+// q and k tiles are double-buffered by item, so that the next item's tiles load while
+// this one is worked on; the item's q slot takes its value heads' v tiles once S is done.
+constexpr int kQ0 = 0;          // 2 x q tile (then v tiles): [64][128] bf16, 128-byte swizzle, two halves
+constexpr int kK0 = 32768;      // 2 x k tile, same layout
+constexpr int kAu = 65536;      // Ainv diag(beta): [64][64] bf16, 128-byte swizzle (K-major A operand)
+constexpr int kAw = 73728;      // Ainv diag(beta e^gamma)
+constexpr int kAX = 81920;      // float [64][kLd]: X = Ainv on and below the diagonal, A^T above it
+constexpr int kT = kAX + 64 * kLd * 4;     // float [3][16][17]: one 16 x 16 block product per warp
 constexpr int kVec = kT + 3 * 16 * 17 * 4;
 constexpr int kBar = kVec + 1024;
-constexpr int kPs = 89088;      // P staging for its TMA store: [64][64] bf16, 128-byte swizzle
+constexpr int kPs = 104448;     // P staging for its TMA store: [64][64] bf16, 128-byte swizzle
 constexpr int kSmemBytes = kPs + 8192 + 1024;
 static_assert(kBar + 64 <= kPs && kPs % 1024 == 0, "shared memory layout");
-// u and w of a full chunk leave through TMA stores from 128-byte-swizzled staging
-// tiles over buffers that are free once the u, w products are complete: u (fp32,
-// four [64][32] tiles) over A and X, w (bf16, two [64][64] halves) over Au, Aw.
-constexpr int kUs = kA, kWs = kAu;
-static_assert(kUs % 1024 == 0 && kUs + 32768 <= kT && kWs + 16384 <= kA, "staging layout");
+// w of a full chunk leaves through TMA stores from a 128-byte-swizzled staging tile
+// (two [64][64] halves) over Au, Aw, free once the u, w products are complete; u
+// (fp32) is stored straight from the accumulator registers.
+constexpr int kWs = kAu;
 static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
 
 // tensor memory: S | G (64 columns each), later u | w (128 columns each)
@@ -116,8 +121,8 @@ struct Prep3Params {
 
 __global__ void __launch_bounds__(kThreads, 2)
 prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_uo,
-             const __grid_constant__ CUtensorMap tm_wo, const __grid_constant__ CUtensorMap tm_po,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_wo,
+             const __grid_constant__ CUtensorMap tm_po,
              const Prep3Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
@@ -128,18 +133,21 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int r0 = 16 * wm + g8, r1 = r0 + 8;
     const int G = d.Hv / d.Hq;
 
-    float(*A)[kLd] = reinterpret_cast<float(*)[kLd]>(smem + kA);
-    float(*X)[kLd] = reinterpret_cast<float(*)[kLd]>(smem + kX);
+    // one fp32 work matrix: X (the inverse) on and below the diagonal, A transposed above it
+    float(*AX)[kLd] = reinterpret_cast<float(*)[kLd]>(smem + kAX);
     float(*T)[16][17] = reinterpret_cast<float(*)[16][17]>(smem + kT);
     float *gam = reinterpret_cast<float *>(smem + kVec);
     float *egam = gam + 64, *bet = gam + 128, *scan = gam + 192;
     uint64_t *tma_bar = reinterpret_cast<uint64_t *>(smem + kBar);
     uint64_t *mma_bar = tma_bar + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tma_bar + 2);
+    uint64_t *qk_bar = tma_bar + 3;  // [2]: the q, k tiles of each buffer
 
     if (tid == 0) {
         mbar_init(tma_bar, 1);
         mbar_init(mma_bar, 1);
+        mbar_init(&qk_bar[0], 1);
+        mbar_init(&qk_bar[1], 1);
         fence_barrier_init();
     }
     if (warp == 0) {
@@ -173,36 +181,50 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tma_prefetch_3d(&tm_v, 64, hq2 * G + gi, t2);
         }
     };
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+    // q, k tiles of the CTA's k-th item go to buffer k % 2 (a consistent sequence table
+    // has an owner for every chunk, an inconsistent one for none, so items are either
+    // all valid or all skipped and the buffer alternation holds)
+    int qk_issued = 0;  // (thread 0) q, k loads issued
+    auto issue_qk = [&](int item) {
+        if (item >= n_items) return;
+        const int cg2 = item / d.Hq, hq2 = item % d.Hq;
+        const int n2 = chunk_owner(d, cg2);
+        if (n2 < 0) return;
+        const SeqRange s2 = seq_range(d, n2);
+        const int t2 = s2.start + (cg2 - s2.chunk0) * C;
+        const int b = qk_issued & 1;
+        mbar_arrive_expect_tx(&qk_bar[b], 4 * 8192);
+        tma_load_3d(smem + kQ0 + b * 16384, &tm_q, &qk_bar[b], 0, hq2, t2);
+        tma_load_3d(smem + kQ0 + b * 16384 + 8192, &tm_q, &qk_bar[b], 64, hq2, t2);
+        tma_load_3d(smem + kK0 + b * 16384, &tm_k, &qk_bar[b], 0, hq2, t2);
+        tma_load_3d(smem + kK0 + b * 16384 + 8192, &tm_k, &qk_bar[b], 64, hq2, t2);
+        ++qk_issued;
+    };
+    if (tid == 0) issue_qk(blockIdx.x);
+    int it_k = 0;  // this CTA's item count
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it_k) {
     const int cg = item / d.Hq, hq = item % d.Hq;
     const int n = chunk_owner(d, cg);
     if (n < 0) continue;  // the whole CTA
     const SeqRange sr = seq_range(d, n);
     const int ci = cg - sr.chunk0;
     const int t0 = sr.start + ci * C, len = min(C, sr.len - ci * C);
-    if (tid == 0) prefetch_item(item + gridDim.x);
+    const int buf = it_k & 1;
+    const uint32_t qv = sb + kQ0 + buf * 16384, kt = sb + kK0 + buf * 16384;  // q (then v), k tiles
+    if (tid == 0) prefetch_item(item + 2 * gridDim.x);
 
-    // ---- q, k tiles by TMA; S = Q K^T and G = K K^T on tcgen05
-    if (tid == 0) {
-        mbar_arrive_expect_tx(tma_bar, 4 * 8192);
-        tma_load_3d(smem + kQV, &tm_q, tma_bar, 0, hq, t0);
-        tma_load_3d(smem + kQV + 8192, &tm_q, tma_bar, 64, hq, t0);
-        tma_load_3d(smem + kKt, &tm_k, tma_bar, 0, hq, t0);
-        tma_load_3d(smem + kKt + 8192, &tm_k, tma_bar, 64, hq, t0);
-        tma_pending = true;
-    }
+    // ---- q, k tiles (loaded during the previous item); S = Q K^T and G = K K^T on tcgen05
     float g_next = 0.f, b_next = 0.f;  // g, beta of the next value head, prefetched
     if (tid < C && tid < len) {
         g_next = prm.g[(size_t)(t0 + tid) * d.Hv + hq * G];
         b_next = prm.beta[(size_t)(t0 + tid) * d.Hv + hq * G];
     }
-    ok = cta_wait(tma_bar, tma_phase & 1);
-    if (ok) ++tma_phase, tma_pending = false;
+    ok = cta_wait(&qk_bar[buf], (it_k >> 1) & 1);
     if (len < C) {
         // a ragged chunk: rows past its end hold the next packed sequence (or zeros); zero them so that
         // a non-finite value there cannot reach this sequence through a product with a zero weight
-        zero_rows(sb + kQV, len, tid);
-        zero_rows(sb + kKt, len, tid);
+        zero_rows(qv, len, tid);
+        zero_rows(kt, len, tid);
         fence_proxy_async();
         __syncthreads();
     }
@@ -211,16 +233,19 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const uint32_t id_S = idesc_bf16(64, 64, false, false);
         for (int ks = 0; ks < 8; ++ks) {
             const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-            mma_bf16(tmem + kColS, smem_desc(sb + kQV + off, 16, 1024, kSw128), smem_desc(sb + kKt + off, 16, 1024, kSw128),
-                     id_S, ks > 0);
-            mma_bf16(tmem + kColG, smem_desc(sb + kKt + off, 16, 1024, kSw128), smem_desc(sb + kKt + off, 16, 1024, kSw128),
-                     id_S, ks > 0);
+            mma_bf16(tmem + kColS, smem_desc(qv + off, 16, 1024, kSw128), smem_desc(kt + off, 16, 1024, kSw128), id_S,
+                     ks > 0);
+            mma_bf16(tmem + kColG, smem_desc(kt + off, 16, 1024, kSw128), smem_desc(kt + off, 16, 1024, kSw128), id_S,
+                     ks > 0);
         }
         mma_commit(mma_bar);
         mma_pending = true;
     }
     ok = ok && cta_wait(mma_bar, mma_phase & 1);
     if (ok) ++mma_phase, mma_pending = false;
+    // the other buffer was last read by the previous item's products, all complete: the next
+    // item's q, k tiles go there now
+    if (ok && tid == 0) issue_qk(item + gridDim.x);
     tc_fence_after();
     // S, G: rows r0, r1, columns 32 wn + 8 j + 2 c4 (+1) -- the warp MMA fragment layout
     float sacc[4][4], gacc[4][4];
@@ -237,8 +262,8 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     __syncthreads();  // q tile and S, G columns free
     auto load_v = [&](int h) {
         mbar_arrive_expect_tx(tma_bar, 2 * 8192);
-        tma_load_3d(smem + kQV, &tm_v, tma_bar, 0, h, t0);
-        tma_load_3d(smem + kQV + 8192, &tm_v, tma_bar, 64, h, t0);
+        tma_load_3d(smem + (qv - sb), &tm_v, tma_bar, 0, h, t0);
+        tma_load_3d(smem + (qv - sb) + 8192, &tm_v, tma_bar, 64, h, t0);
         tma_pending = true;
     };
     if (ok && tid == 0) load_v(hq * G);
@@ -283,9 +308,9 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     const int r = hi ? r1 : r0;
                     const float e0 = s <= r ? __expf(gr[hi] - gs0) : 0.f;
                     const float e1 = s + 1 <= r ? __expf(gr[hi] - gs1) : 0.f;
-                    *reinterpret_cast<float2 *>(&A[r][s]) =
-                        make_float2(s < r ? br[hi] * e0 * gacc[j][2 * hi] : 0.f, s + 1 < r ? br[hi] * e1 * gacc[j][2 * hi + 1] : 0.f);
-                    *reinterpret_cast<float2 *>(&X[r][s]) = make_float2(0.f, 0.f);
+                    // A_rs (s < r) goes transposed above the diagonal; X fills the rest later
+                    if (s < r) AX[s][r] = br[hi] * e0 * gacc[j][2 * hi];
+                    if (s + 1 < r) AX[s + 1][r] = br[hi] * e1 * gacc[j][2 * hi + 1];
                     const bool live = r < len;
                     st_shared_b32(sb + kPs + r * 128 + (((s >> 3) ^ (r & 7)) << 4) + (s & 7) * 2,
                                   pack_bf16(live ? e0 * sacc[j][2 * hi] : 0.f, live ? e1 * sacc[j][2 * hi + 1] : 0.f));
@@ -306,11 +331,13 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             for (int r = 0; r < 16; ++r) {
                 float acc = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-                for (int j = 0; j < r; ++j) acc = fmaf(-A[o + r][o + j], xcol[j], acc);
+                for (int j = 0; j < r; ++j) acc = fmaf(-AX[o + j][o + r], xcol[j], acc);
                 xcol[r] = r < cc ? 0.f : acc;
             }
+            // only on and below the diagonal: above it lies A
 #pragma unroll
-            for (int r = 0; r < 16; ++r) X[o + r][o + cc] = xcol[r];
+            for (int r = 0; r < 16; ++r)
+                if (r >= cc) AX[o + r][o + cc] = xcol[r];
         }
         __syncthreads();
         // ---- off-diagonal blocks, one block diagonal at a time:
@@ -323,12 +350,17 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         const int ac = m * 16 + kk * 8 + c4;
-                        const uint32_t a[4] = {tf32(A[i * 16 + g8][ac]), tf32(A[i * 16 + g8 + 8][ac]),
-                                               tf32(A[i * 16 + g8][ac + 4]), tf32(A[i * 16 + g8 + 8][ac + 4])};
+                        // A_{i,m} (below the diagonal) is stored transposed
+                        const uint32_t a[4] = {tf32(AX[ac][i * 16 + g8]), tf32(AX[ac][i * 16 + g8 + 8]),
+                                               tf32(AX[ac + 4][i * 16 + g8]), tf32(AX[ac + 4][i * 16 + g8 + 8])};
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt) {
                             const int bc = j * 16 + nt * 8 + g8;
-                            mma_tf32(t[nt], a, tf32(X[m * 16 + kk * 8 + c4][bc]), tf32(X[m * 16 + kk * 8 + c4 + 4][bc]));
+                            // X_mj; in a diagonal block (m == j) the entries above the diagonal are zero
+                            const int rr0 = m * 16 + kk * 8 + c4, rr1 = rr0 + 4;
+                            const float x0 = (m == j && bc > rr0) ? 0.f : AX[rr0][bc];
+                            const float x1 = (m == j && bc > rr1) ? 0.f : AX[rr1][bc];
+                            mma_tf32(t[nt], a, tf32(x0), tf32(x1));
                         }
                     }
                 }
@@ -346,8 +378,10 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const int ac = i * 16 + kk * 8 + c4;
-                    const uint32_t a[4] = {tf32(X[i * 16 + g8][ac]), tf32(X[i * 16 + g8 + 8][ac]),
-                                           tf32(X[i * 16 + g8][ac + 4]), tf32(X[i * 16 + g8 + 8][ac + 4])};
+                    // X_ii: zero above the diagonal (A lies there)
+                    const int ra = i * 16 + g8, rb = ra + 8;
+                    const uint32_t a[4] = {tf32(ac > ra ? 0.f : AX[ra][ac]), tf32(ac > rb ? 0.f : AX[rb][ac]),
+                                           tf32(ac + 4 > ra ? 0.f : AX[ra][ac + 4]), tf32(ac + 4 > rb ? 0.f : AX[rb][ac + 4])};
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const int bc = nt * 8 + g8;
@@ -357,10 +391,10 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int col = j * 16 + nt * 8 + 2 * c4;
-                    X[i * 16 + g8][col] = -x[nt][0];
-                    X[i * 16 + g8][col + 1] = -x[nt][1];
-                    X[i * 16 + g8 + 8][col] = -x[nt][2];
-                    X[i * 16 + g8 + 8][col + 1] = -x[nt][3];
+                    AX[i * 16 + g8][col] = -x[nt][0];
+                    AX[i * 16 + g8][col + 1] = -x[nt][1];
+                    AX[i * 16 + g8 + 8][col] = -x[nt][2];
+                    AX[i * 16 + g8 + 8][col + 1] = -x[nt][3];
                 }
             }
             __syncthreads();
@@ -369,7 +403,7 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         //      (the K-major A operands of the u and w products); Ainv -> global (optional)
         for (int e = tid; e < C * C / 2; e += kThreads) {
             const int r = e >> 5, s = (e & 31) * 2;
-            const float x0 = X[r][s], x1 = X[r][s + 1];
+            const float x0 = s <= r ? AX[r][s] : 0.f, x1 = s + 1 <= r ? AX[r][s + 1] : 0.f;
             const float u0 = x0 * bet[s], u1 = x1 * bet[s + 1];
             const uint32_t off = (r >> 3) * 1024 + (r & 7) * 128 + ((((s >> 3) ^ (r & 7))) << 4) + (s & 7) * 2;
             st_shared_b32(sb + kAu + off, pack_bf16(u0, u1));
@@ -384,7 +418,7 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ok = cta_wait(tma_bar, tma_phase & 1);
         if (ok) ++tma_phase, tma_pending = false;
         if (len < C) {
-            zero_rows(sb + kQV, len, tid);  // the v tile's rows past the end, as for q and k
+            zero_rows(qv, len, tid);  // the v tile's rows past the end, as for q and k
             fence_proxy_async();
             __syncthreads();
         }
@@ -393,9 +427,9 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const uint32_t id_W = idesc_bf16(64, 128, false, true);
             for (int ks = 0; ks < 4; ++ks) {
                 mma_bf16(tmem + kColU, smem_desc(sb + kAu + ks * 32, 16, 1024, kSw128),
-                         smem_desc(sb + kQV + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
+                         smem_desc(qv + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
                 mma_bf16(tmem + kColW, smem_desc(sb + kAw + ks * 32, 16, 1024, kSw128),
-                         smem_desc(sb + kKt + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
+                         smem_desc(kt + ks * 2048, 8192, 1024, kSw128), id_W, ks > 0);
             }
             mma_commit(mma_bar);
             mma_pending = true;
@@ -416,11 +450,10 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = hi ? r1 : r0;
-                    const float2 x = make_float2(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
-                    if (full)  // [64][32] fp32 tile per 32 columns: 16-byte chunks XOR (row % 8)
-                        st_shared_v2f(sb + kUs + (col >> 5) * 8192 + r * 128 + ((((col & 31) >> 2) ^ (r & 7)) << 4) + (col & 3) * 4, x.x, x.y);
-                    else if (r < len)
-                        *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r) * d.Hv + h) * V + col) = x;
+                    // u straight to global memory (four lanes write one full 32-byte sector)
+                    if (r < len)
+                        *reinterpret_cast<float2 *>(prm.u_out + ((size_t)(t0 + r) * d.Hv + h) * V + col) =
+                            make_float2(v[4 * i + 2 * hi], v[4 * i + 2 * hi + 1]);
                 }
             }
             tmem_ld16x256_x4(tmem + lane_base + kColW + cb, v);  // w
@@ -453,11 +486,10 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
             }
         }
-        fence_proxy_async();  // u, w -> their TMA stores
+        fence_proxy_async();  // w -> its TMA stores
         tc_fence_before();
-        __syncthreads();  // u, w columns free for the next value head (Au, Aw, A, X once the stores have read them)
+        __syncthreads();  // u, w columns free for the next value head (Au, Aw once the stores have read them)
         if (full && tid == 0) {
-            for (int c = 0; c < 4; ++c) tma_store_3d(&tm_uo, sb + kUs + c * 8192, 32 * c, h, t0);
             tma_store_3d(&tm_wo, sb + kWs, 0, h, t0);
             tma_store_3d(&tm_wo, sb + kWs + 8192, 64, h, t0);
             bulk_commit();
@@ -471,6 +503,12 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (tid == 0) {
             const uint64_t t1 = globaltimer();
             while (tma_pending && !mbar_try_wait(smem_u32(tma_bar), tma_phase & 1) && globaltimer() - t1 < kWaitNs) {
+            }
+            // the last q, k load issued (each buffer has at most one outstanding)
+            if (qk_issued > 0) {
+                const int b = (qk_issued - 1) & 1;
+                while (!mbar_try_wait(smem_u32(&qk_bar[b]), ((qk_issued - 1) >> 1) & 1) && globaltimer() - t1 < kWaitNs) {
+                }
             }
             while (mma_pending && !mbar_try_wait(smem_u32(mma_bar), mma_phase & 1) && globaltimer() - t1 < kWaitNs) {
             }
@@ -492,29 +530,23 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     const Dims &d = a.d;
     if (d.NC == 0) return cudaSuccess;
     if (!a.w16 || !a.u32 || !a.p16 || !a.gamma) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv, muo, mwo, mpo;
+    CUtensorMap mq, mk, mv, mwo, mpo;
     const cuuint64_t T = (cuuint64_t)(d.T_total > 0 ? d.T_total : 1);
     const cuuint64_t dq[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hq, T};
     const cuuint64_t sq[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hq * d.K * 2};
     const cuuint64_t dv[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
     const cuuint64_t sv[2] = {(cuuint64_t)d.V * 2, (cuuint64_t)d.Hv * d.V * 2};
     const cuuint32_t box[3] = {64, 1, 64};
-    // stores: u fp32 [T, Hv, V] in 32-column boxes, w bf16 [T, Hv, K], P bf16 [NC * Hv * 64 rows][64]
-    const cuuint64_t du[3] = {(cuuint64_t)d.V, (cuuint64_t)d.Hv, T};
-    const cuuint64_t su[2] = {(cuuint64_t)d.V * 4, (cuuint64_t)d.Hv * d.V * 4};
-    const cuuint32_t bu[3] = {32, 1, 64};
+    // stores: w bf16 [T, Hv, K], P bf16 [NC * Hv * 64 rows][64] (u is stored from registers)
     const cuuint64_t dw[3] = {(cuuint64_t)d.K, (cuuint64_t)d.Hv, T};
     const cuuint64_t sw[2] = {(cuuint64_t)d.K * 2, (cuuint64_t)d.Hv * d.K * 2};
     const cuuint64_t dp[2] = {64, (cuuint64_t)d.NC * d.Hv * 64};
     const cuuint64_t sp[1] = {128};
     const cuuint32_t bp[2] = {64, 64};
     auto enc = tensor_map_encoder();
-    cuuint32_t estr[3] = {1, 1, 1};
     if (!enc || !make_bf16_map(&mq, a.q, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_bf16_map(&mk, a.k, 3, dq, sq, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_bf16_map(&mv, a.v, 3, dv, sv, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        enc(&muo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.u32, du, su, bu, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
         !make_bf16_map(&mwo, a.w16, 3, dw, sw, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_bf16_map(&mpo, a.p16, 2, dp, sp, bp, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -538,7 +570,7 @@ cudaError_t launch_prep3(const FwdArgs &a) {
     const long long items = (long long)d.NC * d.Hq;
     if (items >= (1ll << 31)) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(items, 2ll * sms);  // persistent, two CTAs per SM
-    prep3_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, muo, mwo, mpo, p);
+    prep3_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, mwo, mpo, p);
     return cudaGetLastError();
 }
 
