@@ -14,23 +14,42 @@
 // dh' [NC][Hv][V/32][4][128][8], dDelta [NC][Hv][V/32][4][64][8]; dh0 (fp32) is
 // the gradient at the sequence start.
 //
-// Organised like the forward chain kernel (gdn_fwd3.cu): one CTA per
-// (sequence, value head, 32-column slice of V), w and P = M o Q K^T of every
-// chunk from the chunk-prep kernel through a TMA ring, 416 threads:
-//   warps 0-7   chain: dh' (128 x 32 fp32) in mma.sync fragments; per chunk
-//               A = K dh', dDelta = e^{gamma_C - gamma} A + scale Y, then
-//               dh = e^{gamma_C} dh' + X - w^T dDelta, with Y and X read
-//               straight from tensor memory (the 16x256b load layout is the
-//               mma.sync accumulator layout, and chain warp p sits on TMEM
-//               sub-partition p);
-//   warps 8-11  aux: dO' = scale e^gamma o dO into shared memory, one chunk
-//               ahead of the chain, and the copies of dh' and dDelta from
-//               shared memory to global memory, off the chain's path;
-//   warp 12     issuer: TMA ring (q, k, w, P, dO per chunk) and, on tcgen05,
-//               Y = P^T dO and X = Q^T dO' into double-buffered TMEM.
-// Y and X do not depend on the chain, so they are ready one or two chunks
-// ahead of it. Hand-over by release/acquire counters and mbarriers; every wait
-// is bounded.
+// Organised like the forward chain kernel (gdn_fwd3.cu), whose chain this one
+// mirrors: one CTA per (sequence, value head, 32-column slice of V), and the
+// scan runs on the transposed gradient dh'^T (rows: value columns v, columns:
+// key dimensions d), held in fp32 registers by four chain warps (warp x: the
+// state for d in [32x, 32x+32), dDelta for the tokens [16x, 16x+16)):
+//
+//   D1 = dh'^T K^T                       (v x tokens, contraction over d)
+//   dDelta^T = e^{gamma_C - gamma} o D1 + scale Y^T,      Y^T = dO^T P
+//   dh^T = e^{gamma_C} dh'^T + X^T - dDelta^T w,           X^T = dO'^T Q,  dO' = scale e^gamma o dO
+//
+// D1 and the update are warp-level MMAs whose A operands (the state, dDelta)
+// come from the accumulators of the previous product; the quarters the warps
+// exchange pass through shared memory in bf16. Y^T and X^T do not depend on
+// the chain: they run on tcgen05 one or two chunks ahead, with M = 128 rows
+// that repeat the slice's 32 value columns four times (the dO tile read with a
+// zero stride between its 32-column atoms), so that every chain warp finds all
+// 32 value rows in its own TMEM lane quarter, in the mma.sync accumulator
+// layout of the 16x256b load, and adds them to its fragments directly.
+//
+// Warp roles (320 threads):
+//   warps 0-3  chain (above).
+//   warps 4-7  dO' = scale e^gamma o dO into shared memory (one warp per
+//              scheduler), then one of their threads issues the X^T MMAs.
+//   warp 8     issuer: the (q, P, dO) TMA ring and the Y^T MMAs.
+// Y^T and X^T go into double-buffered tensor memory, each chunk's pair
+// completing one mbarrier (an arrival from each issuing thread): a single
+// thread spends tens of cycles per tcgen05.mma, so the two products are
+// issued side by side.
+//   warp 9     producer: the (k, w) TMA ring with each chunk's gates, and the
+//              bulk copies of dh' and dDelta to global memory. (L2 prefetches
+//              a few chunks ahead, as the forward chain issues them, measured
+//              a few percent slower here.)
+// Hand-over by mbarriers (hardware completions, the chain's per-chunk
+// hand-over) and release/acquire counters ("buffer free" conditions); every
+// wait is bounded, and a wait that expires records GDN_ERR_TIMEOUT and winds
+// the CTA down after draining its TMA loads and MMAs in flight.
 //
 // Sequence split (long sequences, few heads): a chunk maps its exit-state
 // gradient dh' to dh = A dh' + b with A = e^{gamma_C} I - w^T diag(e^{gamma_C -
@@ -40,6 +59,10 @@
 // on K more columns whose dO tile is read out of range (zero), so Y = X = 0
 // there. A composition walks the segments backwards from dht (gdn_split.cu), and
 // the output pass reruns every segment from its composed dh_end.
+//
+// Rows past the end of a ragged chunk: dDelta is zero there (a select), and the
+// w rows they meet in the update are zeroed in shared memory first, so that
+// whatever follows the sequence in memory cannot turn 0 * x into NaN in dh.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -52,44 +75,50 @@ namespace {
 using namespace sm100;
 using namespace warp;
 
-constexpr int kThreads = 416;
-constexpr int kRole = 256;  // chain threads
-constexpr int kAux = 128;
+constexpr int kChainWarps = 4;
+constexpr int kAuxWarp0 = 4;  // warps 4..7
+constexpr int kIssuerWarp = 8;
+constexpr int kProdWarp = 9;
+constexpr int kThreads = 10 * 32;
+static_assert(kThreads == (kProdWarp + 1) * 32, "the producer is the last warp");
 constexpr int kBV = 32;
-constexpr int kStages = 3;
+constexpr int kCS = 3;        // chain ring stages (k, w)
+constexpr int kOS = 3;        // Y / X ring stages (q, P, dO)
+constexpr int kHB = 2;        // dh' / dDelta buffers (chain -> copies)
 
 // ---- shared memory (bytes from a 1024-aligned base)
-constexpr int kHb = 0;          // 8192       dh' (bf16): (n/8)*2048 + (k/8)*128 + (k%8)*16
-constexpr int kDb = 8192;       // 4096       -dDelta (bf16): (n/8)*1024 + (t/8)*128 + (t%8)*16
-constexpr int kDO2 = 12288;     // 2 x 4096   dO' (bf16), layout of kDb (B of X)
-constexpr int kStage0 = 20480;  // TMA ring
-// per stage: q, k, w [64][128] bf16 (two 64-column halves, 128-byte swizzle),
-// P [64][64] bf16 (128-byte swizzle), dO [64][32] bf16 (64-byte swizzle)
-constexpr int kQ = 0, kK = 16384, kW = 32768, kP = 49152, kDO = 57344, kStageBytes = 61440;
-constexpr int kTxBytes = 3 * 16384 + 8192 + 4096;
-constexpr int kSmall = kStage0 + kStages * kStageBytes;
+constexpr int kC0 = 0;  // chain ring: k, w [64][128] bf16 (two 64-column halves, 128-byte swizzle)
+constexpr int kK = 0, kW = 16384, kCStageBytes = 32768;
+constexpr int kO0 = kC0 + kCS * kCStageBytes;  // Y / X ring: q [64][128], P [64][64] (128-byte
+                                               // swizzle), dO [64][32] bf16 (64-byte swizzle)
+constexpr int kQ = 0, kP = 16384, kDO = 24576, kOStageBytes = 28672;
+constexpr int kHb = kO0 + kOS * kOStageBytes;  // kHB x 8192: dh'^T (bf16): (v/8)*2048 + d*16 + (v%8)*2
+constexpr int kDb = kHb + kHB * 8192;          // kHB x 4096: dDelta (bf16): (v/8)*1024 + t*16 + (v%8)*2
+constexpr int kXb = kDb + kHB * 4096;          // 4096: -dDelta^T A fragments, [group][quarter][lane] x 16 bytes
+constexpr int kDO2 = kXb + 4096;               // 2 x 4096: dO' in the layout of the dO tile
+constexpr int kGam = kDO2 + 2 * 4096;          // kCS x 64 fp32: gamma of each staged chunk
+constexpr int kSmall = kGam + 1024;
 constexpr int kSmemBytes = kSmall + 2048 + 1024;
-static_assert(kStage0 % 1024 == 0 && kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory layout");
+static_assert(kO0 % 1024 == 0 && kHb % 1024 == 0 && kDO2 % 1024 == 0 && kOStageBytes % 1024 == 0 &&
+                  kCS * 64 * 4 <= 1024 && kSmemBytes <= 232448,
+              "shared memory layout");
 
-// Tensor memory: two buffers of 64 columns, Y (M = 64) | X (M = 128).
-constexpr uint32_t kColY = 0, kColX = 32, kYBuf = 64, kTmemCols = 128;
+// Y^T (M = 128, N = 64 tokens) and X^T (M = 128, N = 128 key dims), double-buffered.
+constexpr uint32_t kColY = 0, kColX = 64, kYXBuf = 192, kTmemCols = 512;
 
-// kHbFull / kDbFull: the chain has put dh' / -dDelta of an iteration in kHb / kDb;
-// kHbRead / kDbRead: the aux warps have copied them to global memory.
-enum Ctr { kPReady, kStage, kHbFull, kDbFull, kHbRead, kDbRead, kNumCtr };
+// Counters: kTRead iterations whose Y^T, X^T the chain has read out of tensor
+// memory; kStored iterations whose dh' / dDelta copies have finished reading
+// shared memory.
+enum Ctr { kTRead, kStored, kNumCtr };
 
 struct Small {
-    uint64_t full[kStages];
-    uint64_t mmaB[2];
+    uint64_t cfull[kCS], cempty[kCS], ofull[kOS], hready[kHB], mmaB[2];
     uint32_t ctr[kNumCtr];
-    int loads_issued, loads_landed, mma_issued, mma_seen;
+    int c_issued[kCS], o_issued[kOS], y_issued[2], x_issued[2];
     uint32_t tmem_base;
     int abort_flag;
 };
 static_assert(sizeof(Small) <= 2048, "small area");
-
-__device__ __forceinline__ bool chain_sync(bool pred) { return role_sync_and<kRole>(1, pred); }
-__device__ __forceinline__ bool aux_sync(bool pred) { return role_sync_and<kAux>(2, pred); }
 
 struct BwdDhParams {
     Dims d;
@@ -112,6 +141,26 @@ struct BwdDhParams {
 
 enum BwdDhMode { kBWhole = 0, kBSegPass = 1, kBSegOut = 2 };
 
+// Waits for the six 16x256b.x2 TMEM loads of a chain step (see tmem_wait_ld).
+__device__ __forceinline__ void tmem_wait_ld6(uint32_t (&a)[8], uint32_t (&b)[8], uint32_t (&c)[8], uint32_t (&e)[8],
+                                              uint32_t (&f)[8], uint32_t (&g)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                   "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
+                   "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3]), "+r"(c[4]), "+r"(c[5]), "+r"(c[6]), "+r"(c[7]),
+                   "+r"(e[0]), "+r"(e[1]), "+r"(e[2]), "+r"(e[3]), "+r"(e[4]), "+r"(e[5]), "+r"(e[6]), "+r"(e[7]),
+                   "+r"(f[0]), "+r"(f[1]), "+r"(f[2]), "+r"(f[3]), "+r"(f[4]), "+r"(f[5]), "+r"(f[6]), "+r"(f[7]),
+                   "+r"(g[0]), "+r"(g[1]), "+r"(g[2]), "+r"(g[3]), "+r"(g[4]), "+r"(g[5]), "+r"(g[6]), "+r"(g[7])
+                 :
+                 : "memory");
+}
+
+// Byte offset of (row, col) in a [rows][128] bf16 tile stored as two 64-column
+// halves of 128-byte rows with 128-byte swizzle (what the TMA loads produce).
+__device__ __forceinline__ uint32_t sw_off(int row, int col) {
+    return (uint32_t)((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_p,
@@ -121,6 +170,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
     volatile int *abort_flag = &sm->abort_flag;
     const uint32_t sb = smem_u32(smem);
+    float *gam = reinterpret_cast<float *>(smem + kGam);
 
     const Dims &d = prm.d;
     const int nseg = prm.nseg;
@@ -131,6 +181,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int c0 = zs * kBV;
     const int hq = h / (d.Hv / d.Hq);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int K = 128, V = 128;
     // this CTA's chunks [j0, j1) of the sequence, seen as a sequence of their own
     const SeqRange seq = seq_range(d, n);
     const int nch_seq = (seq.len + kChunk - 1) / kChunk;
@@ -143,18 +194,27 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int nch = j1 - j0;
     const size_t seg_idx = (size_t)n * nseg + sseg;
     const bool outputs = prm.mode != kBSegPass;  // dh' and dDelta of every chunk
-    constexpr int K = 128, V = 128;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm->full[s], 1);
-        mbar_init(&sm->mmaB[0], 1);
-        mbar_init(&sm->mmaB[1], 1);
+        for (int s = 0; s < kCS; ++s) {
+            mbar_init(&sm->cfull[s], 1);
+            mbar_init(&sm->cempty[s], kChainWarps);
+            sm->c_issued[s] = 0;
+        }
+        for (int s = 0; s < kOS; ++s) {
+            mbar_init(&sm->ofull[s], 1);
+            sm->o_issued[s] = 0;
+        }
+        for (int b = 0; b < kHB; ++b) mbar_init(&sm->hready[b], kChainWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm->mmaB[b], 2);  // the Y^T and the X^T issuer
+            sm->y_issued[b] = sm->x_issued[b] = 0;
+        }
         for (int c = 0; c < kNumCtr; ++c) sm->ctr[c] = 0;
-        sm->loads_issued = sm->loads_landed = sm->mma_issued = sm->mma_seen = 0;
         sm->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 12) {
+    if (warp == kIssuerWarp) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -166,18 +226,16 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // iteration it handles chunk nch - 1 - it of the sequence
     auto chunk_of = [&](int it) { return nch - 1 - it; };
-    auto gamma_at = [&](int it, int r) {
-        const int ci = chunk_of(it), len = min(kChunk, sr.len - ci * kChunk);
-        return prm.gamma[(size_t)(sr.start + ci * kChunk + min(r, len - 1)) * d.Hv + h];
-    };
+    auto chunk_len = [&](int it) { return min(kChunk, sr.len - chunk_of(it) * kChunk); };
 
-    if (warp < 8) {
+    if (warp < kChainWarps) {
         // =========================================================== chain
-        const int p = warp & 3, cb = (warp >> 2) * 2;  // state rows 32p.., n-tiles cb, cb+1
-        const int g = lane >> 2, c4 = lane & 3;
-        const uint32_t lane_base = (uint32_t)(p * 32) << 16;
+        const int x = warp;  // d quarter of the state, token quarter of dDelta
+        const int g = lane >> 2, cq = lane & 3, li = lane & 7, mi = lane >> 3;
+        const uint32_t gam_sb = sb + kGam;
         const float scl = prm.scale;
-        float hf[2][2][4];  // [m-tile][n-tile][frag]: rows 32p+16mt+g(+8), cols 8(cb+nt)+2c4(+1)
+        // hs[mt][nt][e]: dh'^T[v = 16mt + g + 8(e>>1)][d = 32x + 8nt + 2cq + (e&1)]
+        float hs[2][4][4];
         {
             const float *src = prm.mode == kBWhole ? (prm.dht ? prm.dht + ((size_t)n * d.Hv + h) * K * V : nullptr)
                                : prm.mode == kBSegOut ? prm.seg_dh + (seg_idx * d.Hv + h) * K * V
@@ -186,142 +244,205 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int dim = 32 * p + 16 * mt + g + ((q >> 1) << 3);
-                        const int col = 8 * (cb + nt) + 2 * c4 + (q & 1);
-                        hf[mt][nt][q] = src ? src[(size_t)dim * V + c0 + col] : (ident && dim == c0 - V + col ? 1.f : 0.f);
+                    for (int e = 0; e < 4; ++e) {
+                        const int v = 16 * mt + g + 8 * (e >> 1), dd = 32 * x + 8 * nt + 2 * cq + (e & 1);
+                        hs[mt][nt][e] = src ? src[(size_t)dd * V + c0 + v] : (ident && dd == c0 - V + v ? 1.f : 0.f);
                     }
         }
-        auto write_hb = [&]() {
-            const uint32_t base = sb + kHb + c4 * 4;
+        bool ok = true;
+        for (int it = 0; it < nch; ++it) {
+            const int s = it % kCS, hb = it % kHB;
+            const int len = chunk_len(it);
+            const uint32_t st = sb + kC0 + s * kCStageBytes;
+            const uint32_t hbuf = sb + kHb + hb * 8192, dbuf = sb + kDb + hb * 4096;
+            bool good = wait_bar(&sm->cfull[s], (it / kCS) & 1, abort_flag);
+            if (lane == 0 && outputs && it >= kHB)  // buffer hb was last copied out for iteration it - kHB
+                good = good && wait_ge(&ctr[kStored], it - kHB + 1, abort_flag);
+            good = __all_sync(0xffffffffu, good);
+            // own quarter of dh' as bf16 A fragments: ao[mt][kk] for k-step 2x + kk
+            uint32_t ao[2][2][4];
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int dim = 32 * p + 16 * mt + g + half * 8;
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        st_shared_b32(base + (cb + nt) * 2048 + (dim >> 3) * 128 + (dim & 7) * 16,
-                                      pack_bf16(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]));
+                for (int kk = 0; kk < 2; ++kk) {
+                    ao[mt][kk][0] = pack_bf16(hs[mt][2 * kk][0], hs[mt][2 * kk][1]);
+                    ao[mt][kk][1] = pack_bf16(hs[mt][2 * kk][2], hs[mt][2 * kk][3]);
+                    ao[mt][kk][2] = pack_bf16(hs[mt][2 * kk + 1][0], hs[mt][2 * kk + 1][1]);
+                    ao[mt][kk][3] = pack_bf16(hs[mt][2 * kk + 1][2], hs[mt][2 * kk + 1][3]);
                 }
-        };
-        write_hb();
-        bool ok = true;
-        float gl = 0.f, gt0 = 0.f, gt1 = 0.f;
-        if (nch > 0) gl = gamma_at(0, 63), gt0 = gamma_at(0, 16 * p + g), gt1 = gamma_at(0, 16 * p + g + 8);
-        for (int it = 0; it < nch && ok; ++it) {
-            const int ci = chunk_of(it);
-            const int len = min(kChunk, sr.len - ci * kChunk);
-            const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
-            // stage landed (and every warp's dh' is in kHb: the barrier orders them)
-            ok = chain_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag));
-            if (!ok) break;
-            if (tid == 0) {
-                sm->loads_landed = it + 1;
-                publish(&ctr[kHbFull], it + 1);  // kHb holds dh' of this chunk (written before the barrier)
-            }
-            const float gC = gl, gtok[2] = {gt0, gt1};
-            if (it + 1 < nch) gl = gamma_at(it + 1, 63), gt0 = gamma_at(it + 1, 16 * p + g), gt1 = gamma_at(it + 1, 16 * p + g + 8);
-            // ---- Y and X of this chunk from tensor memory (issued now, waited after A)
-            // Y, X of this chunk computed; the aux has copied the previous -dDelta out of kDb
-            ok = chain_sync(wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag) &&
-                            (tid != 0 || it < 1 || wait_ge(&ctr[kDbRead], it, abort_flag)));
-            if (!ok) break;
-            if (tid == 0) sm->mma_seen = it + 1;
-            tc_fence_after();
-            uint32_t yr[8], xr0[8], xr1[8];
-            {
-                const uint32_t tb = tmem + (it & 1) * kYBuf + 8 * cb;
-                tmem_ld16x256_x2_nowait(tb + lane_base + kColY, yr);                       // tokens 16p + (g, g+8)
-                tmem_ld16x256_x2_nowait(tb + lane_base + kColX, xr0);                      // state rows 32p + (g, g+8)
-                tmem_ld16x256_x2_nowait(tb + lane_base + ((uint32_t)16 << 16) + kColX, xr1);  // rows 32p + 16 + ..
-            }
-            // ---- A = K dh' : tokens 16p..16p+15, columns of n-tiles cb, cb+1
-            float acc[2][4] = {};
-            {
-                const uint32_t kt = st + kK;
-                const int arow = 16 * p + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int mi = lane >> 3;
-                uint32_t a[2][4], b[2][4];
-                auto load = [&](int ks, int buf) {
-                    const int d0 = 16 * ks + (lane >> 4) * 8;
-                    ldsm_x4(a[buf], kt + (d0 >> 6) * 8192 + arow * 128 + ((((d0 & 63) >> 3) ^ (arow & 7)) << 4));
-                    ldsm_x4_t(b[buf], sb + kHb + (cb + (mi >> 1)) * 2048 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
-                };
-                load(0, 0);
+            // D1 accumulators [m-tile][token n-tile], two independent sets (even / odd k-steps)
+            float acc[2][2][4] = {}, acc2[2][2][4] = {};
+            float gC = 0.f, sc[2][2] = {};
+            uint32_t bk[8][4];  // K fragments (B of D1): bk[2 o + kk] is k-step 2((x + o) & 3) + kk
+            if (good) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    if (ks + 1 < 8) load(ks + 1, (ks + 1) & 1);
-                    hmma(acc[0], a[ks & 1], b[ks & 1][0], b[ks & 1][1]);
-                    hmma(acc[1], a[ks & 1], b[ks & 1][2], b[ks & 1][3]);
-                }
-            }
-            tmem_wait_ld3(yr, xr0, xr1);
-            tc_fence_before();
-            // ---- dDelta = e^{gamma_C - gamma} A + scale Y; -dDelta -> kDb
-            {
-                const uint32_t db = sb + kDb + c4 * 4;
+                for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int tok = 16 * p + g + half * 8;
-                    const bool live = tok < len;
-                    const float sc = __expf(gC - gtok[half]);
-                    const uint32_t off = (tok >> 3) * 128 + (tok & 7) * 16;
+                    for (int kk = 0; kk < 2; ++kk)
+                        stsm_x4_t(hbuf + (2 * mt + (mi & 1)) * 2048 + (32 * x + 16 * kk + 8 * (mi >> 1) + li) * 16,
+                                  ao[mt][kk]);
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const float y0 = __uint_as_float(yr[4 * nt + 2 * half]), y1 = __uint_as_float(yr[4 * nt + 2 * half + 1]);
-                        const float x0 = live ? fmaf(sc, acc[nt][2 * half], scl * y0) : 0.f;
-                        const float x1 = live ? fmaf(sc, acc[nt][2 * half + 1], scl * y1) : 0.f;
-                        st_shared_b32(db + (cb + nt) * 1024 + off, pack_bf16(-x0, -x1));
+                for (int o = 0; o < 4; ++o)
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        ldsm_x4(bk[2 * o + kk],
+                                st + kK + sw_off(16 * x + 8 * (mi >> 1) + li, 16 * (2 * ((x + o) & 3) + kk) + 8 * (mi & 1)));
+                const uint32_t gm = gam_sb + s * kChunk * 4;
+                gC = ld_shared_f32(gm + (kChunk - 1) * 4);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) sc[nt][e] = __expf(gC - ld_shared_f32(gm + (16 * x + 8 * nt + 2 * cq + e) * 4));
+                if (len < kChunk) {
+                    // a ragged chunk: zero the w rows past its end (their dDelta is zero, but a
+                    // non-finite value of the next packed sequence would still turn 0 * x into NaN
+                    // in the update); the barrier below orders this before every update load
+                    for (int i = tid; i < (kChunk - len) * 16; i += kChainWarps * 32) {
+                        const int r = len + (i >> 4), c = i & 15;
+                        st_shared_v4(st + kW + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
                     }
                 }
-            }
-            chain_sync(true);  // every warp reads all 64 tokens of dDelta below
-            if (tid == 0) publish(&ctr[kDbFull], it + 1);
-            // ---- dh = e^{gamma_C} dh' + X + w^T (-dDelta) : rows 32p..+31, 16 columns, K = 64 tokens
-            {
-                const float eC = __expf(gC);
+                // D1 over this warp's own quarter of d (registers): k-steps 2x, 2x+1
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
-                    const uint32_t(&xr)[8] = mt ? xr1 : xr0;
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) hf[mt][nt][q] = fmaf(eC, hf[mt][nt][q], __uint_as_float(xr[4 * nt + q]));
-                }
-                const uint32_t wt = st + kW;
-                const int mi = lane >> 3;
-                uint32_t b[2][4], a[2][2][4];
-                auto load = [&](int ks, int buf) {
-                    ldsm_x4_t(b[buf], sb + kDb + (cb + (mi >> 1)) * 1024 + (2 * ks + (mi & 1)) * 128 + (lane & 7) * 16);
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        // A = w^T rows (state rows) 32p+16mt.., cols (tokens) 16ks..: the
-                        // token-major, 128-byte-swizzled w tile read transposed
-                        const int tt = 16 * ks + (lane & 7) + ((mi >> 1) & 1) * 8;
-                        const int dd = 32 * p + 16 * mt + (mi & 1) * 8;
-                        ldsm_x4_t(a[buf][mt], wt + (dd >> 6) * 8192 + tt * 128 + ((((dd & 63) >> 3) ^ (tt & 7)) << 4));
-                    }
-                };
-                load(0, 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    if (ks + 1 < 4) load(ks + 1, (ks + 1) & 1);
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        hmma(hf[mt][0], a[ks & 1][mt], b[ks & 1][0], b[ks & 1][1]);
-                        hmma(hf[mt][1], a[ks & 1][mt], b[ks & 1][2], b[ks & 1][3]);
-                    }
+                    hmma(acc[mt][0], ao[mt][0], bk[0][0], bk[0][1]);
+                    hmma(acc[mt][1], ao[mt][0], bk[0][2], bk[0][3]);
+                    hmma(acc2[mt][0], ao[mt][1], bk[1][0], bk[1][1]);
+                    hmma(acc2[mt][1], ao[mt][1], bk[1][2], bk[1][3]);
                 }
             }
-            // all reads of kHb, kDb, the stage and this TMEM buffer are done; dh' of this
-            // chunk has been copied out of kHb
-            ok = chain_sync(tid != 0 || wait_ge(&ctr[kHbRead], it + 1, abort_flag));
+            ok = role_sync_and<128>(1, good);  // every quarter of dh' is in hbuf
             if (!ok) break;
-            if (tid == 0) publish(&ctr[kStage], it + 1);
-            write_hb();
+            // Y^T and X^T of this chunk (issued a chunk or more ahead): this warp's token quarter
+            // of Y^T and d quarter of X^T for all 32 value rows (lanes 32x + 16mt + .., the
+            // M = 128 rows repeating the slice), loaded now and waited for after D1
+            bool yx = true;
+            if (lane == 0) yx = wait_bar(&sm->mmaB[it & 1], (it >> 1) & 1, abort_flag);
+            __syncwarp();
+            tc_fence_after();
+            uint32_t yr[2][8], xr[2][2][8];
+            {
+                const uint32_t tb = tmem + (it & 1) * kYXBuf;
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint32_t lb = (uint32_t)(32 * x + 16 * mt) << 16;
+                    tmem_ld16x256_x2_nowait(tb + lb + kColY + 16 * x, yr[mt]);
+                    tmem_ld16x256_x2_nowait(tb + lb + kColX + 32 * x, xr[mt][0]);
+                    tmem_ld16x256_x2_nowait(tb + lb + kColX + 32 * x + 16, xr[mt][1]);
+                }
+            }
+            // D1 over the other three quarters, A fragments of dh' from hbuf
+#pragma unroll
+            for (int o = 1; o < 4; ++o) {
+                uint32_t ah[2][2][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        ldsm_x4_t(ah[mt][kk], hbuf + (2 * mt + (mi & 1)) * 2048 +
+                                                  (16 * (2 * ((x + o) & 3) + kk) + 8 * (mi >> 1) + li) * 16);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        float(&A)[2][2][4] = kk ? acc2 : acc;
+                        hmma(A[mt][0], ah[mt][kk], bk[2 * o + kk][0], bk[2 * o + kk][1]);
+                        hmma(A[mt][1], ah[mt][kk], bk[2 * o + kk][2], bk[2 * o + kk][3]);
+                    }
+            }
+            tmem_wait_ld6(yr[0], yr[1], xr[0][0], xr[0][1], xr[1][0], xr[1][1]);
+            tc_fence_before();
+            // dDelta = e^{gamma_C - gamma} D1 + scale Y on live tokens (a select, so nothing past
+            // the end leaks in); -dDelta^T as the A fragment of the update for this token quarter
+            uint32_t da[2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                float dl[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dl[nt][e] = 16 * x + 8 * nt + 2 * cq + (e & 1) < len
+                                        ? fmaf(sc[nt][e & 1], acc[mt][nt][e] + acc2[mt][nt][e],
+                                               scl * __uint_as_float(yr[mt][4 * nt + e]))
+                                        : 0.f;
+                uint32_t du[4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    da[mt][2 * nt] = pack_bf16(-dl[nt][0], -dl[nt][1]);
+                    da[mt][2 * nt + 1] = pack_bf16(-dl[nt][2], -dl[nt][3]);
+                    du[2 * nt] = pack_bf16(dl[nt][0], dl[nt][1]);
+                    du[2 * nt + 1] = pack_bf16(dl[nt][2], dl[nt][3]);
+                }
+                // A fragment order: (v 0-7, t 0-7), (v 8-15, t 0-7), (v 0-7, t 8-15), (v 8-15, t 8-15)
+                st_shared_v4(sb + kXb + (mt * 4 + x) * 512 + lane * 16, da[mt][0], da[mt][1], da[mt][2], da[mt][3]);
+                if (outputs) stsm_x4_t(dbuf + (2 * mt + (mi & 1)) * 1024 + (16 * x + 8 * (mi >> 1) + li) * 16, du);
+            }
+            // w fragments (B of the update): bw[o] is token quarter (x + o) & 3, this warp's d quarter
+            uint32_t bw[4][2][4];
+#pragma unroll
+            for (int o = 0; o < 4; ++o)
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    const int tq = (x + o) & 3;
+                    ldsm_x4_t(bw[o][np], st + kW + sw_off(16 * tq + 8 * (mi & 1) + li, 32 * x + 16 * np + 8 * (mi >> 1)));
+                }
+            const float eC = __expf(gC);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        hs[mt][nt][e] = fmaf(eC, hs[mt][nt][e], __uint_as_float(xr[mt][nt >> 1][4 * (nt & 1) + e]));
+            // update for the own token quarter: dh^T[:, own d quarter] += (-dDelta)^T w
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    hmma(hs[mt][2 * np], da[mt], bw[0][np][0], bw[0][np][1]);
+                    hmma(hs[mt][2 * np + 1], da[mt], bw[0][np][2], bw[0][np][3]);
+                }
+            // every token quarter of -dDelta^T is in kXb, and every warp has read Y^T, X^T
+            ok = role_sync_and<128>(1, __all_sync(0xffffffffu, yx));
+            if (!ok) break;
+            if (tid == 0) publish(&ctr[kTRead], it + 1);
+            {
+                float h2[2][4][4] = {};  // second accumulator set (latency)
+#pragma unroll
+                for (int o = 1; o < 4; ++o) {
+                    uint32_t pa[2][4];
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        const uint4 p = ld_shared_v4(sb + kXb + (mt * 4 + ((x + o) & 3)) * 512 + lane * 16);
+                        pa[mt][0] = p.x, pa[mt][1] = p.y, pa[mt][2] = p.z, pa[mt][3] = p.w;
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int np = 0; np < 2; ++np) {
+                            float(&H)[2][4][4] = (o & 1) ? h2 : hs;
+                            hmma(H[mt][2 * np], pa[mt], bw[o][np][0], bw[o][np][1]);
+                            hmma(H[mt][2 * np + 1], pa[mt], bw[o][np][2], bw[o][np][3]);
+                        }
+                }
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) hs[mt][nt][e] += h2[mt][nt][e];
+            }
+            // dh' and dDelta of this chunk (generic writes) go to the bulk copies (async
+            // proxy); the stage is free for the producer, and kXb for the next chunk
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                if (outputs) mbar_arrive(&sm->hready[hb]);
+                mbar_arrive(&sm->cempty[s]);
+            }
         }
         if (!ok) {
             if (tid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
@@ -341,149 +462,110 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const int dim = 32 * p + 16 * mt + g + half * 8;
-                            *reinterpret_cast<float2 *>(dst + (size_t)dim * ld + 8 * (cb + nt) + 2 * c4) =
-                                make_float2(hf[mt][nt][2 * half], hf[mt][nt][2 * half + 1]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int v = 16 * mt + g + 8 * (e >> 1), dd = 32 * x + 8 * nt + 2 * cq + (e & 1);
+                            dst[(size_t)dd * ld + v] = hs[mt][nt][e];
                         }
             }
         }
-    } else if (warp < 12) {
-        // ============================================================= aux
-        const int atid = tid - kRole;
+    } else if (warp < kAuxWarp0 + 4) {
+        // ======================================================= dO' makers
+        // dO' = scale e^gamma o dO of iteration it, in the layout of the dO tile (a row of 32
+        // values is 64 contiguous bytes whatever the swizzle), once the tile has landed and
+        // X^T of iteration it - 2 (the buffer's last reader) has been read by the chain; then
+        // thread 0 of the role issues X^T
+        const int at = tid - kAuxWarp0 * 32;
         const float scl = prm.scale;
         bool ok = true;
-        // thread: 16-byte chunks e = atid and atid + 128 of the 64 x 32 dO tile
-        const int ta = atid >> 2, tb2 = (atid + kAux) >> 2, cc = atid & 3;
-        float ga = 0.f, gb = 0.f;
-        if (nch > 0) ga = gamma_at(0, ta), gb = gamma_at(0, tb2);
-        // dO' of iteration it into dO'[it % 2] once its stage has landed and X of
-        // iteration it - 2 (the buffer's last reader) is done
-        auto make_do = [&](int it) -> bool {
-            const int ci = chunk_of(it);
-            const int len = min(kChunk, sr.len - ci * kChunk);
-            if (!aux_sync(wait_bar(&sm->full[it % kStages], (it / kStages) & 1, abort_flag) &&
-                          (atid != 0 || it < 2 || wait_ge(&ctr[kStage], it - 1, abort_flag))))
-                return false;
-            const float fa = ta < len ? scl * __expf(ga) : 0.f, fb = tb2 < len ? scl * __expf(gb) : 0.f;
-            if (it + 1 < nch) ga = gamma_at(it + 1, ta), gb = gamma_at(it + 1, tb2);
-            const uint32_t stg = sb + kStage0 + (it % kStages) * kStageBytes + kDO;
-            const uint32_t ob = sb + kDO2 + (it & 1) * 4096;
+        for (int it = 0; it < nch && ok; ++it) {
+            const int s = it % kOS, len = chunk_len(it);
+            // the dO tile, and the chunk's gates in the chain ring (staged before the chain
+            // reaches the chunk; the stage cannot be refilled before this chunk's X^T is read)
+            bool good = wait_bar(&sm->ofull[s], (it / kOS) & 1, abort_flag) &&
+                        wait_bar(&sm->cfull[it % kCS], (it / kCS) & 1, abort_flag);
+            if (good && at == 0 && it >= 2) good = wait_ge(&ctr[kTRead], it - 1, abort_flag);
+            ok = role_sync_and<128>(2, good);
+            if (!ok) break;
+            const uint32_t src = sb + kO0 + s * kOStageBytes + kDO, dst = sb + kDO2 + (it & 1) * 4096;
+            const uint32_t gm = sb + kGam + (it % kCS) * kChunk * 4;
 #pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-                const int t = e2 ? tb2 : ta;
-                const float f = e2 ? fb : fa;
-                // dO tile: 64-byte rows, 16-byte chunks XOR ((row / 2) % 4)
-                const uint4 raw = ld_shared_v4(stg + t * 64 + ((cc ^ ((t >> 1) & 3)) << 4));
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t o[4];
+            for (int i = 0; i < 2; ++i) {
+                const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
+                const float f = t < len ? scl * __expf(ld_shared_f32(gm + t * 4)) : 0.f;
+                const uint4 raw = ld_shared_v4(src + p * 16);
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t o4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 x = unpack_bf16(w[e]);
-                    o[e] = pack_bf16(f * x.x, f * x.y);
+                    const float2 v2 = unpack_bf16(w4[e]);
+                    o4[e] = pack_bf16(f * v2.x, f * v2.y);
                 }
-                st_shared_v4(ob + cc * 1024 + (t >> 3) * 128 + (t & 7) * 16, o[0], o[1], o[2], o[3]);
+                st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
             }
             fence_proxy_async();
-            aux_sync(true);
-            if (atid == 0) publish(&ctr[kPReady], it + 1);
-            return true;
-        };
-        if (nch > 0) ok = make_do(0);
-        for (int it = 0; it < nch && ok; ++it) {
-            const int ci = chunk_of(it);
-            if (it + 1 < nch) {
-                ok = make_do(it + 1);  // one iteration ahead of the chain
-                if (!ok) break;
-            }
-            // dh' of this iteration: kHb -> dh_chunks, one contiguous block per (chunk, head,
-            // column slice) in the tile layout
-            ok = aux_sync(atid != 0 || wait_ge(&ctr[kHbFull], it + 1, abort_flag));
-            if (!ok) break;
-            {
-                __nv_bfloat16 *hc = prm.dh_chunks + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + zs) * (K * kBV);
+            named_sync<128>(2);  // all of dO' is written
+            if (at == 0) {
+                // X^T = dO'^T Q: A = dO' read transposed (MN-major), its one 32-column atom repeated
+                // over the M = 128 rows (zero stride between atoms); B = the q tile (MN-major, two
+                // 64-column halves)
+                tc_fence_after();
+                const uint32_t tb = tmem + (it & 1) * kYXBuf, stq = sb + kO0 + s * kOStageBytes;
+                const uint32_t id_X = idesc_bf16(128, 128, true, true);
 #pragma unroll
-                for (int i = 0; i < 4 && outputs; ++i) {
-                    const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 128 + k
-                    *reinterpret_cast<uint4 *>(hc + 8 * e) = ld_shared_v4(sb + kHb + e * 16);
-                }
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tb + kColX, smem_desc(dst + ks * 1024, 0, 512, kSw64),
+                             smem_desc(stq + kQ + ks * 2048, 8192, 1024, kSw128), id_X, ks > 0);
+                mma_commit(&sm->mmaB[it & 1]);
+                ++sm->x_issued[it & 1];
             }
-            aux_sync(true);
-            if (atid == 0) publish(&ctr[kHbRead], it + 1);
-            // dDelta of this iteration: kDb holds -dDelta -> ddelta, one contiguous block per
-            // (chunk, head, column slice) in the tile layout (rows past a ragged chunk's end
-            // are zero), sign restored
-            ok = aux_sync(atid != 0 || wait_ge(&ctr[kDbFull], it + 1, abort_flag));
-            if (!ok) break;
-            {
-                __nv_bfloat16 *dc = prm.ddelta + (((size_t)(sr.chunk0 + ci) * d.Hv + h) * (V / kBV) + zs) * (kChunk * kBV);
-#pragma unroll
-                for (int i = 0; i < 2 && outputs; ++i) {
-                    const int e = atid + kAux * i;  // 16-byte piece e = (n/8) * 64 + t
-                    uint4 v4 = ld_shared_v4(sb + kDb + e * 16);
-                    v4.x ^= 0x80008000u, v4.y ^= 0x80008000u, v4.z ^= 0x80008000u, v4.w ^= 0x80008000u;
-                    *reinterpret_cast<uint4 *>(dc + 8 * e) = v4;
-                }
-            }
-            aux_sync(true);
-            if (atid == 0) publish(&ctr[kDbRead], it + 1);
         }
         if (!ok) {
-            if (atid == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
+            if (at == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
             *abort_flag = 1;
         }
-    } else {
+    } else if (warp == kIssuerWarp) {
         // ========================================================== issuer
         if (lane == 0) {
             bool ok = true;
-            auto issue_loads = [&](int it) {
-                const int s = it % kStages;
-                uint8_t *stg = smem + kStage0 + s * kStageBytes;
-                const int ci = chunk_of(it);
-                const int t0 = sr.start + ci * kChunk;
-                const int cg = sr.chunk0 + ci;
-                mbar_arrive_expect_tx(&sm->full[s], kTxBytes);
-                atomicAdd(&sm->loads_issued, 1);
-                tma_load_3d(stg + kQ, &tm_q, &sm->full[s], 0, hq, t0);
-                tma_load_3d(stg + kQ + 8192, &tm_q, &sm->full[s], 64, hq, t0);
-                tma_load_3d(stg + kK, &tm_k, &sm->full[s], 0, hq, t0);
-                tma_load_3d(stg + kK + 8192, &tm_k, &sm->full[s], 64, hq, t0);
-                tma_load_3d(stg + kW, &tm_w, &sm->full[s], 0, h, t0);
-                tma_load_3d(stg + kW + 8192, &tm_w, &sm->full[s], 64, h, t0);
-                tma_load_2d(stg + kP, &tm_p, &sm->full[s], 0, (cg * d.Hv + h) * kChunk);
-                tma_load_3d(stg + kDO, &tm_do, &sm->full[s], c0, h, t0);
+            auto issue_out_loads = [&](int it) {
+                const int s = it % kOS, ci = chunk_of(it);
+                uint8_t *stg = smem + kO0 + s * kOStageBytes;
+                const int t0 = sr.start + ci * kChunk, cg = sr.chunk0 + ci;
+                mbar_arrive_expect_tx(&sm->ofull[s], kOStageBytes);
+                ++sm->o_issued[s];
+                tma_load_3d(stg + kQ, &tm_q, &sm->ofull[s], 0, hq, t0);
+                tma_load_3d(stg + kQ + 8192, &tm_q, &sm->ofull[s], 64, hq, t0);
+                tma_load_2d(stg + kP, &tm_p, &sm->ofull[s], 0, (cg * d.Hv + h) * kChunk);
+                tma_load_3d(stg + kDO, &tm_do, &sm->ofull[s], c0, h, t0);  // out of range (zero) for operator columns
             };
-            for (int c = 0; c < kStages && c < nch; ++c) issue_loads(c);
-            const uint32_t id_Y = idesc_bf16(64, 32, true, true);
-            const uint32_t id_X = idesc_bf16(128, 32, true, true);
+            for (int c = 0; c < kOS && c < nch; ++c) issue_out_loads(c);
+            const uint32_t id_Y = idesc_bf16(128, 64, true, true);
             for (int it = 0; it < nch && ok; ++it) {
-                // Y, X of iteration it into buffer it % 2 once dO' is written and the chain
-                // has read that buffer's previous contents (iteration it - 2). They depend on
-                // loaded tiles only, so they are issued before the refill below, which waits
-                // for the chain to finish iteration it - 1.
-                ok = wait_ge(&ctr[kPReady], it + 1, abort_flag) && wait_ge(&ctr[kStage], it >= 1 ? it - 1 : 0, abort_flag);
+                // the tiles of iteration it landed, and the chain has read the TMEM buffer's
+                // previous contents (iteration it - 2)
+                const int s = it % kOS;
+                ok = wait_bar(&sm->ofull[s], (it / kOS) & 1, abort_flag) &&
+                     (it < 2 || wait_ge(&ctr[kTRead], it - 1, abort_flag));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t st = sb + kStage0 + (it % kStages) * kStageBytes;
-                const uint32_t tb = tmem + (it & 1) * kYBuf, ob = sb + kDO2 + (it & 1) * 4096;
-                for (int ks = 0; ks < 4; ++ks) {
-                    // Y = P^T dO: A = P read transposed (MN-major), B = the dO tile; 16 rows of P per step
-                    mma_bf16(tb + kColY, smem_desc(st + kP + ks * 2048, 8192, 1024, kSw128),
-                             smem_desc(st + kDO + ks * 1024, 4096, 512, kSw64), id_Y, ks > 0);
-                    // X = Q^T dO': A = the q tile read transposed (MN-major, two 64-row halves)
-                    mma_bf16(tb + kColX, smem_desc(st + kQ + ks * 2048, 8192, 1024, kSw128),
-                             smem_desc(ob + ks * 256, 128, 1024, kSwNone), id_X, ks > 0);
-                }
+                const uint32_t stq = sb + kO0 + s * kOStageBytes;
+                const uint32_t tb = tmem + (it & 1) * kYXBuf;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    // Y^T = dO^T P: A = the dO tile read transposed (MN-major), its one 32-column atom
+                    // repeated over the M = 128 rows (zero stride between atoms); B = P (MN-major)
+                    mma_bf16(tb + kColY, smem_desc(stq + kDO + ks * 1024, 0, 512, kSw64),
+                             smem_desc(stq + kP + ks * 2048, 8192, 1024, kSw128), id_Y, ks > 0);
                 mma_commit(&sm->mmaB[it & 1]);
-                sm->mma_issued = it + 1;
-                // refill the stage of iteration it - 1 with iteration it + 2 once the chain is
-                // done with it (which also means its Y, X and dO' are consumed)
-                if (it >= 1 && it + 2 < nch) {
-                    ok = wait_ge(&ctr[kStage], it, abort_flag);
+                ++sm->y_issued[it & 1];
+                // iteration it - 1's products are complete once the chain has read them: its
+                // (q, P, dO) stage takes iteration it - 1 + kOS
+                if (it >= 1 && it - 1 + kOS < nch) {
+                    ok = wait_ge(&ctr[kTRead], it, abort_flag);
                     if (!ok) break;
-                    issue_loads(it + 2);
+                    issue_out_loads(it - 1 + kOS);
                 }
             }
             if (!ok) {
@@ -492,22 +574,87 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         __syncwarp();
+    } else {
+        // ========================================================= producer
+        bool ok = true;
+        // the stage's gates come in by cp.async from every lane, tracked by the stage's mbarrier
+        // (each lane's arrival raises its pending count until the copies land), then k, w by TMA
+        auto stage_chunk = [&](int it) {
+            const int s = it % kCS, ci = chunk_of(it);
+            const int t0 = sr.start + ci * kChunk, len = chunk_len(it);
+            const uint32_t gdst = smem_u32(gam + s * kChunk);
+            cp_async4(gdst + 4 * lane, prm.gamma + (size_t)(t0 + min(lane, len - 1)) * d.Hv + h);
+            cp_async4(gdst + 4 * (lane + 32), prm.gamma + (size_t)(t0 + min(lane + 32, len - 1)) * d.Hv + h);
+            cp_async_mbar_arrive(&sm->cfull[s]);
+            __syncwarp();
+            if (lane == 0) {
+                uint8_t *stg = smem + kC0 + s * kCStageBytes;
+                mbar_arrive_expect_tx(&sm->cfull[s], kCStageBytes);
+                ++sm->c_issued[s];
+                tma_load_3d(stg + kK, &tm_k, &sm->cfull[s], 0, hq, t0);
+                tma_load_3d(stg + kK + 8192, &tm_k, &sm->cfull[s], 64, hq, t0);
+                tma_load_3d(stg + kW, &tm_w, &sm->cfull[s], 0, h, t0);
+                tma_load_3d(stg + kW + 8192, &tm_w, &sm->cfull[s], 64, h, t0);
+            }
+            __syncwarp();
+        };
+        for (int c = 0; c < kCS && c < nch; ++c) stage_chunk(c);
+        for (int it = 0; it < nch && ok; ++it) {
+            // iteration it done by the chain: its stage takes iteration it + kCS
+            if (it + kCS < nch) {
+                ok = wait_bar(&sm->cempty[it % kCS], (it / kCS) & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                stage_chunk(it + kCS);
+            }
+            if (outputs) {
+                // dh' and dDelta of iteration it out of buffer it % kHB, one bulk copy each
+                ok = wait_bar(&sm->hready[it % kHB], (it / kHB) & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                if (lane == 0) {
+                    const size_t blk = ((size_t)(sr.chunk0 + chunk_of(it)) * d.Hv + h) * (V / kBV) + zs;
+                    bulk_store(prm.dh_chunks + blk * (K * kBV), sb + kHb + (it % kHB) * 8192, K * kBV * 2);
+                    bulk_store(prm.ddelta + blk * (kChunk * kBV), sb + kDb + (it % kHB) * 4096, kChunk * kBV * 2);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                    publish(&ctr[kStored], it + 1);
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok) {
+            if (lane == 0) set_status(prm.status, GDN_ERR_TIMEOUT);
+            *abort_flag = 1;
+        }
+        if (lane == 0) bulk_wait_all();  // the copies complete before the CTA's shared memory goes away
+        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) {
-        // let every TMA load and every MMA still in flight finish (bounded) before the CTA exits
+        // let every TMA load and MMA still in flight finish (bounded) before the CTA exits:
+        // each barrier has at most one use outstanding, the last one issued
         const uint64_t t0 = globaltimer();
-        for (int c = sm->loads_landed; c < sm->loads_issued; ++c)
-            while (!mbar_try_wait(smem_u32(&sm->full[c % kStages]), (c / kStages) & 1) && globaltimer() - t0 < kWaitNs) {
-            }
-        for (int c = sm->mma_seen; c < sm->mma_issued; ++c)
-            while (!mbar_try_wait(smem_u32(&sm->mmaB[c & 1]), (c >> 1) & 1) && globaltimer() - t0 < kWaitNs) {
-            }
+        for (int s = 0; s < kCS; ++s)
+            if (sm->c_issued[s] > 0)
+                while (!mbar_try_wait(smem_u32(&sm->cfull[s]), (sm->c_issued[s] - 1) & 1) && globaltimer() - t0 < kWaitNs) {
+                }
+        for (int s = 0; s < kOS; ++s)
+            if (sm->o_issued[s] > 0)
+                while (!mbar_try_wait(smem_u32(&sm->ofull[s]), (sm->o_issued[s] - 1) & 1) && globaltimer() - t0 < kWaitNs) {
+                }
+        // (a use whose other product was never issued cannot complete: that wait runs out)
+        for (int b = 0; b < 2; ++b) {
+            const int uses = max(sm->y_issued[b], sm->x_issued[b]);
+            if (uses > 0)
+                while (!mbar_try_wait(smem_u32(&sm->mmaB[b]), (uses - 1) & 1) && globaltimer() - t0 < kWaitNs) {
+                }
+        }
     }
     __syncthreads();
-    if (warp == 12) {
+    if (warp == kIssuerWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
