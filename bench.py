@@ -187,18 +187,21 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639742464 + 119971328,
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639710720 + 120067328,
                sources=["gdn_bwd_grad.cu"],
-               sha256="d950affb8ccbca052df0113665b5b83ac2259302e965a6acd032a926380a5a35"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238072832 + 170267136,
+               sha256="50a79e1cf29898d9891349dc94c6602f6fdb6b403fa7de5c1a58689dd3465ddf"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238078720 + 164192256,
                sources=["gdn_bwd_dh.cu"],
-               sha256="ca66ab3574fc215bf4fee7b29431bcb20e89949c8d939b5fe71680a0560c0f0a"),
+               sha256="49a44bd71923db2813205fde11a8db8720cf133647f6a7f82644337eaeaa2cc7"),
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303121920 + 231187200,
+               sources=["gdn_fwd3.cu"],
+               sha256="dae6e9a4b5a6e01e6cb1cc6b0ee126b08760043a9f73b86787dc9771795b3338"),
+    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=195796224 + 212856832,
+               sources=["gdn_prep3.cu"],
+               sha256="1a9ce455d596c3d0e7f10611c4b383757217f101d700851e5e494ce65d3d536d"),
     "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549451520 + 481462272,
                sources=["gdn_recurrent.cu"],
                sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),
-    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=138346240 + 213746944,
-               sources=["gdn_prep3.cu"],
-               sha256="d5112d7d5b5bdabaae238225b67aafbcc81991cccfd568afff397ea44998cf48"),
 }
 TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
 
