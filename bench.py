@@ -199,9 +199,9 @@ NCU_TRAFFIC = {
     "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=195796224 + 212856832,
                sources=["gdn_prep3.cu"],
                sha256="1a9ce455d596c3d0e7f10611c4b383757217f101d700851e5e494ce65d3d536d"),
-    "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549451520 + 481462272,
+    "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549401344 + 481335296,
                sources=["gdn_recurrent.cu"],
-               sha256="29bc622e935a5ddfeae4d09b5c2bc95324502d88ed746e7c8dcf4484b974ee8c"),
+               sha256="d290fb9e4423ff7dede5ab4150409b3dbaaafab395af2d7f0dbf87a41e3151fa"),
 }
 TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
 

@@ -111,7 +111,11 @@ size_t gdn_bwd_workspace_size(const gdn_problem *p);
 size_t gdn_saved_size(const gdn_problem *p);
 
 /* Forward. h0 may be NULL (zero initial state); final_state may be NULL (not
- * written); saved may be NULL (not written). o must not be NULL. */
+ * written); saved may be NULL (not written). o must not be NULL.
+ * Packed sequences stay independent even for non-finite values: the rows past
+ * the end of a sequence's last (ragged) chunk are zeroed or selected out
+ * before any product, so a NaN or Inf in one packed sequence cannot reach the
+ * outputs or final state of another. */
 int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void *v,
                   const float *g, const float *beta, const float *h0, void *o,
                   float *final_state, void *saved, void *workspace, size_t workspace_bytes,
@@ -120,7 +124,11 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
 /* Backward. h0 and dht may be NULL (zero); saved may be NULL (gamma and Ainv
  * are then recomputed) or the buffer a gdn_chunk_fwd call with the same
  * problem and inputs filled; dh0 may be NULL (not written). The other
- * outputs must not be NULL. */
+ * outputs must not be NULL.
+ * Unlike the forward, the backward assumes finite inputs in every packed
+ * sequence: the per-chunk gradients multiply the rows past the end of a ragged
+ * chunk (the next packed sequence's tokens) by exact zeros, so a NaN or Inf in
+ * sequence n + 1 can make the gradients of sequence n's last chunk NaN. */
 int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void *v,
                   const float *g, const float *beta, const float *h0, const void *saved,
                   const void *d_o, const float *dht, void *dq, void *dk, void *dv, float *dg,

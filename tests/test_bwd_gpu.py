@@ -106,7 +106,8 @@ def test_autograd_function(oracle_mod):
     check(oracle_mod, x, g, "bwd_autograd", tol=1e-4)
 
 
-@pytest.mark.parametrize("name", ["bwd_b2_t4096_h16", "qwen_prefill_t8192_hv32", "long_split_t65536_h8"])
+@pytest.mark.parametrize("name", ["bwd_b2_t4096_h16", "qwen_prefill_t8192_hv32", "long_split_t65536_h8",
+                                  "varlen_16seq_32k_h32"])
 def test_full_size_workloads(oracle_mod, name):
     w = scaled(WORKLOADS[name], grads=True)
     x = make_inputs(w)
