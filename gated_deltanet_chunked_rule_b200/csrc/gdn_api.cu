@@ -600,7 +600,7 @@ int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void
             }
             {
                 TimedLaunch t("bwd_split_compose", st);
-                if (launch_split_compose_bwd(P.d, P.nseg, dht, sp.seg_r, sp.seg_Q, seg + per * (P.d.V + P.d.K), st) !=
+                if (launch_split_compose_bwd(P.d, P.nseg, dht, sp.seg_r, sp.seg_Q, seg + per * (P.d.V + P.d.K), b.status, st) !=
                     cudaSuccess)
                     return GDN_ERR_CUDA;
             }

@@ -190,7 +190,7 @@ cudaError_t launch_bwd_dh_tc(const BwdArgs &a, const void *w16, const void *p16,
                              const BwdSplit &sp = BwdSplit());
 // Composition of the backward split: seg_dh[nseg-1] = dht, seg_dh[s-1] = Q_s seg_dh[s] + r_s.
 cudaError_t launch_split_compose_bwd(const Dims &d, int nseg, const float *dht, const float *seg_r,
-                                     const float *seg_Q, float *seg_dh, cudaStream_t stream);
+                                     const float *seg_Q, float *seg_dh, unsigned *status, cudaStream_t stream);
 cudaError_t launch_bwd_grad_tc(const BwdArgs &a, const void *h_chunks16, const void *dh_chunks16,
                                const void *delta16, const void *ddelta16);
 
