@@ -60,9 +60,10 @@
 // there. A composition walks the segments backwards from dht (gdn_split.cu), and
 // the output pass reruns every segment from its composed dh_end.
 //
-// Rows past the end of a ragged chunk: dDelta is zero there (a select), and the
-// w rows they meet in the update are zeroed in shared memory first, so that
-// whatever follows the sequence in memory cannot turn 0 * x into NaN in dh.
+// Rows past the end of a ragged chunk hold the next packed sequence: dDelta is
+// zero there (a select), dO' too, and the w, q and dO rows they would meet in a
+// product are zeroed in shared memory first, so that a non-finite value of the
+// next sequence cannot turn 0 * x into NaN in this one.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -108,8 +109,9 @@ constexpr uint32_t kColY = 0, kColX = 64, kYXBuf = 192, kTmemCols = 512;
 
 // Counters: kTRead iterations whose Y^T, X^T the chain has read out of tensor
 // memory; kStored iterations whose dh' / dDelta copies have finished reading
-// shared memory.
-enum Ctr { kTRead, kStored, kNumCtr };
+// shared memory; kMasked iterations whose (q, dO) stage the dO' warps have
+// finished with (for a ragged chunk: its rows past the end zeroed).
+enum Ctr { kTRead, kStored, kMasked, kNumCtr };
 
 struct Small {
     uint64_t cfull[kCS], cempty[kCS], ofull[kOS], hready[kHB], mmaB[2];
@@ -493,19 +495,32 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
-                const float f = t < len ? scl * __expf(ld_shared_f32(gm + t * 4)) : 0.f;
-                const uint4 raw = ld_shared_v4(src + p * 16);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t o4[4];
+                uint32_t o4[4] = {0u, 0u, 0u, 0u};
+                if (t < len) {
+                    const float f = scl * __expf(ld_shared_f32(gm + t * 4));
+                    const uint4 raw = ld_shared_v4(src + p * 16);
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 v2 = unpack_bf16(w4[e]);
-                    o4[e] = pack_bf16(f * v2.x, f * v2.y);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v2 = unpack_bf16(w4[e]);
+                        o4[e] = pack_bf16(f * v2.x, f * v2.y);
+                    }
+                } else {
+                    st_shared_v4(src + p * 16, 0u, 0u, 0u, 0u);  // the dO row of Y^T
                 }
                 st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
             }
+            if (len < kChunk) {
+                // the q rows of X^T past the end (16-byte chunks of the two 64-column halves)
+                const uint32_t qt = sb + kO0 + s * kOStageBytes + kQ;
+                for (int i = at; i < (kChunk - len) * 16; i += 128) {
+                    const int r = len + (i >> 4), c = i & 15;
+                    st_shared_v4(qt + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
+                }
+            }
             fence_proxy_async();
-            named_sync<128>(2);  // all of dO' is written
+            named_sync<128>(2);  // all of dO' is written (and a ragged chunk's rows zeroed)
+            if (at == 0) publish(&ctr[kMasked], it + 1);
             if (at == 0) {
                 // X^T = dO'^T Q: A = dO' read transposed (MN-major), its one 32-column atom repeated
                 // over the M = 128 rows (zero stride between atoms); B = the q tile (MN-major, two
@@ -547,7 +562,8 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // previous contents (iteration it - 2)
                 const int s = it % kOS;
                 ok = wait_bar(&sm->ofull[s], (it / kOS) & 1, abort_flag) &&
-                     (it < 2 || wait_ge(&ctr[kTRead], it - 1, abort_flag));
+                     (it < 2 || wait_ge(&ctr[kTRead], it - 1, abort_flag)) &&
+                     (chunk_len(it) == kChunk || wait_ge(&ctr[kMasked], it + 1, abort_flag));  // dO rows zeroed
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t stq = sb + kO0 + s * kOStageBytes;

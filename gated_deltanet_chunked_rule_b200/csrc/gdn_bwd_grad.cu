@@ -44,10 +44,11 @@
 // TMA stores from shared memory: dv in place of v, dq in place of q, dk in
 // the T1 | dG tiles; a ragged chunk is written row by row.
 //
-// Rows past the end of the chunk are read as whatever follows in memory (the
-// next sequence, or zeros past the tensor): every term they enter is
-// multiplied by an exactly-zero decay mask, Ainv or beta entry, or lands in a
-// row that is not written.
+// Rows past the end of a ragged chunk hold the next packed sequence (or zeros
+// past the tensor): the q, k, v and dO tiles are zeroed there before any
+// product reads them, and the gates are clamped (gamma) or zero (beta), so a
+// non-finite value of the next sequence cannot reach this one; the chain
+// kernels store Delta and dDelta as zero there.
 #include <cstddef>
 
 #include "gdn_internal.cuh"
@@ -113,6 +114,16 @@ static_assert(sizeof(Vecs) <= 4096, "vector area");
 // (half_bytes = rows * 128).
 __device__ __forceinline__ uint32_t sw_off(int r, int c, int half_bytes) {
     return (c >> 6) * half_bytes + (r >> 3) * 1024 + (r & 7) * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
+}
+
+// Zeroes rows [len, 64) of a [64][128] bf16 tile of two 64-column halves of 128-byte
+// rows (the swizzle permutes 16-byte chunks within a row, so whole rows are zeroed
+// regardless of it).
+__device__ __forceinline__ void zero_rows(uint32_t tile, int len, int tid) {
+    for (int i = tid; i < (C - len) * 16; i += kThreads) {
+        const int r = len + (i >> 4), c = i & 15;
+        st_shared_v4(tile + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
+    }
 }
 
 // This warp's kJJ 8-column tiles of a C x C accumulator (16 rows): v[4 jj + q].
@@ -321,6 +332,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         }
         ok = ok && (!first || (wait_bar(kBarQ) && wait_bar(kBarK))) && wait_bar(kBarD0 + db) &&
              wait_bar(kBarDO) && wait_bar(kBarA);
+        if (len < C) {
+            // a ragged chunk: the rows past its end hold the next packed sequence; zero them in
+            // the q, k (the item's first step) and dO tiles before any product reads them
+            if (first) {
+                zero_rows(sb + kQ, len, tid);
+                zero_rows(sb + kKt, len, tid);
+            }
+            zero_rows(sb + kdO, len, tid);
+            fence_proxy_async();
+            __syncthreads();
+        }
 
         // ---- product batch 1: S, G, P1 (64 x 64) and dU (64 x 128)
         if (ok && tid == 0) {
@@ -361,6 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         tc_fence_after();
         if (ok && tid == 0 && nxt.valid) load_a(nxt);  // Ainv and dDelta are consumed
         ok = ok && wait_bar(kBarV);
+        if (len < C) {
+            zero_rows(sb + kVt, len, tid);  // as for q, k and dO
+            __syncthreads();
+        }
 
         float sacc[kJJ][4], gacc[kJJ][4];  // S -> strictly lower E, G: kept for product batch 2
         if (ok) {

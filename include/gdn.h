@@ -125,10 +125,10 @@ int gdn_chunk_fwd(const gdn_problem *p, const void *q, const void *k, const void
  * are then recomputed) or the buffer a gdn_chunk_fwd call with the same
  * problem and inputs filled; dh0 may be NULL (not written). The other
  * outputs must not be NULL.
- * Unlike the forward, the backward assumes finite inputs in every packed
- * sequence: the per-chunk gradients multiply the rows past the end of a ragged
- * chunk (the next packed sequence's tokens) by exact zeros, so a NaN or Inf in
- * sequence n + 1 can make the gradients of sequence n's last chunk NaN. */
+ * As in the forward, packed sequences stay independent for non-finite values:
+ * the rows past the end of a sequence's last chunk are zeroed or selected out
+ * before any product, so a NaN or Inf in one packed sequence cannot reach the
+ * gradients of another. */
 int gdn_chunk_bwd(const gdn_problem *p, const void *q, const void *k, const void *v,
                   const float *g, const float *beta, const float *h0, const void *saved,
                   const void *d_o, const float *dht, void *dq, void *dk, void *dv, float *dg,

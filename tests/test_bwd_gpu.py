@@ -254,3 +254,35 @@ def test_slow_decay_backward_full_size(oracle_mod, name):
     x = make_inputs(w)
     x["g"] = x["g"] * 0.01
     check(oracle_mod, x, gpu_bwd(x), name + "_slow")
+
+
+@pytest.mark.parametrize("use_saved", [True, False])
+def test_nonfinite_values_stay_in_their_sequence(use_saved):
+    # packed batch whose first sequence ends inside a chunk (100 = 64 + 36): the rest of
+    # that chunk's tiles hold the next sequence, here full of Inf and NaN in every per-token
+    # input the backward reads (q, k, v, dO, g, beta). The backward zeroes those rows
+    # before any product, so the first sequence's gradients are bit-equal to a run whose
+    # second sequence is finite (with the forward's saved states, and recomputing them).
+    w = Workload("iso_bwd", B=1, T=300, Hq=2, Hv=4, K=128, V=128, grads=True, seed=43)
+    x = make_inputs(w)
+    x["cu_seqlens"] = torch.tensor([0, 100, 300], dtype=torch.int32)
+    gen = torch.Generator().manual_seed(5)
+    x["h0"] = 0.02 * torch.randn((2, 4, 128, 128), generator=gen)
+    x["dht"] = 0.01 * torch.randn((2, 4, 128, 128), generator=gen)
+    ref = gpu_bwd(x, use_saved)
+    xb = dict(x)
+    for key in ("q", "k", "v", "do"):
+        t = x[key].clone()
+        t[:, 100:120] = float("inf")
+        t[:, 130:140] = float("nan")
+        xb[key] = t
+    for key in ("g", "beta"):
+        t = x[key].clone()
+        t[:, 100:140] = float("nan")
+        xb[key] = t
+    g = gpu_bwd(xb, use_saved)
+    for n in ("dq", "dk", "dv", "dbeta", "dg"):
+        assert torch.isfinite(g[n][:, :100]).all(), n
+        torch.testing.assert_close(g[n][:, :100], ref[n][:, :100], rtol=0, atol=0)
+    assert torch.isfinite(g["dh0"][0]).all()
+    torch.testing.assert_close(g["dh0"][0], ref["dh0"][0], rtol=0, atol=0)
