@@ -157,6 +157,33 @@ __device__ __forceinline__ void tmem_wait_ld6(uint32_t (&a)[8], uint32_t (&b)[8]
                  : "memory");
 }
 
+// dO' of a ragged chunk (kept out of line, off the full chunks' path): rows past
+// the end get dO' = 0, and the dO rows there (read by Y^T) and the q rows (read
+// by X^T) are zeroed in the stage; 128 threads, thread at.
+__device__ __noinline__ void make_dop_ragged(uint32_t src, uint32_t dst, uint32_t qt, uint32_t gm, float scl, int len,
+                                             int at) {
+    for (int i = 0; i < 2; ++i) {
+        const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
+        uint32_t o4[4] = {0u, 0u, 0u, 0u};
+        if (t < len) {
+            const float f = scl * __expf(ld_shared_f32(gm + t * 4));
+            const uint4 raw = ld_shared_v4(src + p * 16);
+            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+            for (int e = 0; e < 4; ++e) {
+                const float2 v2 = unpack_bf16(w4[e]);
+                o4[e] = pack_bf16(f * v2.x, f * v2.y);
+            }
+        } else {
+            st_shared_v4(src + p * 16, 0u, 0u, 0u, 0u);
+        }
+        st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
+    }
+    for (int i = at; i < (kChunk - len) * 16; i += 128) {
+        const int r = len + (i >> 4), c = i & 15;
+        st_shared_v4(qt + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
+    }
+}
+
 // Byte offset of (row, col) in a [rows][128] bf16 tile stored as two 64-column
 // halves of 128-byte rows with 128-byte swizzle (what the TMA loads produce).
 __device__ __forceinline__ uint32_t sw_off(int row, int col) {
@@ -492,31 +519,23 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (!ok) break;
             const uint32_t src = sb + kO0 + s * kOStageBytes + kDO, dst = sb + kDO2 + (it & 1) * 4096;
             const uint32_t gm = sb + kGam + (it % kCS) * kChunk * 4;
+            if (len == kChunk) {
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
-                uint32_t o4[4] = {0u, 0u, 0u, 0u};
-                if (t < len) {
+                for (int i = 0; i < 2; ++i) {
+                    const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
                     const float f = scl * __expf(ld_shared_f32(gm + t * 4));
                     const uint4 raw = ld_shared_v4(src + p * 16);
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t o4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 v2 = unpack_bf16(w4[e]);
                         o4[e] = pack_bf16(f * v2.x, f * v2.y);
                     }
-                } else {
-                    st_shared_v4(src + p * 16, 0u, 0u, 0u, 0u);  // the dO row of Y^T
+                    st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
                 }
-                st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
-            }
-            if (len < kChunk) {
-                // the q rows of X^T past the end (16-byte chunks of the two 64-column halves)
-                const uint32_t qt = sb + kO0 + s * kOStageBytes + kQ;
-                for (int i = at; i < (kChunk - len) * 16; i += 128) {
-                    const int r = len + (i >> 4), c = i & 15;
-                    st_shared_v4(qt + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
-                }
+            } else {
+                make_dop_ragged(src, dst, sb + kO0 + s * kOStageBytes + kQ, gm, scl, len, at);
             }
             fence_proxy_async();
             named_sync<128>(2);  // all of dO' is written (and a ragged chunk's rows zeroed)

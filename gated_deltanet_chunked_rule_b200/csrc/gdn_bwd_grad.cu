@@ -118,8 +118,8 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c, int half_bytes) {
 
 // Zeroes rows [len, 64) of a [64][128] bf16 tile of two 64-column halves of 128-byte
 // rows (the swizzle permutes 16-byte chunks within a row, so whole rows are zeroed
-// regardless of it).
-__device__ __forceinline__ void zero_rows(uint32_t tile, int len, int tid) {
+// regardless of it). Out of line: only ragged chunks call it.
+__device__ __noinline__ void zero_rows(uint32_t tile, int len, int tid) {
     for (int i = tid; i < (C - len) * 16; i += kThreads) {
         const int r = len + (i >> 4), c = i & 15;
         st_shared_v4(tile + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
