@@ -187,12 +187,12 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639710720 + 120067328,
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639731456 + 116727808,
                sources=["gdn_bwd_grad.cu"],
-               sha256="50a79e1cf29898d9891349dc94c6602f6fdb6b403fa7de5c1a58689dd3465ddf"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238078720 + 164192256,
+               sha256="4cb1cde49c2c5c8fbfbcffac2e6661b72db7b80c2c48626d3c3867ba1b659f84"),
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238191104 + 163365888,
                sources=["gdn_bwd_dh.cu"],
-               sha256="49a44bd71923db2813205fde11a8db8720cf133647f6a7f82644337eaeaa2cc7"),
+               sha256="51de9b9a1c70c4f33962babee7ae36da0bd9510e5d5efa0799a3ab862cd37a21"),
     "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303121920 + 231187200,
                sources=["gdn_fwd3.cu"],
                sha256="dae6e9a4b5a6e01e6cb1cc6b0ee126b08760043a9f73b86787dc9771795b3338"),
