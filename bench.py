@@ -193,15 +193,15 @@ NCU_TRAFFIC = {
     "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238191104 + 163365888,
                sources=["gdn_bwd_dh.cu"],
                sha256="51de9b9a1c70c4f33962babee7ae36da0bd9510e5d5efa0799a3ab862cd37a21"),
-    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303121920 + 231187200,
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303132928 + 225866240,
                sources=["gdn_fwd3.cu"],
-               sha256="dae6e9a4b5a6e01e6cb1cc6b0ee126b08760043a9f73b86787dc9771795b3338"),
-    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=195796224 + 212856832,
+               sha256="41e430efdbd23578f76229322115d21d728f5c6efacfc56565e3f043c557e53f"),
+    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=197432320 + 212447744,
                sources=["gdn_prep3.cu"],
-               sha256="1a9ce455d596c3d0e7f10611c4b383757217f101d700851e5e494ce65d3d536d"),
-    "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549401344 + 481335296,
+               sha256="51b40e52ce80096eae1cb27c55d6d8067a160e432d69531e6a0e1b583b68eb92"),
+    "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549415168 + 481711104,
                sources=["gdn_recurrent.cu"],
-               sha256="d290fb9e4423ff7dede5ab4150409b3dbaaafab395af2d7f0dbf87a41e3151fa"),
+               sha256="35e113de4eda5533922853cf613728b9b8d8c372c9964fd87946edc0413bf6a2"),
 }
 TRAFFIC_COMMON_SOURCES = ["gdn_internal.cuh", "gdn_warp.cuh", "sm100_ptx.cuh"]
 
