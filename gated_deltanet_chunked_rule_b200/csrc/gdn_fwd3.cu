@@ -27,8 +27,12 @@
 // chunk they exchange, through shared memory and two 128-thread barriers, only
 // bf16 data: the state quarters (the chunk's entry state, which the output
 // products read anyway) and the Delta~ quarters (1 KB per warp). Each warp
-// issues 64 MMAs per chunk. Shared memory is read with ld.shared / ldmatrix on
-// 32-bit shared addresses throughout (generic loads would take the long path).
+// issues 64 MMAs per chunk, into one accumulator set per product: with ten
+// warps, three share a scheduler's register file, which caps a thread at 168
+// registers, and a second set (to split the dependent MMAs) made the compiler
+// spill inside the chain, costing 15 % of the kernel. Shared memory is read
+// with ld.shared / ldmatrix on 32-bit shared addresses throughout (generic
+// loads would take the long path).
 //
 // Warp roles (320 threads):
 //   warps 0-3    chain (above).
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_u,
             const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_o,
-            const Fwd3Params prm) {
+            const __grid_constant__ Fwd3Params prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     Small *sm = reinterpret_cast<Small *>(smem + kSmall);
@@ -263,8 +267,8 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     ao[mt][kk][2] = pack_bf16(hs[mt][2 * kk + 1][0], hs[mt][2 * kk + 1][1]);
                     ao[mt][kk][3] = pack_bf16(hs[mt][2 * kk + 1][2], hs[mt][2 * kk + 1][3]);
                 }
-            // D1 accumulators [m-tile][token n-tile], two independent sets (even / odd k-steps)
-            float acc[2][2][4] = {}, acc2[2][2][4] = {};
+            // D1 accumulators [m-tile][token n-tile]
+            float acc[2][2][4] = {};
             float gC = 0.f, sc[2][2] = {};
             uint32_t bw[8][4];  // w fragments (B of D1): bw[2 o + kk] is k-step 2((x + o) & 3) + kk
             if (good) {
@@ -310,8 +314,8 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int mt = 0; mt < 2; ++mt) {
                     hmma(acc[mt][0], ao[mt][0], bw[0][0], bw[0][1]);
                     hmma(acc[mt][1], ao[mt][0], bw[0][2], bw[0][3]);
-                    hmma(acc2[mt][0], ao[mt][1], bw[1][0], bw[1][1]);
-                    hmma(acc2[mt][1], ao[mt][1], bw[1][2], bw[1][3]);
+                    hmma(acc[mt][0], ao[mt][1], bw[1][0], bw[1][1]);
+                    hmma(acc[mt][1], ao[mt][1], bw[1][2], bw[1][3]);
                 }
             }
             ok = role_sync_and<128>(1, good);  // every quarter of h_j is in hbuf
@@ -330,7 +334,7 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
-                        float(&A)[2][2][4] = kk ? acc2 : acc;
+                        float(&A)[2][2][4] = acc;
                         hmma(A[mt][0], ah[mt][kk], bw[2 * o + kk][0], bw[2 * o + kk][1]);
                         hmma(A[mt][1], ah[mt][kk], bw[2 * o + kk][2], bw[2 * o + kk][3]);
                     }
@@ -345,7 +349,7 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        dl[nt][e] = 16 * x + 8 * nt + 2 * cq + (e & 1) < len ? -(acc[mt][nt][e] + acc2[mt][nt][e]) : 0.f;
+                        dl[nt][e] = 16 * x + 8 * nt + 2 * cq + (e & 1) < len ? -acc[mt][nt][e] : 0.f;
                 uint32_t du[4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
@@ -383,31 +387,22 @@ fwd3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     hmma(hs[mt][2 * np + 1], da[mt], bk[0][np][2], bk[0][np][3]);
                 }
             named_sync<128>(1);  // every token quarter of Delta~ is in kXb
-            {
-                float h2[2][4][4] = {};  // second accumulator set (latency)
+            // (eight independent accumulator tiles per token quarter cover the MMA latency)
 #pragma unroll
-                for (int o = 1; o < 4; ++o) {
-                    uint32_t pa[2][4];
+            for (int o = 1; o < 4; ++o) {
+                uint32_t pa[2][4];
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        const uint4 p = ld_shared_v4(sb + kXb + (mt * 4 + ((x + o) & 3)) * 512 + lane * 16);
-                        pa[mt][0] = p.x, pa[mt][1] = p.y, pa[mt][2] = p.z, pa[mt][3] = p.w;
-                    }
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                        for (int np = 0; np < 2; ++np) {
-                            float(&H)[2][4][4] = (o & 1) ? h2 : hs;
-                            hmma(H[mt][2 * np], pa[mt], bk[o][np][0], bk[o][np][1]);
-                            hmma(H[mt][2 * np + 1], pa[mt], bk[o][np][2], bk[o][np][3]);
-                        }
+                for (int mt = 0; mt < 2; ++mt) {
+                    const uint4 p = ld_shared_v4(sb + kXb + (mt * 4 + ((x + o) & 3)) * 512 + lane * 16);
+                    pa[mt][0] = p.x, pa[mt][1] = p.y, pa[mt][2] = p.z, pa[mt][3] = p.w;
                 }
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-                    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) hs[mt][nt][e] += h2[mt][nt][e];
+                    for (int np = 0; np < 2; ++np) {
+                        hmma(hs[mt][2 * np], pa[mt], bk[o][np][0], bk[o][np][1]);
+                        hmma(hs[mt][2 * np + 1], pa[mt], bk[o][np][2], bk[o][np][3]);
+                    }
             }
             // h_j and Delta_j (shared memory, generic writes) go to the output MMAs and
             // the state copies (async proxy); the stage is free for the producer
