@@ -33,19 +33,20 @@
 // 32 value rows in its own TMEM lane quarter, in the mma.sync accumulator
 // layout of the 16x256b load, and adds them to its fragments directly.
 //
-// Warp roles (320 threads):
+// Warp roles (256 threads):
 //   warps 0-3  chain (above).
-//   warps 4-7  dO' = scale e^gamma o dO into shared memory (one warp per
-//              scheduler), then one of their threads issues the X^T MMAs.
-//   warp 8     issuer: the (q, P, dO) TMA ring and the Y^T MMAs.
-// Y^T and X^T go into double-buffered tensor memory, each chunk's pair
-// completing one mbarrier (an arrival from each issuing thread): a single
-// thread spends tens of cycles per tcgen05.mma, so the two products are
-// issued side by side.
-//   warp 9     producer: the (k, w) TMA ring with each chunk's gates, and the
+//   warps 4-5  dO' = scale e^gamma o dO into shared memory, then one of their
+//              threads issues the X^T MMAs.
+//   warp 6     issuer: the (q, P, dO) TMA ring and the Y^T MMAs.
+//   warp 7     producer: the (k, w) TMA ring with each chunk's gates, and the
 //              bulk copies of dh' and dDelta to global memory. (L2 prefetches
 //              a few chunks ahead, as the forward chain issues them, measured
 //              a few percent slower here.)
+// Y^T and X^T go into double-buffered tensor memory, each chunk's pair
+// completing one mbarrier (an arrival from each issuing thread): a single
+// thread spends tens of cycles per tcgen05.mma, so the two products are
+// issued side by side. Two dO' warps measured faster than one or four (eight
+// warps in all: no scheduler holds more than two, so the register cap is 255).
 // Hand-over by mbarriers (hardware completions, the chain's per-chunk
 // hand-over) and release/acquire counters ("buffer free" conditions); every
 // wait is bounded, and a wait that expires records GDN_ERR_TIMEOUT and winds
@@ -77,10 +78,12 @@ using namespace sm100;
 using namespace warp;
 
 constexpr int kChainWarps = 4;
-constexpr int kAuxWarp0 = 4;  // warps 4..7
-constexpr int kIssuerWarp = 8;
-constexpr int kProdWarp = 9;
-constexpr int kThreads = 10 * 32;
+constexpr int kAuxWarps = 2;  // dO' makers: warps kAuxWarp0 ..
+constexpr int kAuxWarp0 = 4;
+constexpr int kAuxThreads = kAuxWarps * 32;
+constexpr int kIssuerWarp = kAuxWarp0 + kAuxWarps;
+constexpr int kProdWarp = kIssuerWarp + 1;
+constexpr int kThreads = (kProdWarp + 1) * 32;
 static_assert(kThreads == (kProdWarp + 1) * 32, "the producer is the last warp");
 constexpr int kBV = 32;
 constexpr int kCS = 3;        // chain ring stages (k, w)
@@ -159,11 +162,11 @@ __device__ __forceinline__ void tmem_wait_ld6(uint32_t (&a)[8], uint32_t (&b)[8]
 
 // dO' of a ragged chunk (kept out of line, off the full chunks' path): rows past
 // the end get dO' = 0, and the dO rows there (read by Y^T) and the q rows (read
-// by X^T) are zeroed in the stage; 128 threads, thread at.
+// by X^T) are zeroed in the stage; kAuxThreads threads, thread at.
 __device__ __noinline__ void make_dop_ragged(uint32_t src, uint32_t dst, uint32_t qt, uint32_t gm, float scl, int len,
                                              int at) {
-    for (int i = 0; i < 2; ++i) {
-        const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
+    for (int i = 0; i < 256 / kAuxThreads; ++i) {
+        const int p = at + kAuxThreads * i, t = p >> 2;  // 16-byte piece p of row t
         uint32_t o4[4] = {0u, 0u, 0u, 0u};
         if (t < len) {
             const float f = scl * __expf(ld_shared_f32(gm + t * 4));
@@ -178,7 +181,7 @@ __device__ __noinline__ void make_dop_ragged(uint32_t src, uint32_t dst, uint32_
         }
         st_shared_v4(dst + p * 16, o4[0], o4[1], o4[2], o4[3]);
     }
-    for (int i = at; i < (kChunk - len) * 16; i += 128) {
+    for (int i = at; i < (kChunk - len) * 16; i += kAuxThreads) {
         const int r = len + (i >> 4), c = i & 15;
         st_shared_v4(qt + (c >> 3) * 8192 + r * 128 + (c & 7) * 16, 0u, 0u, 0u, 0u);
     }
@@ -499,7 +502,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         }
             }
         }
-    } else if (warp < kAuxWarp0 + 4) {
+    } else if (warp < kAuxWarp0 + kAuxWarps) {
         // ======================================================= dO' makers
         // dO' = scale e^gamma o dO of iteration it, in the layout of the dO tile (a row of 32
         // values is 64 contiguous bytes whatever the swizzle), once the tile has landed and
@@ -515,14 +518,14 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             bool good = wait_bar(&sm->ofull[s], (it / kOS) & 1, abort_flag) &&
                         wait_bar(&sm->cfull[it % kCS], (it / kCS) & 1, abort_flag);
             if (good && at == 0 && it >= 2) good = wait_ge(&ctr[kTRead], it - 1, abort_flag);
-            ok = role_sync_and<128>(2, good);
+            ok = role_sync_and<kAuxThreads>(2, good);
             if (!ok) break;
             const uint32_t src = sb + kO0 + s * kOStageBytes + kDO, dst = sb + kDO2 + (it & 1) * 4096;
             const uint32_t gm = sb + kGam + (it % kCS) * kChunk * 4;
             if (len == kChunk) {
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int p = at + 128 * i, t = p >> 2;  // 16-byte piece p of row t
+                for (int i = 0; i < 256 / kAuxThreads; ++i) {
+                    const int p = at + kAuxThreads * i, t = p >> 2;  // 16-byte piece p of row t
                     const float f = scl * __expf(ld_shared_f32(gm + t * 4));
                     const uint4 raw = ld_shared_v4(src + p * 16);
                     const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -538,7 +541,7 @@ bwd_dh_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 make_dop_ragged(src, dst, sb + kO0 + s * kOStageBytes + kQ, gm, scl, len, at);
             }
             fence_proxy_async();
-            named_sync<128>(2);  // all of dO' is written (and a ragged chunk's rows zeroed)
+            named_sync<kAuxThreads>(2);  // all of dO' is written (and a ragged chunk's rows zeroed)
             if (at == 0) publish(&ctr[kMasked], it + 1);
             if (at == 0) {
                 // X^T = dO'^T Q: A = dO' read transposed (MN-major), its one 32-column atom repeated
