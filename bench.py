@@ -190,12 +190,12 @@ NCU_TRAFFIC = {
     "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639731456 + 116727808,
                sources=["gdn_bwd_grad.cu"],
                sha256="4cb1cde49c2c5c8fbfbcffac2e6661b72db7b80c2c48626d3c3867ba1b659f84"),
-    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238191104 + 163365888,
+    "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238085376 + 163700992,
                sources=["gdn_bwd_dh.cu"],
-               sha256="51de9b9a1c70c4f33962babee7ae36da0bd9510e5d5efa0799a3ab862cd37a21"),
-    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303132928 + 225866240,
+               sha256="5a6cd00f77d5ef975c74a2dd1a54451b37353939ae3b16825381feefd4ebd379"),
+    "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303272960 + 229458944,
                sources=["gdn_fwd3.cu"],
-               sha256="41e430efdbd23578f76229322115d21d728f5c6efacfc56565e3f043c557e53f"),
+               sha256="4ab2d3258a8acfdbe40dd99c74f8e65bf27fc06b7a8ca712f094ffff60d52952"),
     "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=197432320 + 212447744,
                sources=["gdn_prep3.cu"],
                sha256="51b40e52ce80096eae1cb27c55d6d8067a160e432d69531e6a0e1b583b68eb92"),
