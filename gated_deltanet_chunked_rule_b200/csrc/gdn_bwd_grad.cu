@@ -126,6 +126,19 @@ __device__ __noinline__ void zero_rows(uint32_t tile, int len, int tid) {
     }
 }
 
+// Stores 8 fp32 per thread in the 16x256b.x2 layout (what tmem_ld16x256_x2 reads) and
+// waits until the store has completed.
+__device__ __forceinline__ void tmem_st16x256_x2(uint32_t taddr, const float (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n\t"
+        "tcgen05.wait::st.sync.aligned;"
+        :
+        : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+        : "memory");
+}
+
 // This warp's kJJ 8-column tiles of a C x C accumulator (16 rows): v[4 jj + q].
 static_assert(kJJ == 2, "16 columns of a C x C accumulator per warp");
 __device__ __forceinline__ void ld_cc(uint32_t taddr, float (&v)[4 * kJJ]) { tmem_ld16x256_x2(taddr, v); }
@@ -511,15 +524,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
             }
             // dq = scale diag(e^gamma) dO h^T + T1 K (+ the group's earlier heads);
             // dgamma += scale e^gamma q.(dO h^T)
+            // (16 columns at a time: three 16-value blocks live at once would spill at the
+            // 128-register cap of sixteen warps)
 #pragma unroll
-            for (int part = 0; part < kParts; ++part) {
-                const int cb = ck0 + 32 * part;
-                float a[16], b[16], x[16];
-                tmem_ld16x256_x4(tmem + lane_base + kCQ1 + cb, a);
-                tmem_ld16x256_x4(tmem + lane_base + kCTK + cb, b);
-                if (!first) tmem_ld16x256_x4(park + 32 * part, x);
+            for (int part = 0; part < 2 * kParts; ++part) {
+                const int cb = ck0 + 16 * part;
+                float a[8], b[8], x[8];
+                tmem_ld16x256_x2(tmem + lane_base + kCQ1 + cb, a);
+                tmem_ld16x256_x2(tmem + lane_base + kCTK + cb, b);
+                if (!first) tmem_ld16x256_x2(park + 16 * part, x);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 2; ++i) {
                     const int col = cb + 8 * i + 2 * c4;
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
@@ -539,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
                         }
                     }
                 }
-                if (!last) tmem_st16x256_x4(park + 32 * part, x);
+                if (!last) tmem_st16x256_x2(park + 16 * part, x);
             }
         }
         fence_proxy_async();  // dG -> the tensor core; dq -> the TMA store
@@ -600,27 +615,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
         ok = __syncthreads_and(ok);  // h and dh' are consumed
         if (!ok) break;
         if (tid == 0 && nxt.valid) load_st(nxt);
+        float dotb[2] = {0.f, 0.f}, z3[2] = {0.f, 0.f};  // per row, summed over both column halves
 #pragma unroll
-        for (int part = 0; part < kParts; ++part) {
-            const int cb = ck0 + 32 * part;
-            float kb[16], k2[16], x[16];
-            tmem_ld16x256_x4(tmem + lane_base + kCKb + cb, kb);  // dU h^T = -dKb
-            tmem_ld16x256_x4(tmem + lane_base + kCK2 + cb, k2);  // Delta dh'^T
-            tmem_ld16x256_x4(tmem + lane_base + kCDK + cb, x);   // dk so far + T1^T Q + dG K + dG^T K
+        for (int part = 0; part < 2 * kParts; ++part) {  // 16 columns at a time, as above
+            const int cb = ck0 + 16 * part;
+            float kb[8], k2[8], x[8];
+            tmem_ld16x256_x2(tmem + lane_base + kCKb + cb, kb);  // dU h^T = -dKb
+            tmem_ld16x256_x2(tmem + lane_base + kCK2 + cb, k2);  // Delta dh'^T
+            tmem_ld16x256_x2(tmem + lane_base + kCDK + cb, x);   // dk so far + T1^T Q + dG K + dG^T K
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi) {
                 const int r = hi ? r1 : r0;
                 const float fk = br[hi] * er[hi];                     // dk += beta e^gamma dKb
                 const float f2 = lr[hi] ? __expf(gC - gr[hi]) : 0.f;  // dk += e^{gamma_C - gamma} (Delta dh'^T)
-                float dotb = 0.f, z3 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 2; ++i) {
                     const int col = cb + 8 * i + 2 * c4, e = 4 * i + 2 * hi;
                     const float2 kk = ld_pair_sw(sb + kKt, r, col);
                     const float b0 = -kb[e], b1 = -kb[e + 1];
                     const float e0 = k2[e], e1 = k2[e + 1];
-                    dotb += b0 * kk.x + b1 * kk.y;
-                    z3 += e0 * kk.x + e1 * kk.y;
+                    dotb[hi] += b0 * kk.x + b1 * kk.y;
+                    z3[hi] += e0 * kk.x + e1 * kk.y;
                     x[e] += fk * b0 + f2 * e0;
                     x[e + 1] += fk * b1 + f2 * e1;
                     if (last) {
@@ -631,13 +646,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grad_kernel(const __grid_cons
                             *reinterpret_cast<uint32_t *>(prm.dk + ((size_t)(t0 + r) * d.Hq + cur.hq) * K + col) = dkp;
                     }
                 }
-                rdb[hi] += er[hi] * dotb;
-                rdg[hi] += br[hi] * er[hi] * dotb;
-                z3 *= f2;
-                rdg[hi] -= z3;
-                sdg += z3;
             }
-            if (!last) tmem_st16x256_x4(tmem + lane_base + kCDK + cb, x);
+            if (!last) tmem_st16x256_x2(tmem + lane_base + kCDK + cb, x);
+        }
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+            const float f2 = lr[hi] ? __expf(gC - gr[hi]) : 0.f;
+            rdb[hi] += er[hi] * dotb[hi];
+            rdg[hi] += br[hi] * er[hi] * dotb[hi];
+            const float z = z3[hi] * f2;
+            rdg[hi] -= z;
+            sdg += z;
         }
 
         // ---- fixed-order reductions: quad (row sums), column groups, then across warps
