@@ -187,9 +187,9 @@ def kernel_bytes(name, w, saved=False):
 # workload and step they were taken on and only while the kernel's sources are
 # byte-identical to the captured build (sha256 over the listed files).
 NCU_TRAFFIC = {
-    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639731456 + 116727808,
+    "bwd_grad": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=639716096 + 118936320,
                sources=["gdn_bwd_grad.cu"],
-               sha256="4cb1cde49c2c5c8fbfbcffac2e6661b72db7b80c2c48626d3c3867ba1b659f84"),
+               sha256="cbba0dec59861f9a29b8689f21bf3da92f4ad43f5d64565573c5b558ed9005f1"),
     "bwd_dh": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=238085376 + 163700992,
                sources=["gdn_bwd_dh.cu"],
                sha256="5a6cd00f77d5ef975c74a2dd1a54451b37353939ae3b16825381feefd4ebd379"),
