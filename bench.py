@@ -196,9 +196,9 @@ NCU_TRAFFIC = {
     "fwd_hybrid": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=303272960 + 229458944,
                sources=["gdn_fwd3.cu"],
                sha256="4ab2d3258a8acfdbe40dd99c74f8e65bf27fc06b7a8ca712f094ffff60d52952"),
-    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=197432320 + 212447744,
+    "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=186969600 + 213129728,
                sources=["gdn_prep3.cu"],
-               sha256="51b40e52ce80096eae1cb27c55d6d8067a160e432d69531e6a0e1b583b68eb92"),
+               sha256="06dfdcce0e07ca0da55ba6669fb36d63a66499bff5ae4e86585fb2109c8e3712"),
     "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549415168 + 481711104,
                sources=["gdn_recurrent.cu"],
                sha256="35e113de4eda5533922853cf613728b9b8d8c372c9964fd87946edc0413bf6a2"),

@@ -23,13 +23,14 @@
 // sequence); u goes out straight from the accumulator registers, four lanes per
 // 32-byte sector. The four bulk products (S, G, u, w) run on tcgen05 from
 // TMA-loaded, 128-byte-swizzled tiles. The unit lower-triangular inverse is
-// taken block-wise on 16 x 16 blocks in fp32, in one work matrix that holds the
-// inverse on and below the diagonal and A transposed above it: diagonal blocks by
-// forward substitution, off-diagonal blocks one block diagonal at a time on tf32
-// MMAs. Rows past the end of a sequence have beta = 0, and a ragged chunk's rows
-// past its end are zeroed in the q, k and v tiles before any product, so that
-// whatever the TMA reads there (the next sequence, or zeros) never reaches an
-// output.
+// taken block-wise in fp32, in one work matrix that holds the inverse on and below
+// the diagonal and A transposed above it: 16 x 16 diagonal blocks by forward
+// substitution, then two doubling steps on tf32 MMAs (16 -> 32 -> 64), each
+// X_BA = -X_BB A_BA X_AA for the two halves A, B of a block, so that the critical
+// path holds four dependent products and two CTA barriers. Rows past the end of a
+// sequence have beta = 0, and a ragged chunk's rows past its end are zeroed in the
+// q, k and v tiles before any product, so that whatever the TMA reads there (the
+// next sequence, or zeros) never reaches an output.
 #include <algorithm>
 #include <cstddef>
 
@@ -160,12 +161,15 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = (uint32_t)(wm * 32) << 16;  // TMEM lanes of this warp's rows (M = 64 layout)
     uint32_t tma_phase = 0, mma_phase = 0;  // phases consumed so far
-    bool tma_pending = false, mma_pending = false;  // (thread 0) issued and not yet consumed
+    bool tma_pending = false;  // (every thread) a v tile load issued and not yet consumed
+    bool mma_pending = false;  // (thread 0) products issued and not yet consumed
     bool ok = true;
     const int n_items = d.NC * d.Hq;
-    // Persistent: items (chunk, qk head) in steps of the grid; the tiles of this CTA's next
-    // item are prefetched into L2 while it works on the current one.
-    auto prefetch_item = [&](int item) {
+    // Persistent: items (chunk, qk head) in steps of the grid; the tiles of the item after
+    // this CTA's next one are prefetched into L2 while it works on the current one. Copies
+    // and prefetches are issued by warps that idle during the inverse (a copy's setup holds
+    // its thread for hundreds of cycles, and with it the CTA at the next barrier).
+    auto prefetch_item = [&](int item) {  // by one thread
         if (item >= n_items) return;
         const int cg2 = item / d.Hq, hq2 = item % d.Hq;
         const int n2 = chunk_owner(d, cg2);
@@ -184,8 +188,8 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // q, k tiles of the CTA's k-th item go to buffer k % 2 (a consistent sequence table
     // has an owner for every chunk, an inconsistent one for none, so items are either
     // all valid or all skipped and the buffer alternation holds)
-    int qk_issued = 0;  // (thread 0) q, k loads issued
-    auto issue_qk = [&](int item) {
+    int qk_issued = 0;  // (every thread) q, k loads issued
+    auto issue_qk = [&](int item, int issuer) {  // by every thread; thread `issuer` copies
         if (item >= n_items) return;
         const int cg2 = item / d.Hq, hq2 = item % d.Hq;
         const int n2 = chunk_owner(d, cg2);
@@ -193,14 +197,16 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const SeqRange s2 = seq_range(d, n2);
         const int t2 = s2.start + (cg2 - s2.chunk0) * C;
         const int b = qk_issued & 1;
-        mbar_arrive_expect_tx(&qk_bar[b], 4 * 8192);
-        tma_load_3d(smem + kQ0 + b * 16384, &tm_q, &qk_bar[b], 0, hq2, t2);
-        tma_load_3d(smem + kQ0 + b * 16384 + 8192, &tm_q, &qk_bar[b], 64, hq2, t2);
-        tma_load_3d(smem + kK0 + b * 16384, &tm_k, &qk_bar[b], 0, hq2, t2);
-        tma_load_3d(smem + kK0 + b * 16384 + 8192, &tm_k, &qk_bar[b], 64, hq2, t2);
+        if (tid == issuer) {
+            mbar_arrive_expect_tx(&qk_bar[b], 4 * 8192);
+            tma_load_3d(smem + kQ0 + b * 16384, &tm_q, &qk_bar[b], 0, hq2, t2);
+            tma_load_3d(smem + kQ0 + b * 16384 + 8192, &tm_q, &qk_bar[b], 64, hq2, t2);
+            tma_load_3d(smem + kK0 + b * 16384, &tm_k, &qk_bar[b], 0, hq2, t2);
+            tma_load_3d(smem + kK0 + b * 16384 + 8192, &tm_k, &qk_bar[b], 64, hq2, t2);
+        }
         ++qk_issued;
     };
-    if (tid == 0) issue_qk(blockIdx.x);
+    issue_qk(blockIdx.x, 0);
     int it_k = 0;  // this CTA's item count
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++it_k) {
     const int cg = item / d.Hq, hq = item % d.Hq;
@@ -211,7 +217,6 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int t0 = sr.start + ci * C, len = min(C, sr.len - ci * C);
     const int buf = it_k & 1;
     const uint32_t qv = sb + kQ0 + buf * 16384, kt = sb + kK0 + buf * 16384;  // q (then v), k tiles
-    if (tid == 0) prefetch_item(item + 2 * gridDim.x);
 
     // ---- q, k tiles (loaded during the previous item); S = Q K^T and G = K K^T on tcgen05
     float g_next = 0.f, b_next = 0.f;  // g, beta of the next value head, prefetched
@@ -243,9 +248,6 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     ok = ok && cta_wait(mma_bar, mma_phase & 1);
     if (ok) ++mma_phase, mma_pending = false;
-    // the other buffer was last read by the previous item's products, all complete: the next
-    // item's q, k tiles go there now
-    if (ok && tid == 0) issue_qk(item + gridDim.x);
     tc_fence_after();
     // S, G: rows r0, r1, columns 32 wn + 8 j + 2 c4 (+1) -- the warp MMA fragment layout
     float sacc[4][4], gacc[4][4];
@@ -260,13 +262,14 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     tc_fence_before();
     __syncthreads();  // q tile and S, G columns free
-    auto load_v = [&](int h) {
+    // v tiles go into the q slot. The first value head's is issued by the last warp, which
+    // idles during the inverse: issued by thread 0 here, it held the whole CTA at the next
+    // barrier and cost 4 % of the kernel.
+    auto load_v = [&](int h) {  // by one thread
         mbar_arrive_expect_tx(tma_bar, 2 * 8192);
         tma_load_3d(smem + (qv - sb), &tm_v, tma_bar, 0, h, t0);
         tma_load_3d(smem + (qv - sb) + 8192, &tm_v, tma_bar, 64, h, t0);
-        tma_pending = true;
     };
-    if (ok && tid == 0) load_v(hq * G);
 
     for (int gi = 0; gi < G && ok; ++gi) {
         const int h = hq * G + gi;
@@ -323,82 +326,157 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tma_store_2d(&tm_po, sb + kPs, 0, (cg * d.Hv + h) * C);
             bulk_commit();
         }
-        // ---- diagonal 16 x 16 blocks: thread t -> block t / 16, column t % 16
-        if (tid < 64) {
-            const int b = tid >> 4, cc = tid & 15, o = b * 16;
-            float xcol[16];
+        // ---- the inverse X = (I + A)^-1, unit lower triangular, in two steps of doubling:
+        //  (1) warps 0, 1: the diagonal 16 x 16 blocks of their 32 x 32 block by forward
+        //      substitution (lane -> block lane / 16, column lane % 16), then that block's
+        //      off-diagonal 16 x 16 block X_10 = -X_11 (A_10 X_00) on tf32 MMAs;
+        //  (2) warps 0..3, one 8-column strip each: X_BA = -X_BB (A_BA X_AA) on the 32 x 32
+        //      blocks (A = rows and columns 0..31, B = 32..63).
+        //  Warps 4..7 take no part: three of them issue the copies of the next tiles meanwhile.
+        if (gi == 0 && ok) {
+            if (tid == kThreads - 32) load_v(hq * G);
+            tma_pending = true;
+            // the other q, k buffer was last read by the previous item's products, all
+            // complete: the next item's tiles go there now
+            issue_qk(item + gridDim.x, kThreads - 64);
+            if (tid == kThreads - 96) prefetch_item(item + 2 * gridDim.x);
+        }
+        if (warp < 2) {
+            {
+                const int o = 32 * warp + 16 * (lane >> 4), cc = lane & 15;
+                float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == cc) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) x[r] = r == cc ? 1.f : 0.f;
+                // right-looking: once x_j is final, rows r > j take -A_rj x_j; row j of A^T
+                // (A_rj for r > j) lies contiguous at AX[o + j][o + r]
 #pragma unroll
-                for (int j = 0; j < r; ++j) acc = fmaf(-AX[o + j][o + r], xcol[j], acc);
-                xcol[r] = r < cc ? 0.f : acc;
+                for (int j = 0; j < 15; ++j) {
+#pragma unroll
+                    for (int q = (j + 1) >> 2; q < 4; ++q) {
+                        const float4 a = *reinterpret_cast<const float4 *>(&AX[o + j][o + 4 * q]);
+                        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (4 * q + e > j) x[4 * q + e] = fmaf(-av[e], x[j], x[4 * q + e]);
+                    }
+                }
+                // only on and below the diagonal: above it lies A
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    if (r >= cc) AX[o + r][o + cc] = x[r];
             }
-            // only on and below the diagonal: above it lies A
+            __syncwarp();
+            // X_10 = -X_11 (A_10 X_00) for this warp's 32 x 32 block: rows i0 .., columns j0 ..
+            const int j0 = 32 * warp, i0 = j0 + 16;
+            float t[2][4] = {};
 #pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r >= cc) AX[o + r][o + cc] = xcol[r];
+            for (int kk = 0; kk < 2; ++kk) {
+                const int ac = j0 + kk * 8 + c4;
+                // A_{i0 + row, ac} (below the diagonal) is stored transposed
+                const uint32_t a[4] = {tf32(AX[ac][i0 + g8]), tf32(AX[ac][i0 + g8 + 8]), tf32(AX[ac + 4][i0 + g8]),
+                                       tf32(AX[ac + 4][i0 + g8 + 8])};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int bc = j0 + nt * 8 + g8;
+                    // X_00: zero above the diagonal (A lies there)
+                    const float x0 = bc > ac ? 0.f : AX[ac][bc];
+                    const float x1 = bc > ac + 4 ? 0.f : AX[ac + 4][bc];
+                    mma_tf32(t[nt], a, tf32(x0), tf32(x1));
+                }
+            }
+            float(*Tw)[17] = T[warp];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int col = nt * 8 + 2 * c4;
+                Tw[g8][col] = t[nt][0];
+                Tw[g8][col + 1] = t[nt][1];
+                Tw[g8 + 8][col] = t[nt][2];
+                Tw[g8 + 8][col + 1] = t[nt][3];
+            }
+            __syncwarp();
+            float x[2][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                const int ac = i0 + kk * 8 + c4;
+                const int ra = i0 + g8, rb = ra + 8;
+                const uint32_t a[4] = {tf32(ac > ra ? 0.f : AX[ra][ac]), tf32(ac > rb ? 0.f : AX[rb][ac]),
+                                       tf32(ac + 4 > ra ? 0.f : AX[ra][ac + 4]), tf32(ac + 4 > rb ? 0.f : AX[rb][ac + 4])};
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int bc = nt * 8 + g8;
+                    mma_tf32(x[nt], a, tf32(Tw[kk * 8 + c4][bc]), tf32(Tw[kk * 8 + c4 + 4][bc]));
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int col = j0 + nt * 8 + 2 * c4;
+                AX[i0 + g8][col] = -x[nt][0];
+                AX[i0 + g8][col + 1] = -x[nt][1];
+                AX[i0 + g8 + 8][col] = -x[nt][2];
+                AX[i0 + g8 + 8][col + 1] = -x[nt][3];
+            }
+        }
+        if (warp < 4) {
+            named_sync<128>(1);  // warps 0..3 only: the others go on to the next CTA barrier
+            // columns 8 ct .. 8 ct + 7 of X_BA; T = A_BA X_AA is staged where X_BA goes
+            // (rows 32.., columns 0..31 of the work matrix, free until now), then overwritten
+            const int ct = warp, cb = 8 * ct;
+            float t[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks < ct) continue;  // X_AA is zero above the diagonal
+                const int ac = 8 * ks + c4;
+                const float x0 = cb + g8 > ac ? 0.f : AX[ac][cb + g8];
+                const float x1 = cb + g8 > ac + 4 ? 0.f : AX[ac + 4][cb + g8];
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    const int rr = 32 + 16 * rt + g8;
+                    const uint32_t a[4] = {tf32(AX[ac][rr]), tf32(AX[ac][rr + 8]), tf32(AX[ac + 4][rr]),
+                                           tf32(AX[ac + 4][rr + 8])};
+                    mma_tf32(t[rt], a, tf32(x0), tf32(x1));
+                }
+            }
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt) {
+                const int rr = 32 + 16 * rt + g8;
+                AX[rr][cb + 2 * c4] = t[rt][0];
+                AX[rr][cb + 2 * c4 + 1] = t[rt][1];
+                AX[rr + 8][cb + 2 * c4] = t[rt][2];
+                AX[rr + 8][cb + 2 * c4 + 1] = t[rt][3];
+            }
+            __syncwarp();
+            // every row of this strip of T is read before any of it is overwritten
+            uint32_t tb[4][2];
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                tb[ks][0] = tf32(AX[32 + 8 * ks + c4][cb + g8]);
+                tb[ks][1] = tf32(AX[32 + 8 * ks + c4 + 4][cb + g8]);
+            }
+            __syncwarp();
+            float x[2][4] = {};
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt) {
+                const int ra = 16 * rt + g8, rb = ra + 8;  // rows of X_BB (offset 32)
+#pragma unroll
+                for (int ks = 0; ks < 2 + 2 * rt; ++ks) {
+                    const int ac = 8 * ks + c4;  // columns of X_BB (offset 32): zero above the diagonal
+                    const uint32_t a[4] = {tf32(ac > ra ? 0.f : AX[32 + ra][32 + ac]),
+                                           tf32(ac > rb ? 0.f : AX[32 + rb][32 + ac]),
+                                           tf32(ac + 4 > ra ? 0.f : AX[32 + ra][32 + ac + 4]),
+                                           tf32(ac + 4 > rb ? 0.f : AX[32 + rb][32 + ac + 4])};
+                    mma_tf32(x[rt], a, tb[ks][0], tb[ks][1]);
+                }
+            }
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt) {
+                const int rr = 32 + 16 * rt + g8;
+                AX[rr][cb + 2 * c4] = -x[rt][0];
+                AX[rr][cb + 2 * c4 + 1] = -x[rt][1];
+                AX[rr + 8][cb + 2 * c4] = -x[rt][2];
+                AX[rr + 8][cb + 2 * c4 + 1] = -x[rt][3];
+            }
         }
         __syncthreads();
-        // ---- off-diagonal blocks, one block diagonal at a time:
-        //      X_ij = -X_ii sum_{m=j}^{i-1} A_im X_mj  (16 x 16 x 16 products on tf32 MMAs)
-        for (int lvl = 1; lvl < 4; ++lvl) {
-            if (warp < 4 - lvl) {
-                const int i = lvl + warp, j = warp;
-                float t[2][4] = {};
-                for (int m = j; m < i; ++m) {
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        const int ac = m * 16 + kk * 8 + c4;
-                        // A_{i,m} (below the diagonal) is stored transposed
-                        const uint32_t a[4] = {tf32(AX[ac][i * 16 + g8]), tf32(AX[ac][i * 16 + g8 + 8]),
-                                               tf32(AX[ac + 4][i * 16 + g8]), tf32(AX[ac + 4][i * 16 + g8 + 8])};
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const int bc = j * 16 + nt * 8 + g8;
-                            // X_mj; in a diagonal block (m == j) the entries above the diagonal are zero
-                            const int rr0 = m * 16 + kk * 8 + c4, rr1 = rr0 + 4;
-                            const float x0 = (m == j && bc > rr0) ? 0.f : AX[rr0][bc];
-                            const float x1 = (m == j && bc > rr1) ? 0.f : AX[rr1][bc];
-                            mma_tf32(t[nt], a, tf32(x0), tf32(x1));
-                        }
-                    }
-                }
-                float(*Tw)[17] = T[warp];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int col = nt * 8 + 2 * c4;
-                    Tw[g8][col] = t[nt][0];
-                    Tw[g8][col + 1] = t[nt][1];
-                    Tw[g8 + 8][col] = t[nt][2];
-                    Tw[g8 + 8][col + 1] = t[nt][3];
-                }
-                __syncwarp();
-                float x[2][4] = {};
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const int ac = i * 16 + kk * 8 + c4;
-                    // X_ii: zero above the diagonal (A lies there)
-                    const int ra = i * 16 + g8, rb = ra + 8;
-                    const uint32_t a[4] = {tf32(ac > ra ? 0.f : AX[ra][ac]), tf32(ac > rb ? 0.f : AX[rb][ac]),
-                                           tf32(ac + 4 > ra ? 0.f : AX[ra][ac + 4]), tf32(ac + 4 > rb ? 0.f : AX[rb][ac + 4])};
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int bc = nt * 8 + g8;
-                        mma_tf32(x[nt], a, tf32(Tw[kk * 8 + c4][bc]), tf32(Tw[kk * 8 + c4 + 4][bc]));
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const int col = j * 16 + nt * 8 + 2 * c4;
-                    AX[i * 16 + g8][col] = -x[nt][0];
-                    AX[i * 16 + g8][col + 1] = -x[nt][1];
-                    AX[i * 16 + g8 + 8][col] = -x[nt][2];
-                    AX[i * 16 + g8 + 8][col + 1] = -x[nt][3];
-                }
-            }
-            __syncthreads();
-        }
         // ---- Ainv diag(beta), Ainv diag(beta e^gamma) -> 128-byte-swizzled bf16 tiles
         //      (the K-major A operands of the u and w products); Ainv -> global (optional)
         for (int e = tid; e < C * C / 2; e += kThreads) {
@@ -437,7 +515,10 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         ok = ok && cta_wait(mma_bar, mma_phase & 1);
         if (ok) ++mma_phase, mma_pending = false;
         tc_fence_after();
-        if (ok && tid == 0 && gi + 1 < G) load_v(h + 1);  // the v tile is free again
+        if (ok && gi + 1 < G) {  // the v tile is free again
+            if (tid == 0) load_v(h + 1);
+            tma_pending = true;
+        }
         const bool full = len == C;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // columns 64 wn + 32 part .. +31, 16 values at a time
