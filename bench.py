@@ -198,7 +198,7 @@ NCU_TRAFFIC = {
                sha256="4ab2d3258a8acfdbe40dd99c74f8e65bf27fc06b7a8ca712f094ffff60d52952"),
     "prep3": dict(workload="qwen_prefill_t8192_hv32", step="fwd+bwd", bytes=186969600 + 213129728,
                sources=["gdn_prep3.cu"],
-               sha256="06dfdcce0e07ca0da55ba6669fb36d63a66499bff5ae4e86585fb2109c8e3712"),
+               sha256="819efa9638fb9f2e4f6b742e8ce3fa0267571cb8821d0db411dbdbeae9f90202"),
     "recurrent": dict(workload="decode_b256_hv32", step="decode", bytes=549415168 + 481711104,
                sources=["gdn_recurrent.cu"],
                sha256="35e113de4eda5533922853cf613728b9b8d8c372c9964fd87946edc0413bf6a2"),

@@ -332,7 +332,8 @@ prep3_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         //      off-diagonal 16 x 16 block X_10 = -X_11 (A_10 X_00) on tf32 MMAs;
         //  (2) warps 0..3, one 8-column strip each: X_BA = -X_BB (A_BA X_AA) on the 32 x 32
         //      blocks (A = rows and columns 0..31, B = 32..63).
-        //  Warps 4..7 take no part: three of them issue the copies of the next tiles meanwhile.
+        //  Warps 4..7 take no part; during the item's first value head, three of them issue
+        //  the copies of the next tiles meanwhile.
         if (gi == 0 && ok) {
             if (tid == kThreads - 32) load_v(hq * G);
             tma_pending = true;
